@@ -1,0 +1,275 @@
+"""Plain fp64 CPU oracle of the MC-Sparse (Meta-Cached Sparse Attention) hot path.
+
+TEST INFRASTRUCTURE ONLY.  Only the tests, ``__graft_entry__.smoke()`` and the
+CPU-baseline leg of ``bench.py`` may import this module.  The library's product
+path never calls it, and this module imports nothing from the library: the two
+share no code.  Inputs are bf16 bit patterns widened exactly to float64.
+
+Sources (web pages describing the method; cited by title and section):
+
+* [abstract] aiqbench.com, "MC-Sparse: Deconstructing and Closing the Dense-
+  Sparse Attention Gap in Diffusion Transformers", the arXiv abstract.
+* [p1-mcs] cnshai.top, "output-aware sparse attention / KV cache" post,
+  section "MC-Sparse: three failure modes, one fix".
+* [p1-trips] same post, section "What Trips People Up".
+* [p4-design] cctest.ai, "MC-Sparse Narrows the Dense-Sparse Attention Gap in
+  Diffusion Transformers", the list of three design choices.
+
+What the pages fix: KV tokens are selected individually using exact attention
+probabilities; similar queries are organised into tile-aligned groups; the
+cached metadata are the query groups, the KV indices and the residual between
+dense and sparse attention outputs, reused on later denoising steps
+([abstract]; [p1-mcs]; [p4-design]).  Renormalising over the kept tokens is
+not the dense result, which is why the residual is cached ([p1-trips]).
+
+Readings taken where the pages are silent (each listed in the design notes):
+
+* grouping: centre Q, take the eigenvector of the largest eigenvalue of the
+  centred covariance (sign: its largest-magnitude component, lowest index on
+  ties, is positive), project, stable ascending sort; groups are contiguous
+  runs of G in that order, the last one partial.
+* per-group score of key j: the sum over the group's queries of the exact
+  softmax probability P_ij; keep the k' = min(k, N) largest, ties to the
+  lower key index, stored ascending.
+* sparse output: softmax renormalised over the kept keys; residual
+  R_i = O_dense_i - O_sparse_i in the original token order; a reused step
+  outputs O_sparse(current Q, K, V; cached groups and indices) + cached R.
+
+Every function here is pinned by CPU tests against closed forms, brute force,
+invariants or independent textbook routines; none is "parity unpinned".
+"""
+from __future__ import annotations
+
+import numpy as np
+
+__all__ = [
+    "widen_bf16", "principal_direction", "projections", "group_queries",
+    "group_rows", "scores", "row_stats", "probabilities", "group_prob_sums",
+    "select_kv", "dense_rows", "dense_attention", "sparse_group",
+    "sparse_attention", "residual_group", "plan_head", "reused_step_head",
+]
+
+
+def widen_bf16(u16: np.ndarray) -> np.ndarray:
+    """bf16 bit patterns (uint16) -> float64, exactly."""
+    u = np.asarray(u16, dtype=np.uint16)
+    return (u.astype(np.uint32) << np.uint32(16)).view(np.float32).astype(np.float64)
+
+
+def _as_f64(x) -> np.ndarray:
+    x = np.asarray(x)
+    if x.dtype == np.uint16:
+        return widen_bf16(x)
+    return x.astype(np.float64, copy=False)
+
+
+# ---------------------------------------------------------------------------
+# a1. Tile-aligned grouping of similar queries  ([abstract]; [p4-design]
+#     "Hardware-aware query organization")
+# ---------------------------------------------------------------------------
+
+def principal_direction(Q):
+    """Centre, covariance, top eigenpair of one head's queries.
+
+    Returns (mu [d], C [d,d], v [d], eigenvalues ascending [d]).  v is the unit
+    eigenvector of the largest eigenvalue, its sign fixed so that the first
+    component of largest magnitude is positive.
+    """
+    Q = _as_f64(Q)
+    n = Q.shape[0]
+    mu = Q.mean(axis=0)
+    X = Q - mu
+    C = (X.T @ X) / n
+    lam, U = np.linalg.eigh(C)
+    v = U[:, -1].copy()
+    i = int(np.argmax(np.abs(v)))
+    if v[i] < 0:
+        v = -v
+    return mu, C, v, lam
+
+
+def projections(Q, mu, v) -> np.ndarray:
+    """p_n = (Q_n - mu) . v"""
+    return (_as_f64(Q) - mu) @ v
+
+
+def group_queries(Q) -> np.ndarray:
+    """Query order perm (int64 [N]): stable ascending sort of the projections
+    on the first principal direction.  Group g is perm[g*G : (g+1)*G]."""
+    mu, _, v, _ = principal_direction(Q)
+    p = projections(Q, mu, v)
+    return np.argsort(p, kind="stable")
+
+
+def group_rows(perm: np.ndarray, G: int, g: int) -> np.ndarray:
+    return np.asarray(perm)[g * G:(g + 1) * G]
+
+
+# ---------------------------------------------------------------------------
+# a2. Exact attention probabilities  ([abstract] "KV indices selected using
+#     exact attention probabilities"; [p4-design] "Individual KV selection")
+# ---------------------------------------------------------------------------
+
+def scores(Qrows, K, scale: float) -> np.ndarray:
+    """s_ij = scale * Q_i . K_j"""
+    return scale * (_as_f64(Qrows) @ _as_f64(K).T)
+
+
+def row_stats(Qrows, K, scale: float):
+    """m_i = max_j s_ij, l_i = sum_j exp(s_ij - m_i) over all N keys."""
+    S = scores(Qrows, K, scale)
+    m = S.max(axis=1)
+    l = np.exp(S - m[:, None]).sum(axis=1)
+    return m, l
+
+
+def probabilities(Qrows, K, scale: float) -> np.ndarray:
+    """P_ij = exp(s_ij - m_i) / l_i, the dense softmax rows."""
+    S = scores(Qrows, K, scale)
+    E = np.exp(S - S.max(axis=1, keepdims=True))
+    return E / E.sum(axis=1, keepdims=True)
+
+
+# ---------------------------------------------------------------------------
+# a3 / a4. Per-group selection of individual KV tokens
+# ---------------------------------------------------------------------------
+
+def group_prob_sums(Q, K, scale: float, perm, G: int, groups=None) -> np.ndarray:
+    """c[g, j] = sum over queries i of group g of P_ij.  [len(groups), N]"""
+    Q = _as_f64(Q)
+    K = _as_f64(K)
+    n = Q.shape[0]
+    ng = -(-n // G)
+    groups = range(ng) if groups is None else groups
+    out = np.empty((len(groups), K.shape[0]))
+    for r, g in enumerate(groups):
+        rows = group_rows(perm, G, g)
+        out[r] = probabilities(Q[rows], K, scale).sum(axis=0)
+    return out
+
+
+def select_kv(c: np.ndarray, k: int) -> np.ndarray:
+    """Indices of the k' = min(k, N) largest entries of one group's score row,
+    ties resolved towards the lower key index, returned ascending."""
+    c = np.asarray(c, dtype=np.float64)
+    n = c.shape[0]
+    kk = min(int(k), n)
+    order = np.lexsort((np.arange(n), -c))       # primary: -c, secondary: index
+    return np.sort(order[:kk])
+
+
+# ---------------------------------------------------------------------------
+# a5 / a6 / a7. Dense output, renormalised sparse output, residual
+#     ([abstract] "residuals between dense and sparse attention outputs";
+#      [p1-trips] renormalising over the survivors is not a correction)
+# ---------------------------------------------------------------------------
+
+def dense_rows(Qrows, K, V, scale: float) -> np.ndarray:
+    """O_i = sum_j P_ij V_j for the given query rows."""
+    return probabilities(Qrows, K, scale) @ _as_f64(V)
+
+
+def dense_attention(Q, K, V, scale: float, block: int = 0) -> np.ndarray:
+    """Dense softmax(scale Q K^T) V of one head, query rows in blocks."""
+    Q = _as_f64(Q)
+    K = _as_f64(K)
+    V = _as_f64(V)
+    n = Q.shape[0]
+    if block <= 0:
+        block = max(16, min(1024, (1 << 26) // max(1, K.shape[0])))
+    out = np.empty((n, V.shape[1]))
+    for s in range(0, n, block):
+        out[s:s + block] = dense_rows(Q[s:s + block], K, V, scale)
+    return out
+
+
+def sparse_group(Qrows, K, V, scale: float, idx) -> np.ndarray:
+    """O_sp_i = sum_{j in S} exp(s_ij) V_j / sum_{j in S} exp(s_ij), softmax
+    renormalised over the kept keys S only."""
+    idx = np.asarray(idx)
+    Ks = _as_f64(K)[idx]
+    Vs = _as_f64(V)[idx]
+    S = scores(Qrows, Ks, scale)
+    E = np.exp(S - S.max(axis=1, keepdims=True))
+    return (E / E.sum(axis=1, keepdims=True)) @ Vs
+
+
+def sparse_attention(Q, K, V, scale: float, perm, kv_idx, G: int, groups=None):
+    """Renormalised sparse output in original token order.  With `groups`
+    given, returns (rows, O_sp[rows]) for those groups only."""
+    Q = _as_f64(Q)
+    n, d = Q.shape[0], _as_f64(V).shape[1]
+    ng = -(-n // G)
+    sel = range(ng) if groups is None else groups
+    if groups is None:
+        out = np.empty((n, d))
+        for g in sel:
+            rows = group_rows(perm, G, g)
+            out[rows] = sparse_group(Q[rows], K, V, scale, kv_idx[g])
+        return out
+    rows_all, vals = [], []
+    for g in sel:
+        rows = group_rows(perm, G, g)
+        rows_all.append(rows)
+        vals.append(sparse_group(Q[rows], K, V, scale, kv_idx[g]))
+    return np.concatenate(rows_all), np.concatenate(vals)
+
+
+def residual_group(Qrows, K, V, scale: float, idx):
+    """Residual of one group's rows, computed two ways.
+
+    R = O_dense - O_sp (the definition), and R_alt = U - (1 - alpha) O_sp with
+    U_i = sum_{j not in S} P_ij V_j and alpha_i = sum_{j in S} P_ij (the mass
+    the kept keys hold under the dense softmax).  Returns (R, R_alt, alpha).
+    """
+    P = probabilities(Qrows, K, scale)
+    Vf = _as_f64(V)
+    O_dense = P @ Vf
+    O_sp = sparse_group(Qrows, K, V, scale, idx)
+    mask = np.zeros(P.shape[1], dtype=bool)
+    mask[np.asarray(idx)] = True
+    alpha = P[:, mask].sum(axis=1)
+    U = P[:, ~mask] @ Vf[~mask]
+    R = O_dense - O_sp
+    R_alt = U - (1.0 - alpha)[:, None] * O_sp
+    return R, R_alt, alpha
+
+
+def plan_head(Q, K, V, G: int, k: int, scale: float):
+    """The metadata pass of one head.
+
+    Returns dict(perm int64 [N], kv_idx int64 [n_groups, k'], residual
+    float64 [N, d] in original token order, O_dense float64 [N, d]).
+    """
+    Q = _as_f64(Q)
+    K = _as_f64(K)
+    V = _as_f64(V)
+    n = Q.shape[0]
+    d = V.shape[1]
+    ng = -(-n // G)
+    kk = min(int(k), n)
+    perm = group_queries(Q)
+    kv_idx = np.empty((ng, kk), dtype=np.int64)
+    residual = np.empty((n, d))
+    O_dense = np.empty((n, d))
+    Vf = V
+    for g in range(ng):
+        rows = group_rows(perm, G, g)
+        P = probabilities(Q[rows], K, scale)
+        idx = select_kv(P.sum(axis=0), kk)
+        kv_idx[g] = idx
+        Od = P @ Vf
+        Osp = sparse_group(Q[rows], K, V, scale, idx)
+        O_dense[rows] = Od
+        residual[rows] = Od - Osp
+    return {"perm": perm, "kv_idx": kv_idx, "residual": residual, "O_dense": O_dense}
+
+
+def reused_step_head(Q, K, V, scale: float, perm, kv_idx, residual, G: int, groups=None):
+    """Reused denoising step: O_i = O_sp_i(current Q, K, V; cached groups and
+    indices) + cached R_i.  With `groups`, returns (rows, O[rows])."""
+    residual = np.asarray(residual, dtype=np.float64)
+    if groups is None:
+        return sparse_attention(Q, K, V, scale, perm, kv_idx, G) + residual
+    rows, osp = sparse_attention(Q, K, V, scale, perm, kv_idx, G, groups=groups)
+    return rows, osp + residual[rows]
