@@ -1,0 +1,176 @@
+/*
+ * mcs.h -- C ABI of the MC-Sparse (Meta-Cached Sparse Attention) hot path on
+ * NVIDIA B200 (sm_100a).
+ *
+ * The method (aiqbench.com, "MC-Sparse: Deconstructing and Closing the
+ * Dense-Sparse Attention Gap in Diffusion Transformers", abstract; cctest.ai,
+ * "MC-Sparse Narrows the Dense-Sparse Attention Gap in Diffusion
+ * Transformers", design choices): a metadata pass computes exact dense
+ * attention probabilities, organises similar queries into tile-aligned
+ * groups, selects individual KV tokens per group from those probabilities and
+ * caches the residual between dense and sparse outputs; later denoising steps
+ * reuse the groups, indices and residual.
+ *
+ * Conventions for every entry point
+ *   - Q, K, V, O: bf16, layout [B, H, N, d], contiguous (d fastest), in
+ *     device memory, 16-byte aligned.  d is 64 or 128.
+ *   - scale: softmax scale applied to Q.K (usually 1/sqrt(d)).
+ *   - All device buffers are owned by the caller.  The library allocates no
+ *     device memory and keeps no per-call state.
+ *   - Calls are asynchronous on `stream` (a cudaStream_t; NULL = the legacy
+ *     default stream).  Argument errors are detected on the host before any
+ *     launch and returned synchronously; nothing is launched then.
+ *   - A launch failure returns MCS_ERR_CUDA.  Errors the device detects (a
+ *     bounded wait that ran out) are recorded in a per-device status word
+ *     that mcs_last_device_status() reads; kernels never trap.
+ *   - Query groups: perm[b,h,:] is a permutation of 0..N-1; group g of head
+ *     (b,h) is the queries perm[b,h,g*G .. min((g+1)*G, N)-1]; the last group
+ *     may be partial.  n_groups = ceil(N / G).
+ *   - KV indices: kv_idx[b,h,g,0..k'-1] with k' = min(k, N): unique,
+ *     strictly ascending, in [0, N).
+ *   - Residual: float32 [B, H, N, d] in the original token order.
+ */
+#ifndef MCS_H_
+#define MCS_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#define MCS_ABI_VERSION 1
+
+typedef struct CUstream_st *mcs_stream_t; /* same type as cudaStream_t */
+
+typedef enum {
+  MCS_OK = 0,
+  MCS_ERR_INVALID_ARG = 1,  /* null pointer, bad size, misaligned pointer   */
+  MCS_ERR_UNSUPPORTED = 2,  /* d or G outside the supported set            */
+  MCS_ERR_WORKSPACE = 3,    /* workspace missing or smaller than required  */
+  MCS_ERR_CUDA = 4,         /* a CUDA runtime call or launch failed        */
+  MCS_ERR_TIMEOUT = 5,      /* a bounded device wait ran out               */
+  MCS_ERR_BAD_META = 6      /* metadata failed validation                  */
+} mcs_status;
+
+/* Cached metadata of one plan ("query groups, KV indices ... and residuals",
+ * aiqbench.com abstract).  All pointers are caller-owned device memory. */
+typedef struct {
+  int32_t B, H, N, d, G, k, n_groups; /* k is stored clamped: k = min(k, N) */
+  int32_t *perm;                      /* [B,H,N]                           */
+  int32_t *kv_idx;                    /* [B,H,n_groups,k]                  */
+  float *residual;                    /* [B,H,N,d]                         */
+} mcs_meta;
+
+/* Library ABI version (MCS_ABI_VERSION of the build). */
+int mcs_abi_version(void);
+
+/* Human-readable name of a status code (static string, never NULL). */
+const char *mcs_status_string(mcs_status s);
+
+/* Fill in the scalar fields of `meta` (B, H, N, d, G, k clamped to N,
+ * n_groups) and check them.  Pointers are left untouched. */
+mcs_status mcs_meta_init(mcs_meta *meta, int B, int H, int N, int d, int G, int k);
+
+/* Bytes of workspace mcs_plan and its stages need for this shape; 0 when the
+ * shape is invalid.  The workspace must be 256-byte aligned device memory. */
+size_t mcs_plan_workspace_size(int B, int H, int N, int d, int G, int k);
+
+/*
+ * mcs_plan -- the metadata pass: steps a1..a5 of the hot path.
+ *   a1 grouping: per (b,h), centre Q, take the top principal direction of its
+ *      covariance, sort the projections ascending (stable) -> perm.
+ *   a2 exact probabilities: row max and sum of exp over all N keys, and the
+ *      dense output (fp32, split-precision P.V).
+ *   a3 group scores: colsum[g, j] = sum_{i in g} P_ij.
+ *   a4 selection: per group the k' largest scores, ties to the lower index,
+ *      stored ascending -> kv_idx.
+ *   a5 residual: R = O_dense - O_sparse, O_sparse renormalised over the kept
+ *      keys -> residual.
+ * Sources: aiqbench.com abstract ("KV indices selected using exact attention
+ * probabilities", "residuals between dense and sparse attention outputs");
+ * cnshai.top "output-aware sparse attention / KV cache", section "MC-Sparse:
+ * three failure modes, one fix"; cctest.ai design choices.
+ *
+ * meta: scalar fields are set by this call; meta->perm, ->kv_idx and
+ *   ->residual must point to caller buffers of the sizes given above.
+ * O_dense: optional bf16 [B,H,N,d] output of the dense attention of this step
+ *   (what a plan step of the denoising loop produces); may be NULL.
+ * workspace: >= mcs_plan_workspace_size(...) bytes of device memory.
+ */
+mcs_status mcs_plan(const void *Q, const void *K, const void *V, int B, int H, int N, int d,
+                    int G, int k, float scale, mcs_meta *meta, void *O_dense, void *workspace,
+                    size_t workspace_bytes, mcs_stream_t stream);
+
+/* Step a1 alone: perm int32 [B,H,N].  Same workspace as mcs_plan. */
+mcs_status mcs_plan_group(const void *Q, int B, int H, int N, int d, int32_t *perm,
+                          void *workspace, size_t workspace_bytes, mcs_stream_t stream);
+
+/* Steps a2..a4 for a given grouping `perm` (any permutation): kv_idx int32
+ * [B,H,ceil(N/G),min(k,N)].  Same workspace as mcs_plan. */
+mcs_status mcs_plan_select(const void *Q, const void *K, const int32_t *perm, int B, int H,
+                           int N, int d, int G, int k, float scale, int32_t *kv_idx,
+                           void *workspace, size_t workspace_bytes, mcs_stream_t stream);
+
+/* Steps a2 and a5 for a given grouping and selection: residual float32
+ * [B,H,N,d]; O_dense (bf16, optional) as in mcs_plan.  Same workspace. */
+mcs_status mcs_plan_residual(const void *Q, const void *K, const void *V, const int32_t *perm,
+                             const int32_t *kv_idx, int B, int H, int N, int d, int G, int k,
+                             float scale, float *residual, void *O_dense, void *workspace,
+                             size_t workspace_bytes, mcs_stream_t stream);
+
+/*
+ * mcs_sparse_step -- step a6, the reused denoising step: for every group g,
+ *   O_i = sum_{j in S_g} softmax_j(scale Q_i.K_j) V_j + R_i   (i in g)
+ * on the current step's Q, K, V with the cached groups, indices and residual
+ * (aiqbench.com abstract: metadata "reused across subsequent denoising
+ * steps"; cnshai.top section "MC-Sparse: three failure modes, one fix").
+ * O: bf16 [B,H,N,d], original token order.  Needs no workspace.
+ */
+mcs_status mcs_sparse_step(const void *Q, const void *K, const void *V, const mcs_meta *meta,
+                           float scale, void *O, mcs_stream_t stream);
+
+/*
+ * mcs_dense -- step a7, dense attention O = softmax(scale Q K^T) V, the
+ * comparison baseline the pages measure against ("relative to dense
+ * attention", aiqbench.com abstract).  O: bf16 [B,H,N,d].
+ */
+mcs_status mcs_dense(const void *Q, const void *K, const void *V, int B, int H, int N, int d,
+                     float scale, void *O, mcs_stream_t stream);
+
+/* Bytes of workspace mcs_validate_meta needs (one byte per token). */
+size_t mcs_validate_workspace_size(int B, int H, int N);
+
+/*
+ * Check cached metadata on the device: perm is a permutation per head,
+ * kv_idx entries are in [0, N) and strictly ascending per group, the
+ * residual is finite.  Synchronous: waits for `stream`.  Returns MCS_OK or
+ * MCS_ERR_BAD_META; *first_bad (may be NULL) receives a code of the first
+ * failed check: 1 perm, 2 kv_idx range, 3 kv_idx order, 4 residual.
+ * Never traps.
+ */
+mcs_status mcs_validate_meta(const mcs_meta *meta, void *workspace, size_t workspace_bytes,
+                             int *first_bad, mcs_stream_t stream);
+
+/* Synchronise `stream`, then read and clear this device's status word.
+ * Returns MCS_OK, or MCS_ERR_TIMEOUT if a kernel's bounded wait ran out
+ * since the last read. */
+mcs_status mcs_last_device_status(mcs_stream_t stream);
+
+/* Self-test of the bounded device wait: launches one kernel that waits on an
+ * mbarrier nothing ever arrives on; after `limit_ns` (0 = 1 ms) it gives up,
+ * records MCS_ERR_TIMEOUT in the status word and returns normally, leaving
+ * the context usable.  Asynchronous; read the outcome with
+ * mcs_last_device_status(). */
+mcs_status mcs_selftest_wait_timeout(uint64_t limit_ns, mcs_stream_t stream);
+
+/* Upper bound, in nanoseconds, on any single wait inside the kernels
+ * (default 4e9).  A kernel whose wait runs out records MCS_ERR_TIMEOUT and
+ * returns cleanly.  0 restores the default. */
+void mcs_set_wait_limit_ns(uint64_t ns);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* MCS_H_ */

@@ -1,0 +1,21 @@
+"""MC-Sparse (Meta-Cached Sparse Attention) hot path for NVIDIA B200 (sm_100a).
+
+The CUDA library (libmcs.so, C ABI in include/mcs.h) does all the work; this
+package is its Python binding.  Import is cheap: the library is loaded on the
+first call.
+"""
+from .api import (  # noqa: F401
+    Meta,
+    alloc_workspace,
+    dense,
+    last_device_status,
+    plan,
+    plan_group,
+    plan_residual,
+    plan_select,
+    selftest_wait_timeout,
+    set_wait_limit_ns,
+    sparse_step,
+    validate_meta,
+    workspace_size,
+)

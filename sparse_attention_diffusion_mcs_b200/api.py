@@ -1,0 +1,198 @@
+"""Torch-facing binding of the MC-Sparse C ABI.
+
+Argument marshalling only: every step of the hot path runs in the CUDA
+library.  Tensors must be CUDA, contiguous; Q/K/V/O are bf16 [B, H, N, d].
+Calls are asynchronous on torch's current stream.
+"""
+from __future__ import annotations
+
+import ctypes
+import dataclasses
+import math
+from typing import Optional, Tuple
+
+import torch
+
+from ._lib import McsMeta, check, lib
+
+
+def _ptr(t: Optional[torch.Tensor]):
+    return ctypes.c_void_p(t.data_ptr()) if t is not None else ctypes.c_void_p(0)
+
+
+def _stream():
+    return ctypes.c_void_p(torch.cuda.current_stream().cuda_stream)
+
+
+def _check_qkv(*ts: torch.Tensor):
+    for t in ts:
+        if not (t.is_cuda and t.dtype == torch.bfloat16 and t.is_contiguous() and t.dim() == 4):
+            raise ValueError("Q/K/V must be contiguous CUDA bf16 tensors [B, H, N, d]")
+    if any(t.shape != ts[0].shape for t in ts):
+        raise ValueError("Q/K/V shapes differ")
+
+
+def _scale(d: int, scale: Optional[float]) -> float:
+    return float(scale) if scale is not None else 1.0 / math.sqrt(d)
+
+
+@dataclasses.dataclass
+class Meta:
+    """Cached metadata of a plan: query order, KV indices, residual."""
+    B: int
+    H: int
+    N: int
+    d: int
+    G: int
+    k: int
+    n_groups: int
+    perm: torch.Tensor       # int32 [B, H, N]
+    kv_idx: torch.Tensor     # int32 [B, H, n_groups, k]
+    residual: torch.Tensor   # float32 [B, H, N, d]
+
+    def c_struct(self) -> McsMeta:
+        return McsMeta(self.B, self.H, self.N, self.d, self.G, self.k, self.n_groups,
+                       self.perm.data_ptr(), self.kv_idx.data_ptr(), self.residual.data_ptr())
+
+    @staticmethod
+    def empty(B: int, H: int, N: int, d: int, G: int, k: int, device="cuda") -> "Meta":
+        k = min(int(k), N)
+        ng = -(-N // G)
+        return Meta(B, H, N, d, G, k, ng,
+                    torch.empty((B, H, N), dtype=torch.int32, device=device),
+                    torch.empty((B, H, ng, k), dtype=torch.int32, device=device),
+                    torch.empty((B, H, N, d), dtype=torch.float32, device=device))
+
+    @staticmethod
+    def from_tensors(perm, kv_idx, residual, G: int) -> "Meta":
+        B, H, N, d = residual.shape
+        ng, k = kv_idx.shape[2], kv_idx.shape[3]
+        return Meta(B, H, N, d, G, k, ng, perm.contiguous(), kv_idx.contiguous(),
+                    residual.contiguous())
+
+
+def workspace_size(B: int, H: int, N: int, d: int, G: int, k: int) -> int:
+    n = lib().mcs_plan_workspace_size(B, H, N, d, G, k)
+    if n == 0:
+        raise ValueError("unsupported shape")
+    return int(n)
+
+
+def alloc_workspace(B: int, H: int, N: int, d: int, G: int, k: int, device="cuda") -> torch.Tensor:
+    # torch's caching allocator returns 512-byte aligned blocks
+    return torch.empty(workspace_size(B, H, N, d, G, k), dtype=torch.uint8, device=device)
+
+
+def _ws(ws: Optional[torch.Tensor], B, H, N, d, G, k, device):
+    if ws is None:
+        ws = alloc_workspace(B, H, N, d, G, k, device)
+    return ws
+
+
+def plan(Q, K, V, G: int, k: int, scale: Optional[float] = None,
+         workspace: Optional[torch.Tensor] = None, meta: Optional[Meta] = None,
+         out_dense: Optional[torch.Tensor] = None, return_dense: bool = False):
+    """Metadata pass (steps a1-a5).  Returns Meta, or (Meta, O_dense bf16)."""
+    _check_qkv(Q, K, V)
+    B, H, N, d = Q.shape
+    if meta is None:
+        meta = Meta.empty(B, H, N, d, G, k, Q.device)
+    if return_dense and out_dense is None:
+        out_dense = torch.empty_like(Q)
+    ws = _ws(workspace, B, H, N, d, G, k, Q.device)
+    cm = meta.c_struct()
+    check(lib().mcs_plan(_ptr(Q), _ptr(K), _ptr(V), B, H, N, d, G, k, _scale(d, scale),
+                         ctypes.byref(cm), _ptr(out_dense), _ptr(ws), ws.numel(), _stream()),
+          "mcs_plan")
+    meta.k, meta.n_groups = cm.k, cm.n_groups
+    return (meta, out_dense) if (return_dense or out_dense is not None) else meta
+
+
+def plan_group(Q, workspace: Optional[torch.Tensor] = None) -> torch.Tensor:
+    """Step a1 alone: int32 perm [B, H, N]."""
+    _check_qkv(Q)
+    B, H, N, d = Q.shape
+    perm = torch.empty((B, H, N), dtype=torch.int32, device=Q.device)
+    ws = _ws(workspace, B, H, N, d, 128, 1, Q.device)
+    check(lib().mcs_plan_group(_ptr(Q), B, H, N, d, _ptr(perm), _ptr(ws), ws.numel(), _stream()),
+          "mcs_plan_group")
+    return perm
+
+
+def plan_select(Q, K, perm, G: int, k: int, scale: Optional[float] = None,
+                workspace: Optional[torch.Tensor] = None) -> torch.Tensor:
+    """Steps a2-a4 for a given grouping: int32 kv_idx [B, H, n_groups, min(k, N)]."""
+    _check_qkv(Q, K)
+    B, H, N, d = Q.shape
+    perm = perm.to(torch.int32).contiguous()
+    kk = min(int(k), N)
+    kv = torch.empty((B, H, -(-N // G), kk), dtype=torch.int32, device=Q.device)
+    ws = _ws(workspace, B, H, N, d, G, k, Q.device)
+    check(lib().mcs_plan_select(_ptr(Q), _ptr(K), _ptr(perm), B, H, N, d, G, k, _scale(d, scale),
+                                _ptr(kv), _ptr(ws), ws.numel(), _stream()), "mcs_plan_select")
+    return kv
+
+
+def plan_residual(Q, K, V, perm, kv_idx, G: int, scale: Optional[float] = None,
+                  workspace: Optional[torch.Tensor] = None, return_dense: bool = False):
+    """Steps a2 and a5 for a given grouping and selection: float32 residual."""
+    _check_qkv(Q, K, V)
+    B, H, N, d = Q.shape
+    perm = perm.to(torch.int32).contiguous()
+    kv_idx = kv_idx.to(torch.int32).contiguous()
+    k = kv_idx.shape[-1]
+    res = torch.empty((B, H, N, d), dtype=torch.float32, device=Q.device)
+    od = torch.empty_like(Q) if return_dense else None
+    ws = _ws(workspace, B, H, N, d, G, k, Q.device)
+    check(lib().mcs_plan_residual(_ptr(Q), _ptr(K), _ptr(V), _ptr(perm), _ptr(kv_idx), B, H, N, d,
+                                  G, k, _scale(d, scale), _ptr(res), _ptr(od), _ptr(ws),
+                                  ws.numel(), _stream()), "mcs_plan_residual")
+    return (res, od) if return_dense else res
+
+
+def sparse_step(Q, K, V, meta: Meta, scale: Optional[float] = None,
+                out: Optional[torch.Tensor] = None) -> torch.Tensor:
+    """Reused denoising step (a6): bf16 O [B, H, N, d]."""
+    _check_qkv(Q, K, V)
+    if out is None:
+        out = torch.empty_like(Q)
+    cm = meta.c_struct()
+    check(lib().mcs_sparse_step(_ptr(Q), _ptr(K), _ptr(V), ctypes.byref(cm),
+                                _scale(meta.d, scale), _ptr(out), _stream()), "mcs_sparse_step")
+    return out
+
+
+def dense(Q, K, V, scale: Optional[float] = None, out: Optional[torch.Tensor] = None) -> torch.Tensor:
+    """Dense attention (a7): bf16 O [B, H, N, d]."""
+    _check_qkv(Q, K, V)
+    B, H, N, d = Q.shape
+    if out is None:
+        out = torch.empty_like(Q)
+    check(lib().mcs_dense(_ptr(Q), _ptr(K), _ptr(V), B, H, N, d, _scale(d, scale), _ptr(out),
+                          _stream()), "mcs_dense")
+    return out
+
+
+def validate_meta(meta: Meta) -> Tuple[bool, int]:
+    """(valid, first failing check code); synchronous."""
+    n = lib().mcs_validate_workspace_size(meta.B, meta.H, meta.N)
+    ws = torch.empty(int(n), dtype=torch.uint8, device=meta.perm.device)
+    code = ctypes.c_int(0)
+    cm = meta.c_struct()
+    st = lib().mcs_validate_meta(ctypes.byref(cm), _ptr(ws), ws.numel(), ctypes.byref(code), _stream())
+    if st == 6:
+        return False, code.value
+    check(st, "mcs_validate_meta")
+    return True, 0
+
+
+def last_device_status() -> int:
+    return int(lib().mcs_last_device_status(_stream()))
+
+
+def set_wait_limit_ns(ns: int) -> None:
+    lib().mcs_set_wait_limit_ns(int(ns))
+
+
+def selftest_wait_timeout(limit_ns: int) -> None:
+    check(lib().mcs_selftest_wait_timeout(int(limit_ns), _stream()), "mcs_selftest_wait_timeout")

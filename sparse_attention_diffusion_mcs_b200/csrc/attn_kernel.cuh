@@ -1,0 +1,454 @@
+// attn_kernel.cuh -- one tcgen05 / TMEM flash-attention kernel, four uses.
+//
+//  kModeDense     O = softmax(scale Q K^T) V over all N keys, bf16 out.  The
+//                 dense baseline of the pages ("relative to dense attention",
+//                 aiqbench.com abstract).
+//  kModeStep      the reused denoising step: each CTA owns one query group
+//                 (rows gathered through perm), attends only to the group's
+//                 cached KV indices (rows gathered through kv_idx), adds the
+//                 cached residual in the epilogue and scatters bf16 rows back
+//                 to the original token order (aiqbench.com abstract: query
+//                 groups, KV indices and residuals "reused across subsequent
+//                 denoising steps"; cnshai.top post, section "MC-Sparse:
+//                 three failure modes, one fix").
+//  kModePlanDense dense pass of the metadata plan: exact row statistics
+//                 (m, l) of the softmax over all keys plus the dense output in
+//                 fp32.  P is split into bf16 hi + lo parts, two MMAs, so the
+//                 fp32 output carries ~2^-17 relative error instead of 2^-9.
+//  kModePlanResid sparse pass of the plan with the same split precision;
+//                 epilogue writes R = O_dense - O_sparse (the cached residual
+//                 "between dense and sparse attention outputs").
+//
+// CTA = 128 query rows x all KV tiles of 128 keys; 224 threads:
+//   warps 0-3  softmax + epilogue; thread t owns query row t = TMEM lane t
+//   warp  4    TMEM allocation and the single UMMA-issuing thread
+//   warps 5-6  gather: cp.async 16-byte vectors into 128B-swizzled tiles
+// TMEM: S double buffer (2 x 128 fp32 columns) + O (D columns).
+// Synchronisation is mbarrier-only inside the loops; every wait is bounded.
+#pragma once
+
+#include "mcs_common.cuh"
+
+namespace mcs {
+
+enum AttnMode : int { kModeDense = 0, kModeStep = 1, kModePlanDense = 2, kModePlanResid = 3 };
+
+struct AttnArgs {
+  const bf16 *Q, *K, *V;   // [BH, N, D]
+  int N;                   // tokens per head
+  int G;                   // query group size (sparse modes)
+  int k;                   // kept keys per group (sparse modes), <= N
+  int n_groups;            // ceil(N / G)
+  float scale_log2;        // softmax scale * log2(e)
+  const int32_t *perm;     // [BH, N]               sparse modes
+  const int32_t *kv_idx;   // [BH, n_groups, k]     sparse modes
+  const float *residual;   // [BH, N, D]            kModeStep
+  bf16 *O;                 // [BH, N, D] bf16 out   dense / step / plan-dense (optional)
+  float *O32;              // [BH, N, D]            kModePlanDense
+  const float *O32_in;     // [BH, N, D]            kModePlanResid
+  float *R_out;            // [BH, N, D]            kModePlanResid
+  float *row_m, *row_l;    // [BH, N]               kModePlanDense (log2 domain)
+  unsigned *status;        // device status word
+  uint64_t wait_ns;        // bound on any single wait
+};
+
+template <int D, int MODE>
+struct AttnCfg {
+  static constexpr int BM = 128, BN = 128;
+  static constexpr bool kSparse = (MODE == kModeStep || MODE == kModePlanResid);
+  static constexpr bool kSplit = (MODE == kModePlanDense || MODE == kModePlanResid);
+  static constexpr int NST = (D == 64) ? 3 : 2;             // K ring and V ring depth
+  static constexpr int Q_BYTES = BM * D * 2;
+  static constexpr int KV_BYTES = BN * D * 2;
+  static constexpr int P_BYTES = BM * BN * 2;
+  static constexpr int OFF_Q = 0;
+  static constexpr int OFF_K = OFF_Q + Q_BYTES;
+  static constexpr int OFF_V = OFF_K + NST * KV_BYTES;
+  static constexpr int OFF_P = OFF_V + NST * KV_BYTES;
+  static constexpr int OFF_BAR = OFF_P + (kSplit ? 2 : 1) * P_BYTES;
+  static constexpr int N_BAR = 1 + 4 * NST + 2 + 3;         // q, k/v full/empty, s_full[2], p, pv, drain
+  static constexpr int OFF_MISC = OFF_BAR + 8 * N_BAR;
+  static constexpr int SMEM = OFF_MISC + 16 + 1024;         // + slack to align the base to 1 KB
+  static constexpr int THREADS = 224;
+  static constexpr uint32_t TMEM_COLS = 512;
+  static constexpr uint32_t COL_S0 = 0, COL_S1 = 128, COL_O = 256;
+};
+
+template <int D, int MODE>
+__global__ void __launch_bounds__(224, 1) attn_kernel(const AttnArgs a) {
+  using C = AttnCfg<D, MODE>;
+  constexpr int BM = C::BM, BN = C::BN, NST = C::NST;
+  constexpr int CPR = D / 8;           // 16-byte chunks per row
+  constexpr int RPP = 64 / CPR;        // rows covered per loader pass (64 loader threads)
+
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                              ~static_cast<uintptr_t>(1023));
+  const uint32_t sbase = smem_u32(smem);
+  const uint32_t sQ = sbase + C::OFF_Q;
+  const uint32_t sK0 = sbase + C::OFF_K;
+  const uint32_t sV0 = sbase + C::OFF_V;
+  const uint32_t sP = sbase + C::OFF_P;
+  const uint32_t bar0 = sbase + C::OFF_BAR;
+  // barrier addresses
+  const uint32_t b_q = bar0;
+  auto b_kfull = [&](int s) { return bar0 + 8 * (1 + s); };
+  auto b_kempty = [&](int s) { return bar0 + 8 * (1 + NST + s); };
+  auto b_vfull = [&](int s) { return bar0 + 8 * (1 + 2 * NST + s); };
+  auto b_vempty = [&](int s) { return bar0 + 8 * (1 + 3 * NST + s); };
+  const uint32_t b_sfull0 = bar0 + 8 * (1 + 4 * NST);
+  const uint32_t b_p = bar0 + 8 * (3 + 4 * NST);
+  const uint32_t b_pv = bar0 + 8 * (4 + 4 * NST);
+  const uint32_t b_drain = bar0 + 8 * (5 + 4 * NST);
+  uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem + C::OFF_MISC);
+  volatile int *abort_flag = reinterpret_cast<volatile int *>(smem + C::OFF_MISC + 4);
+
+  const int tid = threadIdx.x;
+  const int warp = tid >> 5;
+  const int tile = blockIdx.x;          // query tile (dense) or query group (sparse)
+  const int bh = blockIdx.y;
+  const int N = a.N;
+  const size_t head = static_cast<size_t>(bh) * N;
+
+  // number of keys this CTA attends to, and KV tiles
+  const int nkeys = C::kSparse ? a.k : N;
+  const int T = (nkeys + BN - 1) / BN;
+  const int32_t *kv_list =
+      C::kSparse ? a.kv_idx + (static_cast<size_t>(bh) * a.n_groups + tile) * a.k : nullptr;
+
+  // query row r of this tile -> token index, or -1 when the row is padding
+  auto q_token = [&](int r) -> int {
+    if (C::kSparse) {
+      const int gr = tile * a.G + r;
+      if (r >= a.G || gr >= N) return -1;
+      const int q = a.perm[head + gr];
+      if (static_cast<unsigned>(q) >= static_cast<unsigned>(N)) {   // corrupt metadata: never gather out of range
+        record_status(a.status, kStatusBadMeta);
+        return -1;
+      }
+      return q;
+    } else {
+      const int q = tile * BM + r;
+      return q < N ? q : -1;
+    }
+  };
+
+  if (tid == 0) {
+    mbar_init(b_q, 64);
+    for (int s = 0; s < NST; ++s) {
+      mbar_init(b_kfull(s), 64);
+      mbar_init(b_vfull(s), 64);
+      mbar_init(b_kempty(s), 1);
+      mbar_init(b_vempty(s), 1);
+    }
+    mbar_init(b_sfull0, 1);
+    mbar_init(b_sfull0 + 8, 1);
+    mbar_init(b_p, 128);
+    mbar_init(b_pv, 1);
+    mbar_init(b_drain, 1);
+    *abort_flag = 0;
+    mbar_init_fence();
+  }
+  if (warp == 4) {
+    tmem_alloc(smem_u32(tmem_slot), C::TMEM_COLS);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tbase = *tmem_slot;
+
+  if (warp >= 5) {
+    // ------------------------------------------------------------------ gather
+    const int lt = tid - 160;   // 0..63
+    const int c = lt % CPR;
+    const int r0 = lt / CPR;
+    // Q rows (through perm in the sparse modes)
+#pragma unroll 4
+    for (int i = 0; i < 128 / RPP; ++i) {
+      const int r = r0 + i * RPP;
+      const int q = q_token(r);
+      const bf16 *src = q >= 0 ? a.Q + (head + q) * D + c * 8 : a.Q;
+      cp_async16(sQ + sw128_offset(r, c, BM), src, q >= 0 ? 16u : 0u);
+    }
+    cp_async_arrive_noinc(b_q);
+    if (MODE == kModeStep || MODE == kModePlanResid) {
+      // warm L2 with the rows the epilogue will read
+      const float *ep = MODE == kModeStep ? a.residual : a.O32_in;
+      for (int i = lt; i < 128 * (D / 32); i += 64) {
+        const int r = i / (D / 32);
+        const int q = q_token(r);
+        if (q >= 0)
+          asm volatile("prefetch.global.L2 [%0];" ::"l"(ep + (head + q) * D + (i % (D / 32)) * 32));
+      }
+    }
+    bool ok = true;
+    for (int j = 0; j < T && ok; ++j) {
+      const int s = j % NST;
+      const uint32_t ph = (j / NST) & 1;
+      int key[128 / RPP];
+#pragma unroll
+      for (int i = 0; i < 128 / RPP; ++i) {
+        const int pos = j * BN + r0 + i * RPP;
+        key[i] = pos < nkeys ? (C::kSparse ? kv_list[pos] : pos) : -1;
+        if (C::kSparse && key[i] >= N) {   // corrupt metadata: treat as padding, report
+          record_status(a.status, kStatusBadMeta);
+          key[i] = -1;
+        }
+      }
+      if (!mbar_wait(b_kempty(s), ph ^ 1, a.wait_ns, abort_flag)) { ok = false; break; }
+      const uint32_t dK = sK0 + s * C::KV_BYTES;
+#pragma unroll
+      for (int i = 0; i < 128 / RPP; ++i) {
+        const int r = r0 + i * RPP;
+        const bf16 *src = key[i] >= 0 ? a.K + (head + key[i]) * D + c * 8 : a.K;
+        cp_async16(dK + sw128_offset(r, c, BN), src, key[i] >= 0 ? 16u : 0u);
+      }
+      cp_async_arrive_noinc(b_kfull(s));
+      if (!mbar_wait(b_vempty(s), ph ^ 1, a.wait_ns, abort_flag)) { ok = false; break; }
+      const uint32_t dV = sV0 + s * C::KV_BYTES;
+#pragma unroll
+      for (int i = 0; i < 128 / RPP; ++i) {
+        const int r = r0 + i * RPP;
+        const bf16 *src = key[i] >= 0 ? a.V + (head + key[i]) * D + c * 8 : a.V;
+        cp_async16(dV + sw128_offset(r, c, BN), src, key[i] >= 0 ? 16u : 0u);
+      }
+      cp_async_arrive_noinc(b_vfull(s));
+    }
+    if (!ok && !*abort_flag) {
+      *abort_flag = 1;
+      record_status(a.status, kStatusTimeout);
+    }
+    cp_async_wait_all();
+  } else if (warp == 4) {
+    // ------------------------------------------------------------------ UMMA issue
+    if (tid == 128) {
+      constexpr uint32_t idesc_qk = idesc_bf16_f32(BM, BN, 0);
+      constexpr uint32_t idesc_pv = idesc_bf16_f32(BM, D, 1);
+      const uint32_t tS0 = tbase + C::COL_S0, tS1 = tbase + C::COL_S1, tO = tbase + C::COL_O;
+      bool ok = mbar_wait(b_q, 0, a.wait_ns, abort_flag);
+      auto issue_qk = [&](int j) -> bool {
+        const int s = j % NST;
+        if (!mbar_wait(b_kfull(s), (j / NST) & 1, a.wait_ns, abort_flag)) return false;
+        tc_fence_after();
+        fence_proxy_async_smem();
+        const uint32_t kb = sK0 + s * C::KV_BYTES;
+        const uint32_t tS = (j & 1) ? tS1 : tS0;
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk) {
+          const uint32_t off = (kk >> 2) * (128 * 128) + (kk & 3) * 32;
+          umma_bf16_ss(tS, sdesc_sw128(sQ + off, 16, 1024), sdesc_sw128(kb + off, 16, 1024),
+                       idesc_qk, kk > 0 ? 1u : 0u);
+        }
+        umma_commit(b_sfull0 + 8 * (j & 1));
+        umma_commit(b_kempty(s));
+        return true;
+      };
+      auto issue_pv = [&](int j) -> bool {
+        const int s = j % NST;
+        if (!mbar_wait(b_p, j & 1, a.wait_ns, abort_flag)) return false;
+        if (!mbar_wait(b_vfull(s), (j / NST) & 1, a.wait_ns, abort_flag)) return false;
+        tc_fence_after();
+        fence_proxy_async_smem();
+        const uint32_t vb = sV0 + s * C::KV_BYTES;
+#pragma unroll
+        for (int kk = 0; kk < BN / 16; ++kk) {
+          const uint32_t offp = (kk >> 2) * (128 * 128) + (kk & 3) * 32;
+          const uint64_t bdesc = sdesc_sw128(vb + kk * 16 * 128, BN * 128, 1024);
+          umma_bf16_ss(tO, sdesc_sw128(sP + offp, 16, 1024), bdesc, idesc_pv,
+                       (j > 0 || kk > 0) ? 1u : 0u);
+        }
+        if (C::kSplit) {
+#pragma unroll
+          for (int kk = 0; kk < BN / 16; ++kk) {
+            const uint32_t offp = (kk >> 2) * (128 * 128) + (kk & 3) * 32;
+            const uint64_t bdesc = sdesc_sw128(vb + kk * 16 * 128, BN * 128, 1024);
+            umma_bf16_ss(tO, sdesc_sw128(sP + C::P_BYTES + offp, 16, 1024), bdesc, idesc_pv, 1u);
+          }
+        }
+        umma_commit(b_pv);
+        umma_commit(b_vempty(s));
+        return true;
+      };
+      if (ok) ok = issue_qk(0);
+      if (ok && T > 1) ok = issue_qk(1);
+      for (int j = 0; j < T && ok; ++j) {
+        ok = issue_pv(j);
+        if (ok && j + 2 < T) ok = issue_qk(j + 2);
+      }
+      if (!ok && !*abort_flag) {
+        *abort_flag = 1;
+        record_status(a.status, kStatusTimeout);
+      }
+      // make sure nothing issued is still running before TMEM is released
+      umma_commit(b_drain);
+      volatile int never = 0;
+      mbar_wait(b_drain, 0, 2000000000ull, &never);
+    }
+  } else {
+    // ------------------------------------------------------------------ softmax
+    const int r = tid;                           // query row == TMEM lane
+    const uint32_t lane_addr = static_cast<uint32_t>(warp * 32) << 16;
+    const float sl2 = a.scale_log2;
+    float m_run = -INFINITY, l_run = 0.f;
+    bool ok = true;
+    float s[BN];
+    for (int j = 0; j < T; ++j) {
+      if (!mbar_wait(b_sfull0 + 8 * (j & 1), (j >> 1) & 1, a.wait_ns, abort_flag)) { ok = false; break; }
+      tc_fence_after();
+      const uint32_t tS = tbase + lane_addr + ((j & 1) ? C::COL_S1 : C::COL_S0);
+#pragma unroll
+      for (int cc = 0; cc < BN / 32; ++cc) {
+        float tmp[32];
+        tmem_ld32(tS + cc * 32, tmp);
+#pragma unroll
+        for (int i = 0; i < 32; ++i) s[cc * 32 + i] = tmp[i];
+      }
+      tmem_wait_ld();
+      const int nvalid = nkeys - j * BN;   // >= 1
+      float mx = -INFINITY;
+#pragma unroll
+      for (int i = 0; i < BN; ++i) {
+        if (i >= nvalid) s[i] = -INFINITY;
+        mx = fmaxf(mx, s[i]);
+      }
+      mx *= sl2;
+      float alpha = 1.f;
+      bool resc = false;
+      if (j == 0) {
+        m_run = mx;
+      } else if (mx > m_run + 8.f) {      // lazy rescale: only when the max grew by > 2^8
+        alpha = ex2_approx(m_run - mx);
+        m_run = mx;
+        resc = true;
+      }
+      float rs = 0.f;
+#pragma unroll
+      for (int i = 0; i < BN; ++i) {
+        s[i] = ex2_approx(fmaf(s[i], sl2, -m_run));
+        rs += s[i];
+      }
+      l_run = fmaf(l_run, alpha, rs);
+      // P buffer and O are free once the previous P.V has completed
+      if (j > 0) {
+        if (!mbar_wait(b_pv, (j - 1) & 1, a.wait_ns, abort_flag)) { ok = false; break; }
+        tc_fence_after();
+        if (__any_sync(0xffffffffu, resc)) {
+          const uint32_t tO = tbase + lane_addr + C::COL_O;
+#pragma unroll
+          for (int cc = 0; cc < D / 32; ++cc) {
+            float o[32];
+            tmem_ld32(tO + cc * 32, o);
+            tmem_wait_ld();
+#pragma unroll
+            for (int i = 0; i < 32; ++i) o[i] *= alpha;
+            tmem_st32(tO + cc * 32, o);
+          }
+          tmem_wait_st();
+        }
+      }
+      uint8_t *pP = smem + C::OFF_P;
+#pragma unroll
+      for (int c16 = 0; c16 < BN / 8; ++c16) {
+        uint4 hi;
+        hi.x = pack_bf16x2(s[c16 * 8 + 0], s[c16 * 8 + 1]);
+        hi.y = pack_bf16x2(s[c16 * 8 + 2], s[c16 * 8 + 3]);
+        hi.z = pack_bf16x2(s[c16 * 8 + 4], s[c16 * 8 + 5]);
+        hi.w = pack_bf16x2(s[c16 * 8 + 6], s[c16 * 8 + 7]);
+        const uint32_t off = sw128_offset(r, c16, BM);
+        *reinterpret_cast<uint4 *>(pP + off) = hi;
+        if (C::kSplit) {
+          const __nv_bfloat162 *h2 = reinterpret_cast<const __nv_bfloat162 *>(&hi);
+          uint4 lo;
+          uint32_t *lw = reinterpret_cast<uint32_t *>(&lo);
+#pragma unroll
+          for (int u = 0; u < 4; ++u) {
+            const float2 hf = __bfloat1622float2(h2[u]);
+            lw[u] = pack_bf16x2(s[c16 * 8 + 2 * u] - hf.x, s[c16 * 8 + 2 * u + 1] - hf.y);
+          }
+          *reinterpret_cast<uint4 *>(pP + C::P_BYTES + off) = lo;
+        }
+      }
+      fence_proxy_async_smem();
+      tc_fence_before();
+      mbar_arrive(b_p);
+    }
+    if (ok && T > 0) {
+      if (!mbar_wait(b_pv, (T - 1) & 1, a.wait_ns, abort_flag)) ok = false;
+    }
+    if (!ok) {
+      if (!*abort_flag) {
+        *abort_flag = 1;
+        record_status(a.status, kStatusTimeout);
+      }
+    } else {
+      // ------------------------------------------------------------------ epilogue
+      tc_fence_after();
+      const int q = q_token(r);
+      const float inv_l = 1.f / l_run;
+      const uint32_t tO = tbase + lane_addr + C::COL_O;
+      const size_t row = (head + (q >= 0 ? q : 0)) * D;
+#pragma unroll
+      for (int cc = 0; cc < D / 32; ++cc) {
+        float o[32];
+        tmem_ld32(tO + cc * 32, o);
+        tmem_wait_ld();
+        if (q < 0) continue;
+#pragma unroll
+        for (int i = 0; i < 32; ++i) o[i] *= inv_l;
+        if (MODE == kModeStep) {
+          const float4 *rp = reinterpret_cast<const float4 *>(a.residual + row + cc * 32);
+#pragma unroll
+          for (int u = 0; u < 8; ++u) {
+            const float4 rv = __ldg(rp + u);
+            o[4 * u + 0] += rv.x;
+            o[4 * u + 1] += rv.y;
+            o[4 * u + 2] += rv.z;
+            o[4 * u + 3] += rv.w;
+          }
+        }
+        if (MODE == kModePlanResid) {
+          const float4 *dp = reinterpret_cast<const float4 *>(a.O32_in + row + cc * 32);
+          float4 *rp = reinterpret_cast<float4 *>(a.R_out + row + cc * 32);
+#pragma unroll
+          for (int u = 0; u < 8; ++u) {
+            const float4 dv = __ldg(dp + u);
+            rp[u] = make_float4(dv.x - o[4 * u], dv.y - o[4 * u + 1], dv.z - o[4 * u + 2],
+                                dv.w - o[4 * u + 3]);
+          }
+        }
+        if (MODE == kModePlanDense) {
+          float4 *op = reinterpret_cast<float4 *>(a.O32 + row + cc * 32);
+#pragma unroll
+          for (int u = 0; u < 8; ++u)
+            op[u] = make_float4(o[4 * u], o[4 * u + 1], o[4 * u + 2], o[4 * u + 3]);
+        }
+        if (MODE == kModeDense || MODE == kModeStep || (MODE == kModePlanDense && a.O != nullptr)) {
+          uint4 *op = reinterpret_cast<uint4 *>(a.O + row + cc * 32);
+#pragma unroll
+          for (int u = 0; u < 4; ++u) {
+            uint4 w;
+            w.x = pack_bf16x2(o[8 * u + 0], o[8 * u + 1]);
+            w.y = pack_bf16x2(o[8 * u + 2], o[8 * u + 3]);
+            w.z = pack_bf16x2(o[8 * u + 4], o[8 * u + 5]);
+            w.w = pack_bf16x2(o[8 * u + 6], o[8 * u + 7]);
+            op[u] = w;
+          }
+        }
+      }
+      if (MODE == kModePlanDense && q >= 0) {
+        a.row_m[head + q] = m_run;
+        a.row_l[head + q] = l_run;
+      }
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 4) {
+    tc_fence_after();
+    tmem_dealloc(tbase, C::TMEM_COLS);
+  }
+}
+
+}  // namespace mcs

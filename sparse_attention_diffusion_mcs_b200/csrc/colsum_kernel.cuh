@@ -1,0 +1,228 @@
+// colsum_kernel.cuh -- group probability sums, step a3 of the plan.
+//
+//   colsum[g, j] = sum_{i in group g} P_ij,  P_ij = 2^(s_ij*scale*log2e - m_i) / l_i
+//
+// with (m_i, l_i) the exact row statistics from the dense pass ("KV indices
+// selected using exact attention probabilities", aiqbench.com abstract; the
+// per-group sum is the selection score this library adopts).
+//
+// The score tile is computed transposed, S^T = K_tile . Q_g^T (keys on TMEM
+// lanes, the group's queries on columns), so each thread owns one key and the
+// sum over the group is a private loop over its TMEM row: no cross-thread
+// reduction.  CTA = one (head, group); loops over all N/128 key tiles.
+//   warps 0-3 reduce, warp 4 issues UMMA, warps 5-6 stream K tiles (cp.async).
+#pragma once
+
+#include "mcs_common.cuh"
+
+namespace mcs {
+
+struct ColsumArgs {
+  const bf16 *Q, *K;        // [BH, N, D]
+  const int32_t *perm;      // [BH, N]
+  const float *row_m;       // [BH, N] (log2 domain)
+  const float *row_l;       // [BH, N]
+  float *colsum;            // [BH, n_groups, N]
+  int N, G, n_groups;
+  float scale_log2;
+  unsigned *status;
+  uint64_t wait_ns;
+};
+
+template <int D>
+struct ColsumCfg {
+  static constexpr int BM = 128, BN = 128;   // BM keys per tile (MMA M), BN queries (MMA N)
+  static constexpr int NST = 4;
+  static constexpr int Q_BYTES = BN * D * 2;
+  static constexpr int K_BYTES = BM * D * 2;
+  static constexpr int OFF_Q = 0;
+  static constexpr int OFF_K = Q_BYTES;
+  static constexpr int OFF_STAT = OFF_K + NST * K_BYTES;     // float2 (m, 1/l) x 128
+  static constexpr int OFF_BAR = OFF_STAT + 128 * 8;
+  static constexpr int N_BAR = 1 + 2 * NST + 5;              // q, k full/empty, s_full[2], s_free[2], drain
+  static constexpr int OFF_MISC = OFF_BAR + 8 * N_BAR;
+  static constexpr int SMEM = OFF_MISC + 16 + 1024;
+  static constexpr uint32_t TMEM_COLS = 256;
+};
+
+template <int D>
+__global__ void __launch_bounds__(224, 1) colsum_kernel(const ColsumArgs a) {
+  using C = ColsumCfg<D>;
+  constexpr int BM = C::BM, NST = C::NST;
+  constexpr int CPR = D / 8;
+  constexpr int RPP = 64 / CPR;         // rows per loader pass (64 loader threads)
+
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                              ~static_cast<uintptr_t>(1023));
+  const uint32_t sbase = smem_u32(smem);
+  const uint32_t sQ = sbase + C::OFF_Q;
+  const uint32_t sK0 = sbase + C::OFF_K;
+  float2 *stat = reinterpret_cast<float2 *>(smem + C::OFF_STAT);
+  const uint32_t bar0 = sbase + C::OFF_BAR;
+  const uint32_t b_q = bar0;
+  auto b_kfull = [&](int s) { return bar0 + 8 * (1 + s); };
+  auto b_kempty = [&](int s) { return bar0 + 8 * (1 + NST + s); };
+  const uint32_t b_sfull0 = bar0 + 8 * (1 + 2 * NST);
+  const uint32_t b_sfree0 = bar0 + 8 * (3 + 2 * NST);
+  const uint32_t b_drain = bar0 + 8 * (5 + 2 * NST);
+  uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem + C::OFF_MISC);
+  volatile int *abort_flag = reinterpret_cast<volatile int *>(smem + C::OFF_MISC + 4);
+
+  const int tid = threadIdx.x;
+  const int warp = tid >> 5;
+  const int g = blockIdx.x;
+  const int bh = blockIdx.y;
+  const int N = a.N;
+  const size_t head = static_cast<size_t>(bh) * N;
+  const int T = (N + BM - 1) / BM;
+
+  auto q_token = [&](int r) -> int {
+    const int gr = g * a.G + r;
+    if (r >= a.G || gr >= N) return -1;
+    const int q = a.perm[head + gr];
+    if (static_cast<unsigned>(q) >= static_cast<unsigned>(N)) {   // corrupt metadata: never gather out of range
+      record_status(a.status, kStatusBadMeta);
+      return -1;
+    }
+    return q;
+  };
+
+  if (tid == 0) {
+    mbar_init(b_q, 64);
+    for (int s = 0; s < NST; ++s) {
+      mbar_init(b_kfull(s), 64);
+      mbar_init(b_kempty(s), 1);
+    }
+    mbar_init(b_sfull0, 1);
+    mbar_init(b_sfull0 + 8, 1);
+    mbar_init(b_sfree0, 128);
+    mbar_init(b_sfree0 + 8, 128);
+    mbar_init(b_drain, 1);
+    *abort_flag = 0;
+    mbar_init_fence();
+  }
+  if (tid < 128) {
+    const int q = q_token(tid);
+    if (q >= 0) {
+      stat[tid] = make_float2(a.row_m[head + q], 1.f / a.row_l[head + q]);
+    } else {
+      stat[tid] = make_float2(INFINITY, 0.f);   // padding query contributes 0
+    }
+  }
+  if (warp == 4) {
+    tmem_alloc(smem_u32(tmem_slot), C::TMEM_COLS);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tbase = *tmem_slot;
+
+  if (warp >= 5) {
+    const int lt = tid - 160;   // 0..63
+    const int c = lt % CPR;
+    const int r0 = lt / CPR;
+#pragma unroll 4
+    for (int i = 0; i < 128 / RPP; ++i) {
+      const int r = r0 + i * RPP;
+      const int q = q_token(r);
+      const bf16 *src = q >= 0 ? a.Q + (head + q) * D + c * 8 : a.Q;
+      cp_async16(sQ + sw128_offset(r, c, 128), src, q >= 0 ? 16u : 0u);
+    }
+    cp_async_arrive_noinc(b_q);
+    bool ok = true;
+    for (int j = 0; j < T; ++j) {
+      const int s = j % NST;
+      if (!mbar_wait(b_kempty(s), ((j / NST) & 1) ^ 1, a.wait_ns, abort_flag)) { ok = false; break; }
+      const uint32_t dK = sK0 + s * C::K_BYTES;
+#pragma unroll
+      for (int i = 0; i < 128 / RPP; ++i) {
+        const int r = r0 + i * RPP;
+        const int key = j * BM + r;
+        const bf16 *src = key < N ? a.K + (head + key) * D + c * 8 : a.K;
+        cp_async16(dK + sw128_offset(r, c, BM), src, key < N ? 16u : 0u);
+      }
+      cp_async_arrive_noinc(b_kfull(s));
+    }
+    if (!ok && !*abort_flag) {
+      *abort_flag = 1;
+      record_status(a.status, kStatusTimeout);
+    }
+    cp_async_wait_all();
+  } else if (warp == 4) {
+    if (tid == 128) {
+      constexpr uint32_t idesc = idesc_bf16_f32(BM, 128, 0);
+      bool ok = mbar_wait(b_q, 0, a.wait_ns, abort_flag);
+      for (int j = 0; j < T && ok; ++j) {
+        const int s = j % NST;
+        const int b = j & 1;
+        if (j >= 2 && !mbar_wait(b_sfree0 + 8 * b, ((j >> 1) - 1) & 1, a.wait_ns, abort_flag)) {
+          ok = false;
+          break;
+        }
+        if (!mbar_wait(b_kfull(s), (j / NST) & 1, a.wait_ns, abort_flag)) { ok = false; break; }
+        tc_fence_after();
+        fence_proxy_async_smem();
+        const uint32_t kb = sK0 + s * C::K_BYTES;
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk) {
+          const uint32_t off = (kk >> 2) * (128 * 128) + (kk & 3) * 32;
+          umma_bf16_ss(tbase + b * 128, sdesc_sw128(kb + off, 16, 1024),
+                       sdesc_sw128(sQ + off, 16, 1024), idesc, kk > 0 ? 1u : 0u);
+        }
+        umma_commit(b_sfull0 + 8 * b);
+        umma_commit(b_kempty(s));
+      }
+      if (!ok && !*abort_flag) {
+        *abort_flag = 1;
+        record_status(a.status, kStatusTimeout);
+      }
+      // make sure nothing issued is still running before TMEM is released
+      umma_commit(b_drain);
+      volatile int never = 0;
+      mbar_wait(b_drain, 0, 2000000000ull, &never);
+    }
+  } else {
+    const uint32_t lane_addr = static_cast<uint32_t>(warp * 32) << 16;
+    const float sl2 = a.scale_log2;
+    float *out = a.colsum + (static_cast<size_t>(bh) * a.n_groups + g) * N;
+    bool ok = true;
+    for (int j = 0; j < T; ++j) {
+      const int b = j & 1;
+      if (!mbar_wait(b_sfull0 + 8 * b, (j >> 1) & 1, a.wait_ns, abort_flag)) { ok = false; break; }
+      tc_fence_after();
+      float acc0 = 0.f, acc1 = 0.f;
+#pragma unroll
+      for (int cc = 0; cc < 4; ++cc) {
+        float v[32];
+        tmem_ld32(tbase + lane_addr + b * 128 + cc * 32, v);
+        tmem_wait_ld();
+#pragma unroll
+        for (int i = 0; i < 32; i += 2) {
+          const float2 s0 = stat[cc * 32 + i];
+          const float2 s1 = stat[cc * 32 + i + 1];
+          acc0 = fmaf(ex2_approx(fmaf(v[i], sl2, -s0.x)), s0.y, acc0);
+          acc1 = fmaf(ex2_approx(fmaf(v[i + 1], sl2, -s1.x)), s1.y, acc1);
+        }
+      }
+      tc_fence_before();
+      mbar_arrive(b_sfree0 + 8 * b);
+      const int key = j * BM + tid;
+      if (key < N) out[key] = acc0 + acc1;
+    }
+    if (!ok && !*abort_flag) {
+      *abort_flag = 1;
+      record_status(a.status, kStatusTimeout);
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 4) {
+    tc_fence_after();
+    tmem_dealloc(tbase, C::TMEM_COLS);
+  }
+}
+
+}  // namespace mcs

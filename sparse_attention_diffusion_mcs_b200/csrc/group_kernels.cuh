@@ -1,0 +1,331 @@
+// group_kernels.cuh -- tile-aligned grouping of similar queries, step a1.
+//
+// "organizing similar queries into tile-aligned groups for efficient GPU
+// execution" (aiqbench.com abstract; cctest.ai "Hardware-aware query
+// organization").  The pages do not say how similarity is measured; this
+// library orders each head's queries by their projection on the first
+// principal direction of Q and cuts the order into contiguous runs of G.
+//
+// Everything runs in fp64 (bf16 inputs are exact in fp64), so the order is
+// the order of the exact projections up to fp64 rounding:
+//   mean_kernel       per (head, chunk of rows): column sums of Q
+//   cov_kernel        per (head, chunk): sum of (q - mu)(q - mu)^T
+//   eig_kernel        per head: combine chunks, top eigenvector by repeated
+//                     squaring + power iteration, sign fixed so the
+//                     largest-magnitude component is positive
+//   project_kernel    p_n = (q_n - mu) . v  -> order-preserving uint64 key
+//   sort_kernel       per head: stable LSD radix sort of (key, n) -> perm
+#pragma once
+
+#include "mcs_common.cuh"
+
+namespace mcs {
+
+constexpr int kGroupChunk = 2048;     // rows per chunk of the mean / covariance passes
+constexpr int kSortThreads = 1024;
+
+// ---------------------------------------------------------------- mean
+template <int D>
+__global__ void __launch_bounds__(256) mean_kernel(const bf16 *__restrict__ Q, int N, int n_chunks,
+                                                   double *__restrict__ part) {
+  const int chunk = blockIdx.x, bh = blockIdx.y;
+  const int r0 = chunk * kGroupChunk;
+  const int r1 = min(N, r0 + kGroupChunk);
+  constexpr int RSTEP = 256 / D;
+  const int col = threadIdx.x % D;
+  const int rr = threadIdx.x / D;
+  const bf16 *q = Q + static_cast<size_t>(bh) * N * D;
+  double acc = 0.0;
+  for (int r = r0 + rr; r < r1; r += RSTEP) acc += __bfloat162float(q[static_cast<size_t>(r) * D + col]);
+  __shared__ double red[256];
+  red[threadIdx.x] = acc;
+  __syncthreads();
+  if (threadIdx.x < D) {
+    double sum = 0.0;
+    for (int i = 0; i < RSTEP; ++i) sum += red[i * D + threadIdx.x];
+    part[(static_cast<size_t>(bh) * n_chunks + chunk) * D + threadIdx.x] = sum;
+  }
+}
+
+template <int D>
+__global__ void mean_finalize_kernel(const double *__restrict__ part, int N, int n_chunks,
+                                     double *__restrict__ mean) {
+  const int bh = blockIdx.x, c = threadIdx.x;
+  if (c >= D) return;
+  double sum = 0.0;
+  for (int i = 0; i < n_chunks; ++i) sum += part[(static_cast<size_t>(bh) * n_chunks + i) * D + c];
+  mean[bh * D + c] = sum / N;
+}
+
+// ---------------------------------------------------------------- covariance
+// 256 threads; thread (ti, tj) accumulates an RxR block of the DxD matrix in
+// fp64, R = D/16.  Rows are staged (centred) through shared memory.
+template <int D>
+__global__ void __launch_bounds__(256) cov_kernel(const bf16 *__restrict__ Q, const double *__restrict__ mean,
+                                                  int N, int n_chunks, double *__restrict__ part) {
+  constexpr int R = D / 16;
+  constexpr int ROWS = 16;
+  __shared__ double xs[ROWS][D + 1];
+  const int chunk = blockIdx.x, bh = blockIdx.y;
+  const int r0 = chunk * kGroupChunk;
+  const int r1 = min(N, r0 + kGroupChunk);
+  const int ti = threadIdx.x / 16, tj = threadIdx.x % 16;
+  const bf16 *q = Q + static_cast<size_t>(bh) * N * D;
+  const double *mu = mean + bh * D;
+  double acc[R][R];
+#pragma unroll
+  for (int i = 0; i < R; ++i)
+#pragma unroll
+    for (int j = 0; j < R; ++j) acc[i][j] = 0.0;
+  for (int rb = r0; rb < r1; rb += ROWS) {
+    __syncthreads();
+    for (int e = threadIdx.x; e < ROWS * D; e += 256) {
+      const int rr = e / D, c = e % D;
+      const int r = rb + rr;
+      xs[rr][c] = r < r1 ? static_cast<double>(__bfloat162float(q[static_cast<size_t>(r) * D + c])) - mu[c] : 0.0;
+    }
+    __syncthreads();
+#pragma unroll 2
+    for (int rr = 0; rr < ROWS; ++rr) {
+      double xi[R], xj[R];
+#pragma unroll
+      for (int i = 0; i < R; ++i) {
+        xi[i] = xs[rr][ti * R + i];
+        xj[i] = xs[rr][tj * R + i];
+      }
+#pragma unroll
+      for (int i = 0; i < R; ++i)
+#pragma unroll
+        for (int j = 0; j < R; ++j) acc[i][j] = fma(xi[i], xj[j], acc[i][j]);
+    }
+  }
+  double *out = part + (static_cast<size_t>(bh) * n_chunks + chunk) * D * D;
+#pragma unroll
+  for (int i = 0; i < R; ++i)
+#pragma unroll
+    for (int j = 0; j < R; ++j) out[(ti * R + i) * D + tj * R + j] = acc[i][j];
+}
+
+// ---------------------------------------------------------------- eigenvector
+// One CTA of 256 threads per head.  C (fp64) and the squaring scratch live in
+// workspace (L2-resident, D*D doubles each); M, a normalised power of C
+// obtained by repeated squaring, lives in shared memory.  Squaring separates
+// the top eigenvector even for small spectral gaps; a few power iterations
+// with M and then with C itself give v.
+template <int D>
+__global__ void __launch_bounds__(256) eig_kernel(const double *__restrict__ part, int N, int n_chunks,
+                                                  double *__restrict__ cov, double *__restrict__ scratch,
+                                                  double *__restrict__ vdir, float *__restrict__ lambda) {
+  extern __shared__ double dsm[];
+  double *M = dsm;               // D*D
+  double *vec = M + D * D;       // D
+  double *tmp = vec + D;         // D
+  __shared__ double red[256];
+  const int bh = blockIdx.x, tid = threadIdx.x;
+  double *Cm = cov + static_cast<size_t>(bh) * D * D;
+  double *T = scratch + static_cast<size_t>(bh) * D * D;
+
+  auto block_sum = [&](double x) -> double {
+    red[tid] = x;
+    __syncthreads();
+    for (int o = 128; o > 0; o >>= 1) {
+      if (tid < o) red[tid] += red[tid + o];
+      __syncthreads();
+    }
+    const double r = red[0];
+    __syncthreads();
+    return r;
+  };
+
+  for (int e = tid; e < D * D; e += 256) {
+    double sum = 0.0;
+    for (int i = 0; i < n_chunks; ++i) sum += part[(static_cast<size_t>(bh) * n_chunks + i) * D * D + e];
+    Cm[e] = sum / N;
+  }
+  __syncthreads();
+  const double tr = block_sum(tid < D ? Cm[tid * D + tid] : 0.0);
+  if (!(tr > 0.0)) {   // all queries identical: every direction is principal; take e_0
+    if (tid < D) vdir[bh * D + tid] = tid == 0 ? 1.0 : 0.0;
+    if (tid == 0) lambda[bh] = 0.f;
+    return;
+  }
+  for (int e = tid; e < D * D; e += 256) M[e] = Cm[e] / tr;
+  __syncthreads();
+  for (int sq = 0; sq < 10; ++sq) {        // M <- M^2 / trace(M^2)  ->  C^(2^10), normalised
+    for (int e = tid; e < D * D; e += 256) {
+      const int i = e / D, j = e % D;
+      double acc = 0.0;
+      for (int t = 0; t < D; ++t) acc += M[i * D + t] * M[t * D + j];
+      T[e] = acc;
+    }
+    __syncthreads();
+    const double t2 = block_sum(tid < D ? T[tid * D + tid] : 0.0);
+    for (int e = tid; e < D * D; e += 256) M[e] = T[e] / t2;
+    __syncthreads();
+  }
+  // start from the column of M with the largest diagonal entry
+  if (tid == 0) {
+    int best = 0;
+    for (int i = 1; i < D; ++i)
+      if (M[i * D + i] > M[best * D + best]) best = i;
+    red[0] = best;
+  }
+  __syncthreads();
+  const int best = static_cast<int>(red[0]);
+  __syncthreads();
+  if (tid < D) vec[tid] = M[tid * D + best];
+  __syncthreads();
+  auto matvec_norm = [&](const double *A) {
+    if (tid < D) {
+      double acc = 0.0;
+      for (int t = 0; t < D; ++t) acc += A[tid * D + t] * vec[t];
+      tmp[tid] = acc;
+    }
+    __syncthreads();
+    const double nn = block_sum(tid < D ? tmp[tid] * tmp[tid] : 0.0);
+    const double inv = nn > 0.0 ? 1.0 / sqrt(nn) : 0.0;
+    if (tid < D) vec[tid] = tmp[tid] * inv;
+    __syncthreads();
+  };
+  for (int it = 0; it < 8; ++it) matvec_norm(M);
+  for (int it = 0; it < 64; ++it) matvec_norm(Cm);
+  // sign: the first component of largest magnitude is positive
+  if (tid == 0) {
+    int im = 0;
+    for (int i = 1; i < D; ++i)
+      if (fabs(vec[i]) > fabs(vec[im])) im = i;
+    red[0] = vec[im] < 0.0 ? -1.0 : 1.0;
+  }
+  __syncthreads();
+  const double sg = red[0];
+  __syncthreads();
+  if (tid < D) {
+    double acc = 0.0;
+    for (int t = 0; t < D; ++t) acc += Cm[tid * D + t] * vec[t];
+    tmp[tid] = acc * vec[tid];
+  }
+  __syncthreads();
+  const double lam = block_sum(tid < D ? tmp[tid] : 0.0);
+  if (tid < D) vdir[bh * D + tid] = sg * vec[tid];
+  if (tid == 0) lambda[bh] = static_cast<float>(lam);
+}
+
+// ---------------------------------------------------------------- projection
+__device__ __forceinline__ unsigned long long double_order_key(double f) {
+  const unsigned long long b = static_cast<unsigned long long>(__double_as_longlong(f));
+  return (b & 0x8000000000000000ull) ? ~b : (b | 0x8000000000000000ull);
+}
+
+template <int D>
+__global__ void __launch_bounds__(256) project_kernel(const bf16 *__restrict__ Q, const double *__restrict__ mean,
+                                                      const double *__restrict__ vdir, int N,
+                                                      unsigned long long *__restrict__ keys,
+                                                      int32_t *__restrict__ vals) {
+  // one warp per row; lanes split the columns
+  const int bh = blockIdx.y;
+  const int row = blockIdx.x * 8 + (threadIdx.x >> 5);
+  const int lane = threadIdx.x & 31;
+  if (row >= N) return;
+  const bf16 *q = Q + (static_cast<size_t>(bh) * N + row) * D;
+  const double *mu = mean + bh * D;
+  const double *v = vdir + bh * D;
+  double acc = 0.0;
+  for (int c = lane; c < D; c += 32) acc = fma(static_cast<double>(__bfloat162float(q[c])) - mu[c], v[c], acc);
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
+  if (lane == 0) {
+    keys[static_cast<size_t>(bh) * N + row] = double_order_key(acc);
+    vals[static_cast<size_t>(bh) * N + row] = row;
+  }
+}
+
+// ---------------------------------------------------------------- stable LSD radix sort
+// One CTA per head, 8 passes of 8 bits over 64-bit keys.  Each pass:
+// histogram, exclusive scan, then a scatter over tiles of 1024 keys in index
+// order, ranking equal digits by (warp, lane) so the pass is stable.
+__global__ void __launch_bounds__(kSortThreads) sort_kernel(unsigned long long *keys_a, int32_t *vals_a,
+                                                            unsigned long long *keys_b, int32_t *vals_b,
+                                                            int N, int32_t *__restrict__ perm) {
+  __shared__ unsigned bins[256];
+  __shared__ unsigned base[256];
+  __shared__ unsigned tile_tot[256];
+  __shared__ unsigned short wcnt[32][256];   // per-warp digit counts, then exclusive prefixes
+  const int bh = blockIdx.x;
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const unsigned lt_mask = (1u << lane) - 1u;
+  unsigned long long *kin = keys_a + static_cast<size_t>(bh) * N;
+  int32_t *vin = vals_a + static_cast<size_t>(bh) * N;
+  unsigned long long *kout = keys_b + static_cast<size_t>(bh) * N;
+  int32_t *vout = vals_b + static_cast<size_t>(bh) * N;
+
+  for (int pass = 0; pass < 8; ++pass) {
+    const int shift = pass * 8;
+    for (int i = tid; i < 256; i += kSortThreads) bins[i] = 0;
+    __syncthreads();
+    for (int j = tid; j < N; j += kSortThreads) atomicAdd(&bins[static_cast<unsigned>(kin[j] >> shift) & 255u], 1u);
+    __syncthreads();
+    if (warp == 0) {
+      unsigned c[8], sum = 0;
+#pragma unroll
+      for (int b = 0; b < 8; ++b) {
+        c[b] = bins[lane * 8 + b];
+        sum += c[b];
+      }
+      unsigned inc = sum;
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const unsigned y = __shfl_up_sync(0xffffffffu, inc, o);
+        if (lane >= o) inc += y;
+      }
+      unsigned run = inc - sum;
+#pragma unroll
+      for (int b = 0; b < 8; ++b) {
+        base[lane * 8 + b] = run;
+        run += c[b];
+      }
+    }
+    __syncthreads();
+    for (int t0 = 0; t0 < N; t0 += kSortThreads) {
+      const int j = t0 + tid;
+      const bool valid = j < N;
+      unsigned long long key = 0;
+      int32_t val = 0;
+      if (valid) {
+        key = kin[j];
+        val = vin[j];
+      }
+      const unsigned digit = valid ? (static_cast<unsigned>(key >> shift) & 255u) : 256u;
+      for (int b = lane; b < 256; b += 32) wcnt[warp][b] = 0;
+      __syncwarp();
+      const unsigned peers = __match_any_sync(0xffffffffu, digit);
+      const unsigned rank_in_warp = __popc(peers & lt_mask);
+      if (valid && rank_in_warp == 0) wcnt[warp][digit] = static_cast<unsigned short>(__popc(peers));
+      __syncthreads();
+      if (tid < 256) {
+        unsigned run = 0;
+        for (int w = 0; w < 32; ++w) {
+          const unsigned cnt = wcnt[w][tid];
+          wcnt[w][tid] = static_cast<unsigned short>(run);
+          run += cnt;
+        }
+        tile_tot[tid] = run;
+      }
+      __syncthreads();
+      if (valid) {
+        const unsigned pos = base[digit] + wcnt[warp][digit] + rank_in_warp;
+        kout[pos] = key;
+        vout[pos] = val;
+      }
+      __syncthreads();
+      if (tid < 256) base[tid] += tile_tot[tid];
+      __syncthreads();
+    }
+    unsigned long long *kt = kin; kin = kout; kout = kt;
+    int32_t *vt = vin; vin = vout; vout = vt;
+    __syncthreads();
+  }
+  // after an even number of passes the sorted data is back in keys_a / vals_a
+  for (int j = tid; j < N; j += kSortThreads) perm[static_cast<size_t>(bh) * N + j] = vin[j];
+}
+
+}  // namespace mcs

@@ -1,0 +1,434 @@
+// mcs_api.cu -- host side of the C ABI declared in include/mcs.h: argument
+// checks, workspace carving and kernel launches on the caller's stream.
+#include <climits>
+#include <cstdint>
+#include <cstring>
+#include <mutex>
+
+#include "../../include/mcs.h"
+#include "attn_kernel.cuh"
+#include "colsum_kernel.cuh"
+#include "group_kernels.cuh"
+#include "topk_kernel.cuh"
+#include "validate_kernels.cuh"
+
+using namespace mcs;
+
+namespace {
+
+__device__ unsigned g_status_word;
+
+constexpr int kMaxDevices = 64;
+uint64_t g_wait_ns = 4000000000ull;
+std::mutex g_mu;
+unsigned *g_status_ptr[kMaxDevices];
+
+unsigned *status_ptr() {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return nullptr;
+  std::lock_guard<std::mutex> lk(g_mu);
+  if (!g_status_ptr[dev]) {
+    void *p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_status_word) != cudaSuccess) return nullptr;
+    g_status_ptr[dev] = static_cast<unsigned *>(p);
+  }
+  return g_status_ptr[dev];
+}
+
+inline bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+inline size_t align256(size_t x) { return (x + 255) & ~static_cast<size_t>(255); }
+
+bool shape_ok(int B, int H, int N, int d) {
+  if (B < 1 || H < 1 || N < 1) return false;
+  if (static_cast<long long>(B) * H > 65535) return false;
+  if (N > (1 << 24)) return false;
+  (void)d;
+  return true;
+}
+bool d_ok(int d) { return d == 64 || d == 128; }
+bool g_ok(int G) { return G == 64 || G == 128; }
+
+template <typename F>
+cudaError_t set_smem(F *fn, int bytes) {
+  return cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+}
+
+// ---------------------------------------------------------------- attention launches
+template <int D, int MODE>
+cudaError_t launch_attn(const AttnArgs &a, int grid_x, int BH, cudaStream_t s) {
+  using C = AttnCfg<D, MODE>;
+  static_assert(C::SMEM <= 232448, "shared memory budget");
+  cudaError_t e = set_smem(attn_kernel<D, MODE>, C::SMEM);
+  if (e != cudaSuccess) return e;
+  attn_kernel<D, MODE><<<dim3(grid_x, BH), C::THREADS, C::SMEM, s>>>(a);
+  return cudaGetLastError();
+}
+
+template <int MODE>
+cudaError_t launch_attn_d(int d, const AttnArgs &a, int grid_x, int BH, cudaStream_t s) {
+  return d == 64 ? launch_attn<64, MODE>(a, grid_x, BH, s) : launch_attn<128, MODE>(a, grid_x, BH, s);
+}
+
+AttnArgs base_args(const void *Q, const void *K, const void *V, int N, float scale) {
+  AttnArgs a;
+  std::memset(&a, 0, sizeof(a));
+  a.Q = static_cast<const bf16 *>(Q);
+  a.K = static_cast<const bf16 *>(K);
+  a.V = static_cast<const bf16 *>(V);
+  a.N = N;
+  a.scale_log2 = scale * 1.4426950408889634f;
+  a.status = status_ptr();
+  a.wait_ns = g_wait_ns;
+  return a;
+}
+
+// ---------------------------------------------------------------- plan workspace
+struct PlanWs {
+  size_t mean_part, mean, cov_part, cov64, sq64, vdir, lambda, keys0, vals0, keys1, vals1;
+  size_t row_m, row_l, O32, colsum, total;
+};
+
+PlanWs plan_ws(int B, int H, int N, int d, int G) {
+  const size_t BH = static_cast<size_t>(B) * H;
+  const size_t nch = (N + kGroupChunk - 1) / kGroupChunk;
+  const size_t ng = (N + G - 1) / G;
+  PlanWs w;
+  size_t o = 0;
+  auto take = [&](size_t bytes) {
+    const size_t at = o;
+    o = align256(o + bytes);
+    return at;
+  };
+  w.mean_part = take(BH * nch * d * 8);
+  w.mean = take(BH * d * 8);
+  w.cov_part = take(BH * nch * d * d * 8);
+  w.cov64 = take(BH * d * d * 8);
+  w.sq64 = take(BH * d * d * 8);
+  w.vdir = take(BH * d * 8);
+  w.lambda = take(BH * 4);
+  w.keys0 = take(BH * N * 8);
+  w.vals0 = take(BH * N * 4);
+  w.keys1 = take(BH * N * 8);
+  w.vals1 = take(BH * N * 4);
+  w.row_m = take(BH * N * 4);
+  w.row_l = take(BH * N * 4);
+  w.O32 = take(BH * N * static_cast<size_t>(d) * 4);
+  w.colsum = take(BH * ng * static_cast<size_t>(N) * 4);
+  w.total = o;
+  return w;
+}
+
+template <typename T>
+T *at(void *ws, size_t off) {
+  return reinterpret_cast<T *>(static_cast<uint8_t *>(ws) + off);
+}
+
+mcs_status cuda_status(cudaError_t e) { return e == cudaSuccess ? MCS_OK : MCS_ERR_CUDA; }
+
+// ---------------------------------------------------------------- stages
+template <int D>
+cudaError_t run_group(const void *Q, int BH, int N, int32_t *perm, void *ws, const PlanWs &w,
+                      cudaStream_t s) {
+  const int nch = (N + kGroupChunk - 1) / kGroupChunk;
+  const bf16 *q = static_cast<const bf16 *>(Q);
+  mean_kernel<D><<<dim3(nch, BH), 256, 0, s>>>(q, N, nch, at<double>(ws, w.mean_part));
+  mean_finalize_kernel<D><<<BH, D, 0, s>>>(at<double>(ws, w.mean_part), N, nch, at<double>(ws, w.mean));
+  cov_kernel<D><<<dim3(nch, BH), 256, 0, s>>>(q, at<double>(ws, w.mean), N, nch, at<double>(ws, w.cov_part));
+  const int eig_smem = (D * D + 2 * D) * 8;
+  cudaError_t e = set_smem(eig_kernel<D>, eig_smem);
+  if (e != cudaSuccess) return e;
+  eig_kernel<D><<<BH, 256, eig_smem, s>>>(at<double>(ws, w.cov_part), N, nch, at<double>(ws, w.cov64),
+                                           at<double>(ws, w.sq64), at<double>(ws, w.vdir),
+                                           at<float>(ws, w.lambda));
+  project_kernel<D><<<dim3((N + 7) / 8, BH), 256, 0, s>>>(q, at<double>(ws, w.mean), at<double>(ws, w.vdir), N,
+                                                           at<unsigned long long>(ws, w.keys0),
+                                                           at<int32_t>(ws, w.vals0));
+  sort_kernel<<<BH, kSortThreads, 0, s>>>(at<unsigned long long>(ws, w.keys0), at<int32_t>(ws, w.vals0),
+                                          at<unsigned long long>(ws, w.keys1), at<int32_t>(ws, w.vals1), N,
+                                          perm);
+  return cudaGetLastError();
+}
+
+cudaError_t run_plan_dense(const void *Q, const void *K, const void *V, int BH, int N, int d, float scale,
+                           void *O_dense, void *ws, const PlanWs &w, cudaStream_t s) {
+  AttnArgs a = base_args(Q, K, V, N, scale);
+  a.O = static_cast<bf16 *>(O_dense);
+  a.O32 = at<float>(ws, w.O32);
+  a.row_m = at<float>(ws, w.row_m);
+  a.row_l = at<float>(ws, w.row_l);
+  return launch_attn_d<kModePlanDense>(d, a, (N + 127) / 128, BH, s);
+}
+
+cudaError_t run_select(const void *Q, const void *K, const int32_t *perm, int BH, int N, int d, int G,
+                       int k, float scale, int32_t *kv_idx, void *ws, const PlanWs &w, cudaStream_t s) {
+  const int ng = (N + G - 1) / G;
+  ColsumArgs c;
+  c.Q = static_cast<const bf16 *>(Q);
+  c.K = static_cast<const bf16 *>(K);
+  c.perm = perm;
+  c.row_m = at<float>(ws, w.row_m);
+  c.row_l = at<float>(ws, w.row_l);
+  c.colsum = at<float>(ws, w.colsum);
+  c.N = N;
+  c.G = G;
+  c.n_groups = ng;
+  c.scale_log2 = scale * 1.4426950408889634f;
+  c.status = status_ptr();
+  c.wait_ns = g_wait_ns;
+  cudaError_t e;
+  if (d == 64) {
+    e = set_smem(colsum_kernel<64>, ColsumCfg<64>::SMEM);
+    if (e != cudaSuccess) return e;
+    colsum_kernel<64><<<dim3(ng, BH), 224, ColsumCfg<64>::SMEM, s>>>(c);
+  } else {
+    e = set_smem(colsum_kernel<128>, ColsumCfg<128>::SMEM);
+    if (e != cudaSuccess) return e;
+    colsum_kernel<128><<<dim3(ng, BH), 224, ColsumCfg<128>::SMEM, s>>>(c);
+  }
+  e = cudaGetLastError();
+  if (e != cudaSuccess) return e;
+  topk_kernel<<<BH * ng, kTopkThreads, 0, s>>>(at<float>(ws, w.colsum), N, k, kv_idx);
+  return cudaGetLastError();
+}
+
+cudaError_t run_residual(const void *Q, const void *K, const void *V, const int32_t *perm,
+                         const int32_t *kv_idx, int BH, int N, int d, int G, int k, float scale,
+                         float *residual, void *ws, const PlanWs &w, cudaStream_t s) {
+  AttnArgs a = base_args(Q, K, V, N, scale);
+  a.G = G;
+  a.k = k;
+  a.n_groups = (N + G - 1) / G;
+  a.perm = perm;
+  a.kv_idx = kv_idx;
+  a.O32_in = at<float>(ws, w.O32);
+  a.R_out = residual;
+  return launch_attn_d<kModePlanResid>(d, a, a.n_groups, BH, s);
+}
+
+mcs_status check_common(const void *Q, const void *K, const void *V, int B, int H, int N, int d,
+                        float scale) {
+  if (!Q || !K || !V) return MCS_ERR_INVALID_ARG;
+  if (!aligned16(Q) || !aligned16(K) || !aligned16(V)) return MCS_ERR_INVALID_ARG;
+  if (!shape_ok(B, H, N, d)) return MCS_ERR_INVALID_ARG;
+  if (!(scale > 0.f) || !(scale < INFINITY)) return MCS_ERR_INVALID_ARG;
+  if (!d_ok(d)) return MCS_ERR_UNSUPPORTED;
+  return MCS_OK;
+}
+
+mcs_status check_ws(void *ws, size_t bytes, size_t need) {
+  if (!ws || bytes < need || (reinterpret_cast<uintptr_t>(ws) & 255u)) return MCS_ERR_WORKSPACE;
+  return MCS_OK;
+}
+
+}  // namespace
+
+// ============================================================================ C ABI
+
+extern "C" {
+
+int mcs_abi_version(void) { return MCS_ABI_VERSION; }
+
+const char *mcs_status_string(mcs_status s) {
+  switch (s) {
+    case MCS_OK: return "MCS_OK";
+    case MCS_ERR_INVALID_ARG: return "MCS_ERR_INVALID_ARG";
+    case MCS_ERR_UNSUPPORTED: return "MCS_ERR_UNSUPPORTED";
+    case MCS_ERR_WORKSPACE: return "MCS_ERR_WORKSPACE";
+    case MCS_ERR_CUDA: return "MCS_ERR_CUDA";
+    case MCS_ERR_TIMEOUT: return "MCS_ERR_TIMEOUT";
+    case MCS_ERR_BAD_META: return "MCS_ERR_BAD_META";
+  }
+  return "MCS_ERR_UNKNOWN";
+}
+
+mcs_status mcs_meta_init(mcs_meta *meta, int B, int H, int N, int d, int G, int k) {
+  if (!meta) return MCS_ERR_INVALID_ARG;
+  if (!shape_ok(B, H, N, d) || k < 1) return MCS_ERR_INVALID_ARG;
+  if (!d_ok(d) || !g_ok(G)) return MCS_ERR_UNSUPPORTED;
+  meta->B = B;
+  meta->H = H;
+  meta->N = N;
+  meta->d = d;
+  meta->G = G;
+  meta->k = k < N ? k : N;
+  meta->n_groups = (N + G - 1) / G;
+  return MCS_OK;
+}
+
+size_t mcs_plan_workspace_size(int B, int H, int N, int d, int G, int k) {
+  if (!shape_ok(B, H, N, d) || !d_ok(d) || !g_ok(G) || k < 1) return 0;
+  return plan_ws(B, H, N, d, G).total;
+}
+
+mcs_status mcs_plan_group(const void *Q, int B, int H, int N, int d, int32_t *perm, void *workspace,
+                          size_t workspace_bytes, mcs_stream_t stream) {
+  mcs_status st = check_common(Q, Q, Q, B, H, N, d, 1.f);
+  if (st != MCS_OK) return st;
+  if (!perm) return MCS_ERR_INVALID_ARG;
+  const PlanWs w = plan_ws(B, H, N, d, 128);
+  // grouping needs only the part of the workspace before the statistics
+  if ((st = check_ws(workspace, workspace_bytes, w.row_m)) != MCS_OK) return st;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  const int BH = B * H;
+  return cuda_status(d == 64 ? run_group<64>(Q, BH, N, perm, workspace, w, s)
+                             : run_group<128>(Q, BH, N, perm, workspace, w, s));
+}
+
+mcs_status mcs_plan_select(const void *Q, const void *K, const int32_t *perm, int B, int H, int N, int d,
+                           int G, int k, float scale, int32_t *kv_idx, void *workspace,
+                           size_t workspace_bytes, mcs_stream_t stream) {
+  mcs_status st = check_common(Q, K, K, B, H, N, d, scale);
+  if (st != MCS_OK) return st;
+  if (!perm || !kv_idx || k < 1) return MCS_ERR_INVALID_ARG;
+  if (!g_ok(G)) return MCS_ERR_UNSUPPORTED;
+  const PlanWs w = plan_ws(B, H, N, d, G);
+  if ((st = check_ws(workspace, workspace_bytes, w.total)) != MCS_OK) return st;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  const int BH = B * H;
+  const int kk = k < N ? k : N;
+  // statistics pass needs V only for its (discarded) output: use K as V
+  cudaError_t e = run_plan_dense(Q, K, K, BH, N, d, scale, nullptr, workspace, w, s);
+  if (e == cudaSuccess) e = run_select(Q, K, perm, BH, N, d, G, kk, scale, kv_idx, workspace, w, s);
+  return cuda_status(e);
+}
+
+mcs_status mcs_plan_residual(const void *Q, const void *K, const void *V, const int32_t *perm,
+                             const int32_t *kv_idx, int B, int H, int N, int d, int G, int k, float scale,
+                             float *residual, void *O_dense, void *workspace, size_t workspace_bytes,
+                             mcs_stream_t stream) {
+  mcs_status st = check_common(Q, K, V, B, H, N, d, scale);
+  if (st != MCS_OK) return st;
+  if (!perm || !kv_idx || !residual || k < 1) return MCS_ERR_INVALID_ARG;
+  if (!aligned16(residual) || (O_dense && !aligned16(O_dense))) return MCS_ERR_INVALID_ARG;
+  if (!g_ok(G)) return MCS_ERR_UNSUPPORTED;
+  const PlanWs w = plan_ws(B, H, N, d, G);
+  if ((st = check_ws(workspace, workspace_bytes, w.total)) != MCS_OK) return st;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  const int BH = B * H;
+  const int kk = k < N ? k : N;
+  cudaError_t e = run_plan_dense(Q, K, V, BH, N, d, scale, O_dense, workspace, w, s);
+  if (e == cudaSuccess) e = run_residual(Q, K, V, perm, kv_idx, BH, N, d, G, kk, scale, residual, workspace, w, s);
+  return cuda_status(e);
+}
+
+mcs_status mcs_plan(const void *Q, const void *K, const void *V, int B, int H, int N, int d, int G, int k,
+                    float scale, mcs_meta *meta, void *O_dense, void *workspace, size_t workspace_bytes,
+                    mcs_stream_t stream) {
+  mcs_status st = check_common(Q, K, V, B, H, N, d, scale);
+  if (st != MCS_OK) return st;
+  if (!meta || !meta->perm || !meta->kv_idx || !meta->residual) return MCS_ERR_INVALID_ARG;
+  if (!aligned16(meta->residual) || (O_dense && !aligned16(O_dense))) return MCS_ERR_INVALID_ARG;
+  if ((st = mcs_meta_init(meta, B, H, N, d, G, k)) != MCS_OK) return st;
+  const PlanWs w = plan_ws(B, H, N, d, G);
+  if ((st = check_ws(workspace, workspace_bytes, w.total)) != MCS_OK) return st;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  const int BH = B * H;
+  cudaError_t e = d == 64 ? run_group<64>(Q, BH, N, meta->perm, workspace, w, s)
+                          : run_group<128>(Q, BH, N, meta->perm, workspace, w, s);
+  if (e == cudaSuccess) e = run_plan_dense(Q, K, V, BH, N, d, scale, O_dense, workspace, w, s);
+  if (e == cudaSuccess)
+    e = run_select(Q, K, meta->perm, BH, N, d, G, meta->k, scale, meta->kv_idx, workspace, w, s);
+  if (e == cudaSuccess)
+    e = run_residual(Q, K, V, meta->perm, meta->kv_idx, BH, N, d, G, meta->k, scale, meta->residual,
+                     workspace, w, s);
+  return cuda_status(e);
+}
+
+mcs_status mcs_sparse_step(const void *Q, const void *K, const void *V, const mcs_meta *meta, float scale,
+                           void *O, mcs_stream_t stream) {
+  if (!meta) return MCS_ERR_INVALID_ARG;
+  mcs_status st = check_common(Q, K, V, meta->B, meta->H, meta->N, meta->d, scale);
+  if (st != MCS_OK) return st;
+  if (!O || !aligned16(O) || !meta->perm || !meta->kv_idx || !meta->residual) return MCS_ERR_INVALID_ARG;
+  if (!aligned16(meta->residual)) return MCS_ERR_INVALID_ARG;
+  if (!g_ok(meta->G)) return MCS_ERR_UNSUPPORTED;
+  if (meta->k < 1 || meta->k > meta->N || meta->n_groups != (meta->N + meta->G - 1) / meta->G)
+    return MCS_ERR_INVALID_ARG;
+  AttnArgs a = base_args(Q, K, V, meta->N, scale);
+  a.G = meta->G;
+  a.k = meta->k;
+  a.n_groups = meta->n_groups;
+  a.perm = meta->perm;
+  a.kv_idx = meta->kv_idx;
+  a.residual = meta->residual;
+  a.O = static_cast<bf16 *>(O);
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  return cuda_status(launch_attn_d<kModeStep>(meta->d, a, meta->n_groups, meta->B * meta->H, s));
+}
+
+mcs_status mcs_dense(const void *Q, const void *K, const void *V, int B, int H, int N, int d, float scale,
+                     void *O, mcs_stream_t stream) {
+  mcs_status st = check_common(Q, K, V, B, H, N, d, scale);
+  if (st != MCS_OK) return st;
+  if (!O || !aligned16(O)) return MCS_ERR_INVALID_ARG;
+  AttnArgs a = base_args(Q, K, V, N, scale);
+  a.O = static_cast<bf16 *>(O);
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  return cuda_status(launch_attn_d<kModeDense>(d, a, (N + 127) / 128, B * H, s));
+}
+
+size_t mcs_validate_workspace_size(int B, int H, int N) {
+  if (B < 1 || H < 1 || N < 1) return 0;
+  const size_t bits = static_cast<size_t>(B) * H * N;
+  return align256(256 + ((bits + 31) / 32) * 4);
+}
+
+mcs_status mcs_validate_meta(const mcs_meta *meta, void *workspace, size_t workspace_bytes, int *first_bad,
+                             mcs_stream_t stream) {
+  if (first_bad) *first_bad = 0;
+  if (!meta || !meta->perm || !meta->kv_idx || !meta->residual) return MCS_ERR_INVALID_ARG;
+  if (!shape_ok(meta->B, meta->H, meta->N, meta->d) || !d_ok(meta->d) || !g_ok(meta->G))
+    return MCS_ERR_INVALID_ARG;
+  if (meta->k < 1 || meta->k > meta->N || meta->n_groups != (meta->N + meta->G - 1) / meta->G)
+    return MCS_ERR_INVALID_ARG;
+  const size_t need = mcs_validate_workspace_size(meta->B, meta->H, meta->N);
+  mcs_status st = check_ws(workspace, workspace_bytes, need);
+  if (st != MCS_OK) return st;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  const int BH = meta->B * meta->H;
+  int *bad = static_cast<int *>(workspace);
+  unsigned *seen = reinterpret_cast<unsigned *>(static_cast<uint8_t *>(workspace) + 256);
+  const int init = INT_MAX;
+  cudaError_t e = cudaMemcpyAsync(bad, &init, sizeof(int), cudaMemcpyHostToDevice, s);
+  if (e == cudaSuccess) e = cudaMemsetAsync(seen, 0, need - 256, s);
+  if (e != cudaSuccess) return MCS_ERR_CUDA;
+  const int grid = 148 * 8;
+  perm_mark_kernel<<<grid, 256, 0, s>>>(meta->perm, meta->N, BH, seen, bad);
+  kv_check_kernel<<<grid, 256, 0, s>>>(meta->kv_idx, meta->N, meta->k,
+                                       static_cast<size_t>(BH) * meta->n_groups, bad);
+  residual_check_kernel<<<grid, 256, 0, s>>>(meta->residual,
+                                             static_cast<size_t>(BH) * meta->N * meta->d, bad);
+  if (cudaGetLastError() != cudaSuccess) return MCS_ERR_CUDA;
+  int h = INT_MAX;
+  e = cudaMemcpyAsync(&h, bad, sizeof(int), cudaMemcpyDeviceToHost, s);
+  if (e == cudaSuccess) e = cudaStreamSynchronize(s);
+  if (e != cudaSuccess) return MCS_ERR_CUDA;
+  if (h == INT_MAX) return MCS_OK;
+  if (first_bad) *first_bad = h;
+  return MCS_ERR_BAD_META;
+}
+
+mcs_status mcs_last_device_status(mcs_stream_t stream) {
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  unsigned *p = status_ptr();
+  if (!p) return MCS_ERR_CUDA;
+  unsigned h = 0;
+  cudaError_t e = cudaMemcpyAsync(&h, p, sizeof(unsigned), cudaMemcpyDeviceToHost, s);
+  if (e == cudaSuccess) e = cudaMemsetAsync(p, 0, sizeof(unsigned), s);
+  if (e == cudaSuccess) e = cudaStreamSynchronize(s);
+  if (e != cudaSuccess) return MCS_ERR_CUDA;
+  return h == 0 ? MCS_OK : static_cast<mcs_status>(h);
+}
+
+void mcs_set_wait_limit_ns(uint64_t ns) { g_wait_ns = ns ? ns : 4000000000ull; }
+
+// Self-test of the bounded wait (declared in mcs.h).
+mcs_status mcs_selftest_wait_timeout(uint64_t limit_ns, mcs_stream_t stream) {
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  unsigned *p = status_ptr();
+  if (!p) return MCS_ERR_CUDA;
+  wait_selftest_kernel<<<1, 32, 0, s>>>(limit_ns ? limit_ns : 1000000ull, p);
+  return cuda_status(cudaGetLastError());
+}
+
+}  // extern "C"

@@ -176,3 +176,13 @@ def random_metadata_head(w: Workload, bh: int, r_scale: float = 0.1):
         kv[g] = np.sort(rng.choice(N, size=k, replace=False)).astype(np.int32)
     res = (r_scale * rng.standard_normal((N, w.d))).astype(np.float32)
     return perm, kv, res
+
+
+def random_qkv(B: int, H: int, N: int, d: int, seed: int = 0, q_std: float = 1.0):
+    """Plain Gaussian Q, K, V (bf16 bit patterns, [B, H, N, d]) for shape
+    sweeps that need no DiT structure: Q ~ q_std * N(0, 1), K, V ~ N(0, 1)."""
+    rng = np.random.default_rng(np.random.SeedSequence(entropy=seed, spawn_key=(99, B, H, N, d)))
+    q = (q_std * rng.standard_normal((B, H, N, d))).astype(np.float32)
+    k = rng.standard_normal((B, H, N, d), dtype=np.float32)
+    v = rng.standard_normal((B, H, N, d), dtype=np.float32)
+    return bf16_round(q), bf16_round(k), bf16_round(v)

@@ -25,3 +25,11 @@ def pytest_collection_modifyitems(config, items):
     for it in items:
         if "gpu" in it.keywords:
             it.add_marker(skip)
+
+
+@pytest.fixture(scope="session", autouse=True)
+def _built_library():
+    """Make sure the in-tree CUDA library matches the sources (nvcc only; no GPU)."""
+    from sparse_attention_diffusion_mcs_b200 import build
+    build.build()
+    yield

@@ -1,0 +1,49 @@
+"""Helpers shared by the GPU parity tests: device upload of bf16 bit patterns
+and the comparisons the tolerances are stated for."""
+import numpy as np
+import torch
+
+# Tolerances (bf16 outputs; fp32 residual), stated once.
+OUT_MAX_ABS = 2e-2
+OUT_REL_L2 = 1e-2
+RES_REL_L2 = 1e-3
+KV_THRESHOLD_REL = 1e-4
+
+
+def dev_bf16(u16: np.ndarray) -> torch.Tensor:
+    return torch.from_numpy(np.ascontiguousarray(u16).view(np.int16)).view(torch.bfloat16).cuda()
+
+
+def host(t: torch.Tensor) -> np.ndarray:
+    return t.detach().float().cpu().numpy().astype(np.float64)
+
+
+def assert_out_close(got: np.ndarray, ref: np.ndarray, what: str):
+    err = float(np.abs(got - ref).max())
+    rel = float(np.linalg.norm(got - ref) / max(np.linalg.norm(ref), 1e-30))
+    assert err <= OUT_MAX_ABS and rel <= OUT_REL_L2, f"{what}: max-abs {err:.3e} rel-L2 {rel:.3e}"
+    return err, rel
+
+
+def assert_residual_close(got: np.ndarray, ref: np.ndarray, what: str):
+    rel = float(np.linalg.norm(got - ref) / max(np.linalg.norm(ref), 1e-30))
+    assert rel <= RES_REL_L2, f"{what}: residual rel-L2 {rel:.3e}"
+    return rel
+
+
+def kv_sets_agree(got_idx: np.ndarray, score_row: np.ndarray, k: int) -> int:
+    """GPU kv set vs the oracle score row: the sets may differ only in keys
+    whose score lies within KV_THRESHOLD_REL of the k-th largest score.
+    Also checks the GPU list is strictly ascending.  Returns #differences."""
+    got_idx = np.asarray(got_idx)
+    assert np.all(np.diff(got_idx) > 0), "kv indices not strictly ascending"
+    n = score_row.shape[0]
+    kk = min(k, n)
+    order = np.lexsort((np.arange(n), -score_row))
+    ref = set(order[:kk].tolist())
+    thr = score_row[order[kk - 1]]
+    diff = ref.symmetric_difference(set(got_idx.tolist()))
+    for j in diff:
+        assert abs(score_row[j] - thr) <= KV_THRESHOLD_REL * abs(thr), (
+            f"key {j}: score {score_row[j]:.6e} vs k-th {thr:.6e}")
+    return len(diff)

@@ -1,0 +1,128 @@
+"""The C ABI: the library loads without a GPU, exports every entry point the
+header declares, and rejects bad arguments on the host with the documented
+status codes before touching CUDA."""
+import ctypes
+import os
+import re
+
+import pytest
+
+from sparse_attention_diffusion_mcs_b200 import _lib
+from sparse_attention_diffusion_mcs_b200 import build as _build
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "mcs.h")
+
+OK, INVALID, UNSUPPORTED, WORKSPACE = 0, 1, 2, 3
+FAKE = 0x10000   # 16-byte aligned non-null address; never dereferenced on these paths
+
+
+@pytest.fixture(scope="module")
+def L():
+    _build.build()
+    return _lib.lib()
+
+
+def declared_functions():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(mcs_[a-z_0-9]+)\s*\(", text)))
+
+
+def test_every_declared_symbol_is_exported_and_bound(L):
+    names = declared_functions()
+    assert len(names) >= 15
+    for n in names:
+        assert hasattr(L, n), n
+        assert n in _lib.PROTOTYPES, n
+    assert set(_lib.PROTOTYPES) == set(names)
+
+
+def test_version_and_status_strings(L):
+    assert L.mcs_abi_version() == 1
+    for code, name in _lib.STATUS_NAMES.items():
+        assert L.mcs_status_string(code).decode() == name
+
+
+def test_meta_init_clamps_k_and_checks(L):
+    m = _lib.McsMeta()
+    assert L.mcs_meta_init(ctypes.byref(m), 1, 24, 32760, 128, 128, 1638) == OK
+    assert (m.k, m.n_groups) == (1638, 256)
+    assert L.mcs_meta_init(ctypes.byref(m), 1, 1, 100, 64, 64, 5000) == OK
+    assert (m.k, m.n_groups) == (100, 2)
+    assert L.mcs_meta_init(ctypes.byref(m), 1, 1, 100, 96, 64, 5) == UNSUPPORTED
+    assert L.mcs_meta_init(ctypes.byref(m), 1, 1, 100, 64, 32, 5) == UNSUPPORTED
+    assert L.mcs_meta_init(ctypes.byref(m), 1, 1, 0, 64, 64, 5) == INVALID
+    assert L.mcs_meta_init(ctypes.byref(m), 1, 1, 100, 64, 64, 0) == INVALID
+    assert L.mcs_meta_init(None, 1, 1, 100, 64, 64, 5) == INVALID
+
+
+def test_workspace_size(L):
+    assert L.mcs_plan_workspace_size(1, 24, 32760, 128, 128, 1638) > 24 * 256 * 32760 * 4
+    assert L.mcs_plan_workspace_size(1, 1, 100, 96, 128, 5) == 0
+    assert L.mcs_plan_workspace_size(0, 1, 100, 64, 128, 5) == 0
+    assert L.mcs_validate_workspace_size(1, 2, 1024) >= 2 * 1024 // 8
+
+
+def test_dense_argument_errors(L):
+    s = None
+    assert L.mcs_dense(None, FAKE, FAKE, 1, 1, 128, 64, 0.125, FAKE, s) == INVALID
+    assert L.mcs_dense(FAKE, FAKE, FAKE, 1, 1, 128, 64, 0.125, None, s) == INVALID
+    assert L.mcs_dense(FAKE + 8, FAKE, FAKE, 1, 1, 128, 64, 0.125, FAKE, s) == INVALID
+    assert L.mcs_dense(FAKE, FAKE, FAKE, 1, 1, 128, 96, 0.125, FAKE, s) == UNSUPPORTED
+    assert L.mcs_dense(FAKE, FAKE, FAKE, 1, 1, 0, 64, 0.125, FAKE, s) == INVALID
+    assert L.mcs_dense(FAKE, FAKE, FAKE, 1, 1, 128, 64, 0.0, FAKE, s) == INVALID
+    assert L.mcs_dense(FAKE, FAKE, FAKE, 1, 1, 128, 64, float("nan"), FAKE, s) == INVALID
+    assert L.mcs_dense(FAKE, FAKE, FAKE, 70000, 1, 128, 64, 0.1, FAKE, s) == INVALID
+
+
+def test_plan_argument_errors(L):
+    m = _lib.McsMeta()
+    m.perm, m.kv_idx, m.residual = FAKE, FAKE, FAKE
+    need = L.mcs_plan_workspace_size(1, 2, 1024, 64, 64, 128)
+    args = lambda ws, nbytes, G=64, d=64: (FAKE, FAKE, FAKE, 1, 2, 1024, d, G, 128, 0.125,
+                                           ctypes.byref(m), None, ws, nbytes, None)
+    assert L.mcs_plan(*args(None, need)) == WORKSPACE
+    assert L.mcs_plan(*args(FAKE, need - 1)) == WORKSPACE
+    assert L.mcs_plan(*args(FAKE + 16, need)) == WORKSPACE         # not 256-byte aligned
+    assert L.mcs_plan(*args(FAKE, need, G=96)) == UNSUPPORTED
+    assert L.mcs_plan(*args(FAKE, need, d=80)) == UNSUPPORTED
+    m.residual = None
+    assert L.mcs_plan(*args(FAKE, need)) == INVALID
+    assert L.mcs_plan_group(None, 1, 1, 10, 64, FAKE, FAKE, 1 << 20, None) == INVALID
+    assert L.mcs_plan_select(FAKE, FAKE, None, 1, 1, 10, 64, 64, 4, 0.1, FAKE, FAKE, 1 << 20,
+                             None) == INVALID
+    assert L.mcs_plan_residual(FAKE, FAKE, FAKE, FAKE, FAKE, 1, 1, 10, 64, 64, 4, 0.1, None, None,
+                               FAKE, 1 << 20, None) == INVALID
+
+
+def test_sparse_step_argument_errors(L):
+    m = _lib.McsMeta()
+    assert L.mcs_meta_init(ctypes.byref(m), 1, 2, 1024, 64, 64, 128) == OK
+    m.perm, m.kv_idx, m.residual = FAKE, FAKE, FAKE
+    assert L.mcs_sparse_step(FAKE, FAKE, FAKE, None, 0.125, FAKE, None) == INVALID
+    assert L.mcs_sparse_step(FAKE, FAKE, FAKE, ctypes.byref(m), 0.125, None, None) == INVALID
+    m.n_groups = 3
+    assert L.mcs_sparse_step(FAKE, FAKE, FAKE, ctypes.byref(m), 0.125, FAKE, None) == INVALID
+    m.n_groups = 16
+    m.k = 2000
+    assert L.mcs_sparse_step(FAKE, FAKE, FAKE, ctypes.byref(m), 0.125, FAKE, None) == INVALID
+    m.k = 128
+    m.G = 100
+    assert L.mcs_sparse_step(FAKE, FAKE, FAKE, ctypes.byref(m), 0.125, FAKE, None) == UNSUPPORTED
+
+
+def test_validate_argument_errors(L):
+    m = _lib.McsMeta()
+    assert L.mcs_meta_init(ctypes.byref(m), 1, 2, 1024, 64, 64, 128) == OK
+    code = ctypes.c_int(-1)
+    assert L.mcs_validate_meta(ctypes.byref(m), FAKE, 1 << 20, ctypes.byref(code), None) == INVALID
+    m.perm, m.kv_idx, m.residual = FAKE, FAKE, FAKE
+    assert L.mcs_validate_meta(ctypes.byref(m), None, 1 << 20, ctypes.byref(code), None) == WORKSPACE
+
+
+def test_binding_refuses_to_run_without_library(monkeypatch, tmp_path):
+    monkeypatch.setattr(_lib, "LIB_PATH", str(tmp_path / "missing.so"))
+    monkeypatch.setattr(_lib, "_lib", None)
+    with pytest.raises(ImportError):
+        _lib.lib()
