@@ -1,0 +1,450 @@
+#!/usr/bin/env python
+"""Benchmark of the MC-Sparse hot path on B200.
+
+One timed step = one pass of the whole hot path over one synthetic DiT layer:
+the metadata plan on the step-s inputs (grouping, exact statistics + dense
+output, group scores, top-k, residual), the reused sparse step on the drifted
+step-(s+1) inputs, and dense attention on those same inputs (the speedup
+denominator).  Every call goes through the C ABI and is bracketed by CUDA
+events on the launching stream.
+
+The headline metric is the reused step's effective TFLOP/s (4*B*H*N*k*d per
+step); ms per reused step, per plan and per dense call, and the speedup over
+dense, are reported beside it.  Multi-GPU runs are weak-scaled: every rank
+runs its own layer (heads are independent; no collective on the data path).
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl reference]
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+import numpy as np  # noqa: E402
+
+import synth  # noqa: E402
+
+KERNELS_PER_STEP = 12   # grouping 6, stats 1, scores 1, top-k 1, residual 1, step 1, dense 1
+
+
+def parse_args():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=10)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", choices=["mcs", "reference"], default="mcs")
+    ap.add_argument("--config", type=int, default=3, help="workload id (default: 32K-token video layer)")
+    ap.add_argument("--k", type=int, default=None, help="override keys per group")
+    ap.add_argument("--G", type=int, default=None, help="override group size")
+    ap.add_argument("--cpu-seconds", type=float, default=12.0, help="CPU baseline budget")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-e2e", action="store_true")
+    return ap.parse_args()
+
+
+# ----------------------------------------------------------------------------- inputs
+
+def _gen_head(args):
+    cfg, k, G, bh, seed_shift = args
+    w = synth.workload(cfg, k=k, G=G).with_(seed=seed_shift)
+    q1, k1, v1 = synth.head_tensors(w, bh, step=1)
+    q2 = synth.drift_head(q1, w, 2, 0, bh)
+    k2 = synth.drift_head(k1, w, 2, 1, bh)
+    v2 = synth.drift_head(v1, w, 2, 2, bh)
+    return bh, (q1, k1, v1), (q2, k2, v2)
+
+
+def make_inputs(w, rank: int):
+    """Step-1 (plan) and step-2 (reused) tensors of one layer, uint16 [B,H,N,d]."""
+    import concurrent.futures as cf
+    import multiprocessing as mp
+    shape = (w.BH, w.N, w.d)
+    s1 = [np.empty(shape, np.uint16) for _ in range(3)]
+    s2 = [np.empty(shape, np.uint16) for _ in range(3)]
+    jobs = [(w.cfg_id, w.k, w.G, bh, w.seed + rank) for bh in range(w.BH)]
+    nproc = max(1, min(len(jobs), len(os.sched_getaffinity(0)), 16))
+    with cf.ProcessPoolExecutor(nproc, mp_context=mp.get_context("spawn")) as ex:
+        for bh, a, b in ex.map(_gen_head, jobs):
+            for i in range(3):
+                s1[i][bh] = a[i]
+                s2[i][bh] = b[i]
+    rs = lambda x: x.reshape(w.B, w.H, w.N, w.d)
+    return [rs(x) for x in s1], [rs(x) for x in s2]
+
+
+# ----------------------------------------------------------------------------- clocks
+
+class ClockSampler:
+    QUERY = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+             "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+             "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, uuid: str | None):
+        self.uuid = uuid
+        self.proc = None
+        self.path = os.path.join("/tmp", f"mcs_clocks_{os.getpid()}.csv")
+
+    def start(self):
+        cmd = ["nvidia-smi", f"--query-gpu={self.QUERY}", "--format=csv,noheader,nounits", "-lms", "200"]
+        if self.uuid:
+            cmd += ["-i", self.uuid]
+        try:
+            self.fh = open(self.path, "w")
+            self.proc = subprocess.Popen(cmd, stdout=self.fh, stderr=subprocess.DEVNULL)
+        except Exception:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unsampled"]}
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except Exception:
+            self.proc.kill()
+        self.fh.close()
+        sm, mx, reasons, power = [], [], set(), []
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for line in open(self.path):
+            parts = [p.strip() for p in line.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                sm.append(float(parts[1]))
+                mx.append(float(parts[2]))
+                power.append(float(parts[3]))
+            except ValueError:
+                continue
+            for nm, val in zip(names, parts[5:9]):
+                if val.lower().startswith("active"):
+                    reasons.add(nm)
+        os.unlink(self.path)
+        if not sm:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unsampled"]}
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": max(mx), "samples": len(sm),
+                "power_w_max": max(power) if power else None, "reasons": sorted(reasons)}
+
+
+# ----------------------------------------------------------------------------- peaks
+
+def measured_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        d = json.load(open(p))
+        return {"hbm_gbs": float(d["hbm_gbs"]), "bf16_tflops": float(d["bf16_tflops"]),
+                "bf16_tflops_sustained": float(d.get("bf16_tflops_sustained", d["bf16_tflops"])),
+                "source": "measured"}
+    except Exception:
+        return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0,
+                "source": "fallback"}
+
+
+# ----------------------------------------------------------------------------- CPU baseline
+
+def cpu_baseline(w, seconds: float):
+    """The fp64 oracle's reused step, timed on the host cores over a bounded
+    sample of query groups of head 0 (seeded metadata of the same shape)."""
+    from oracle import mcs_oracle as orc
+    try:
+        from threadpoolctl import threadpool_info
+        threads = max([i.get("num_threads", 1) for i in threadpool_info()] or [1])
+    except Exception:
+        threads = len(os.sched_getaffinity(0))
+    q, k, v = synth.head_tensors(w, 0, step=2)
+    perm, kv, res = synth.random_metadata_head(w, 0)
+    Qf, Kf, Vf = orc.widen_bf16(q), orc.widen_bf16(k), orc.widen_bf16(v)
+    done, flops, t0 = 0, 0.0, time.perf_counter()
+    g = 0
+    while time.perf_counter() - t0 < seconds and g < w.n_groups:
+        rows, _ = orc.reused_step_head(Qf, Kf, Vf, w.scale, perm, kv, res, w.G, groups=[g])
+        flops += 4.0 * len(rows) * min(w.k, w.N) * w.d
+        g += 1
+        done += 1
+    dt = time.perf_counter() - t0
+    return {"value": flops / dt / 1e12, "unit": "TFLOP/s", "cores": int(threads), "kind": "oracle",
+            "sample": f"reused step of {done} query groups of head 0 (of {w.BH * w.n_groups} groups), "
+                      f"fp64 NumPy, {dt:.1f} s"}
+
+
+def run_reference(args):
+    """--impl reference: the fp64 oracle on the host cores, same metric and workload."""
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return 0
+    w = synth.workload(args.config, k=args.k, G=args.G)
+    from oracle import mcs_oracle as orc
+    q, k, v = synth.head_tensors(w, 0, step=2)
+    perm, kv, res = synth.random_metadata_head(w, 0)
+    Qf, Kf, Vf = orc.widen_bf16(q), orc.widen_bf16(k), orc.widen_bf16(v)
+    groups_per_step = 4
+    def one(i):
+        gs = [(i * groups_per_step + j) % w.n_groups for j in range(groups_per_step)]
+        rows, _ = orc.reused_step_head(Qf, Kf, Vf, w.scale, perm, kv, res, w.G, groups=gs)
+        return 4.0 * len(rows) * min(w.k, w.N) * w.d
+    for i in range(args.warmup):
+        one(i)
+    t0 = time.perf_counter()
+    flops = sum(one(args.warmup + i) for i in range(args.steps))
+    dt = time.perf_counter() - t0
+    try:
+        from threadpoolctl import threadpool_info
+        threads = max([i.get("num_threads", 1) for i in threadpool_info()] or [1])
+    except Exception:
+        threads = len(os.sched_getaffinity(0))
+    val = flops / dt / 1e12
+    line = {
+        "impl": "reference", "metric": "reused-step sparse attention effective TFLOP/s",
+        "value": val, "unit": "TFLOP/s", "n_gpus": args.gpus, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": dt / args.steps * 1e3, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": workload_config(w, args.gpus),
+        "cpu_baseline": {"value": val, "unit": "TFLOP/s", "cores": int(threads), "kind": "oracle",
+                         "sample": f"{groups_per_step} query groups of head 0 per step"},
+        "e2e": {"value": val, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def workload_config(w, n):
+    return {"workload": f"{w.name}: B={w.B} H={w.H} grid={'x'.join(map(str, w.grid))} N={w.N} "
+                        f"d={w.d} G={w.G} k={w.k}",
+            "B": w.B, "H": w.H, "N": w.N, "d": w.d, "G": w.G, "k": w.k, "n_groups": w.n_groups,
+            "global_batch": w.B * n, "seq_len": w.N,
+            "l2": "inputs larger than L2 (each of Q, K, V is "
+                  f"{w.BH * w.N * w.d * 2 / 1e6:.0f} MB per step; no explicit flush)",
+            "parallelism": f"weak scaling, {n} independent layer(s), one per GPU"}
+
+
+# ----------------------------------------------------------------------------- main arm
+
+def main():
+    args = parse_args()
+    if args.impl == "reference":
+        return run_reference(args)
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    w = synth.workload(args.config, k=args.k, G=args.G)
+    # host inputs first (process pool before any CUDA work)
+    s1, s2 = make_inputs(w, rank)
+
+    import torch
+    import torch.distributed as dist
+    import sparse_attention_diffusion_mcs_b200 as mcs
+
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        from datetime import timedelta
+        dist.init_process_group("nccl", timeout=timedelta(seconds=300), device_id=dev)
+
+    up = lambda a: torch.from_numpy(a.view(np.int16)).view(torch.bfloat16).to(dev)
+    Q1, K1, V1 = (up(x) for x in s1)
+    Q2, K2, V2 = (up(x) for x in s2)
+    B, H, N, d, G, k = w.B, w.H, w.N, w.d, w.G, w.k
+    ws = mcs.alloc_workspace(B, H, N, d, G, k, dev)
+    meta = mcs.Meta.empty(B, H, N, d, G, k, dev)
+    O_dense_plan = torch.empty_like(Q1)
+    O_step = torch.empty_like(Q2)
+    O_dense = torch.empty_like(Q2)
+    stream = torch.cuda.current_stream()
+
+    stages = ["group", "stats", "scores", "topk", "residual", "step", "dense"]
+
+    def one_step(ev):
+        ev[0].record(stream)
+        mcs.plan_group(Q1, ws, out=meta.perm)
+        ev[1].record(stream)
+        mcs.plan_stats(Q1, K1, V1, G, k, w.scale, ws, out_dense=O_dense_plan)
+        ev[2].record(stream)
+        mcs.plan_scores(Q1, K1, meta.perm, G, k, ws, w.scale)
+        ev[3].record(stream)
+        mcs.plan_topk(B, H, N, d, G, k, ws, out=meta.kv_idx)
+        ev[4].record(stream)
+        mcs.plan_residual(Q1, K1, V1, meta.perm, meta.kv_idx, G, w.scale, workspace=ws,
+                          stats_done=True, out=meta.residual)
+        ev[5].record(stream)
+        mcs.sparse_step(Q2, K2, V2, meta, w.scale, out=O_step)
+        ev[6].record(stream)
+        mcs.dense(Q2, K2, V2, w.scale, out=O_dense)
+        ev[7].record(stream)
+
+    mk = lambda: [torch.cuda.Event(enable_timing=True) for _ in range(8)]
+    for _ in range(args.warmup):
+        one_step(mk())
+    torch.cuda.synchronize()
+    if mcs.last_device_status() != 0:
+        raise RuntimeError("device status after warm-up is not OK")
+
+    uuid = None
+    try:
+        uuid = "GPU-" + str(torch.cuda.get_device_properties(dev).uuid)
+    except Exception:
+        uuid = None
+    clocks = ClockSampler(uuid)
+    clocks.start()
+    time.sleep(0.3)
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    evs = [mk() for _ in range(args.steps)]
+    t_start = torch.cuda.Event(enable_timing=True)
+    t_end = torch.cuda.Event(enable_timing=True)
+    t_start.record(stream)
+    for i in range(args.steps):
+        one_step(evs[i])
+    t_end.record(stream)
+    torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    clk = clocks.stop()
+    status = mcs.last_device_status()
+    total_ms = t_start.elapsed_time(t_end)
+    per = {s: [] for s in stages}
+    for ev in evs:
+        for i, s in enumerate(stages):
+            per[s].append(ev[i].elapsed_time(ev[i + 1]))
+    mean = {s: statistics.fmean(v) for s, v in per.items()}
+
+    # max over ranks
+    vec = torch.tensor([total_ms] + [mean[s] for s in stages], dtype=torch.float64, device=dev)
+    if world > 1:
+        dist.all_reduce(vec, op=dist.ReduceOp.MAX)
+    total_ms = float(vec[0])
+    mean = {s: float(vec[1 + i]) for i, s in enumerate(stages)}
+
+    # ------------------------------------------------------------- e2e through the public API
+    e2e = None
+    if not args.no_e2e:
+        hq, hk, hv = (torch.from_numpy(x.view(np.int16)).view(torch.bfloat16).pin_memory() for x in s2)
+        ho = torch.empty(O_step.shape, dtype=torch.bfloat16).pin_memory()
+        dq, dk, dv = torch.empty_like(Q2), torch.empty_like(K2), torch.empty_like(V2)
+
+        def e2e_step():
+            dq.copy_(hq, non_blocking=True)
+            dk.copy_(hk, non_blocking=True)
+            dv.copy_(hv, non_blocking=True)
+            mcs.sparse_step(dq, dk, dv, meta, w.scale, out=O_step)
+            ho.copy_(O_step, non_blocking=True)
+
+        for _ in range(max(1, args.warmup)):
+            e2e_step()
+        torch.cuda.synchronize()
+        if world > 1:
+            dist.barrier()
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        for _ in range(args.steps):
+            e2e_step()
+        b.record(stream)
+        torch.cuda.synchronize()
+        e2e_ms = a.elapsed_time(b) / args.steps
+        t = torch.tensor([e2e_ms], dtype=torch.float64, device=dev)
+        if world > 1:
+            dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        e2e_ms = float(t[0])
+        e2e = {"value": world * w.sparse_flops / (e2e_ms * 1e-3) / 1e12, "unit": "TFLOP/s",
+               "ms_per_step": e2e_ms,
+               "h2d_bytes_per_step": int(3 * Q2.numel() * 2), "d2h_bytes_per_step": int(O_step.numel() * 2)}
+
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+    if rank != 0:
+        return 0
+
+    peaks = measured_peaks()
+    tc = peaks["bf16_tflops_sustained"]
+    BH, kk = w.BH, min(w.k, w.N)
+    bpe = 2
+    # algorithmic work per launch of each stage
+    work = {
+        "group": ("hbm", BH * N * d * bpe + BH * N * 4),
+        "stats": ("tensor", 4.0 * BH * N * N * d),
+        "scores": ("tensor", 2.0 * BH * N * N * d),
+        "topk": ("hbm", 4.0 * BH * w.n_groups * N + 4.0 * BH * w.n_groups * kk),
+        "residual": ("tensor", 4.0 * BH * N * kk * d),
+        "step": ("tensor", float(w.sparse_flops)),
+        "dense": ("tensor", float(w.dense_flops)),
+    }
+    kernels = {}
+    for s in stages:
+        bound, amt = work[s]
+        t = mean[s] * 1e-3
+        if bound == "tensor":
+            ach = amt / t / 1e12
+            kernels[s] = {"ms": mean[s], "bound": "tensor", "achieved": ach, "unit": "TFLOP/s",
+                          "frac": ach / tc}
+        else:
+            ach = amt / t / 1e9
+            kernels[s] = {"ms": mean[s], "bound": "hbm", "achieved": ach, "unit": "GB/s",
+                          "frac": ach / peaks["hbm_gbs"]}
+    dom = max(stages, key=lambda s: mean[s])
+    # the reused step also moves unique bytes: Q, K, V, O (bf16), R (fp32), indices
+    step_bytes = 4 * BH * N * d * bpe + BH * N * d * 4 + 4 * BH * w.n_groups * kk + 4 * BH * N
+    kernels["step"]["hbm_gbs"] = step_bytes / (mean["step"] * 1e-3) / 1e9
+    kernels["step"]["hbm_frac"] = kernels["step"]["hbm_gbs"] / peaks["hbm_gbs"]
+    kernels["step"]["gathered_kv_gbs"] = (BH * w.n_groups * 4.0 * kk * d) / (mean["step"] * 1e-3) / 1e9
+
+    def roof(s):
+        r = kernels[s]
+        return {"kernel": s, "bound": r["bound"], "achieved": r["achieved"],
+                "peak": tc if r["bound"] == "tensor" else peaks["hbm_gbs"], "unit": r["unit"],
+                "frac": r["frac"], "traffic": None,
+                "peak_kind": f"{peaks['source']} bf16 sustained" if r["bound"] == "tensor"
+                else f"{peaks['source']} HBM copy"}
+
+    plan_ms = sum(mean[s] for s in ["group", "stats", "scores", "topk", "residual"])
+    S, P = w.steps, len(w.plan_steps)
+    line = {
+        "metric": "reused-step sparse attention effective TFLOP/s (4*B*H*N*k*d per step), 1xB200 per rank",
+        "value": world * w.sparse_flops / (mean["step"] * 1e-3) / 1e12,
+        "unit": "TFLOP/s",
+        "n_gpus": world,
+        "steps": args.steps,
+        "warmup": args.warmup,
+        "ms_per_step": total_ms / args.steps,
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": "bf16",
+        "data": "synthetic (seeded DiT-layer generator; see DESIGN.md)",
+        "config": workload_config(w, world),
+        "reused_step_ms": mean["step"],
+        "plan_ms": plan_ms,
+        "dense_ms": mean["dense"],
+        "speedup_vs_dense": mean["dense"] / mean["step"],
+        "amortized_speedup": S * mean["dense"] / (P * plan_ms + (S - P) * mean["step"]),
+        "schedule": f"{S} denoising steps, plan at {list(w.plan_steps)}",
+        "roofline": roof("step"),
+        "roofline_dominant": roof(dom),
+        "kernels": kernels,
+        "clocks": clk,
+        "gpu_launches": KERNELS_PER_STEP * args.steps,
+        "device_status": status,
+        "peaks": peaks,
+        "context_page_speedups": {"video_dit": 1.80, "asset3d": 2.32,
+                                  "note": "end-to-end denoising, hardware not stated"},
+    }
+    if e2e is not None:
+        line["e2e"] = e2e
+    if world == 1 and not args.no_cpu_baseline:
+        line["cpu_baseline"] = cpu_baseline(w, args.cpu_seconds)
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -103,21 +103,43 @@ mcs_status mcs_plan(const void *Q, const void *K, const void *V, int B, int H, i
                     int G, int k, float scale, mcs_meta *meta, void *O_dense, void *workspace,
                     size_t workspace_bytes, mcs_stream_t stream);
 
-/* Step a1 alone: perm int32 [B,H,N].  Same workspace as mcs_plan. */
+/*
+ * The plan's steps one by one.  mcs_plan is exactly mcs_plan_group,
+ * mcs_plan_stats, mcs_plan_scores, mcs_plan_topk and mcs_plan_residual in this
+ * order on one workspace (>= mcs_plan_workspace_size(B,H,N,d,G,k) bytes).
+ * The later steps read what the earlier ones left in the workspace, so they
+ * must run in this order, on the same workspace and the same shape; any
+ * grouping perm (a permutation per head) and any valid selection may be fed
+ * in between.
+ */
+
+/* a1: perm int32 [B,H,N]. */
 mcs_status mcs_plan_group(const void *Q, int B, int H, int N, int d, int32_t *perm,
                           void *workspace, size_t workspace_bytes, mcs_stream_t stream);
 
-/* Steps a2..a4 for a given grouping `perm` (any permutation): kv_idx int32
- * [B,H,ceil(N/G),min(k,N)].  Same workspace as mcs_plan. */
-mcs_status mcs_plan_select(const void *Q, const void *K, const int32_t *perm, int B, int H,
-                           int N, int d, int G, int k, float scale, int32_t *kv_idx,
-                           void *workspace, size_t workspace_bytes, mcs_stream_t stream);
+/* a2: exact softmax row statistics over all N keys and the dense output in
+ * fp32 (split-precision P.V) into the workspace; O_dense (bf16, optional, may
+ * be NULL) receives the same dense output rounded to bf16. */
+mcs_status mcs_plan_stats(const void *Q, const void *K, const void *V, int B, int H, int N, int d,
+                          int G, int k, float scale, void *O_dense, void *workspace,
+                          size_t workspace_bytes, mcs_stream_t stream);
 
-/* Steps a2 and a5 for a given grouping and selection: residual float32
- * [B,H,N,d]; O_dense (bf16, optional) as in mcs_plan.  Same workspace. */
+/* a3: group probability sums colsum[b,h,g,j] = sum_{i in group g} P_ij into
+ * the workspace, for the grouping `perm`.  Needs mcs_plan_stats first. */
+mcs_status mcs_plan_scores(const void *Q, const void *K, const int32_t *perm, int B, int H,
+                           int N, int d, int G, int k, float scale, void *workspace,
+                           size_t workspace_bytes, mcs_stream_t stream);
+
+/* a4: per group the min(k,N) largest scores, ties to the lower key index,
+ * ascending -> kv_idx int32 [B,H,ceil(N/G),min(k,N)].  Needs mcs_plan_scores. */
+mcs_status mcs_plan_topk(int B, int H, int N, int d, int G, int k, int32_t *kv_idx,
+                         void *workspace, size_t workspace_bytes, mcs_stream_t stream);
+
+/* a5: residual float32 [B,H,N,d] = dense output (from mcs_plan_stats, same
+ * Q, K, V) minus the output renormalised over each group's kept keys. */
 mcs_status mcs_plan_residual(const void *Q, const void *K, const void *V, const int32_t *perm,
                              const int32_t *kv_idx, int B, int H, int N, int d, int G, int k,
-                             float scale, float *residual, void *O_dense, void *workspace,
+                             float scale, float *residual, void *workspace,
                              size_t workspace_bytes, mcs_stream_t stream);
 
 /*

@@ -12,7 +12,10 @@ from .api import (  # noqa: F401
     plan,
     plan_group,
     plan_residual,
+    plan_scores,
     plan_select,
+    plan_stats,
+    plan_topk,
     selftest_wait_timeout,
     set_wait_limit_ns,
     sparse_step,

@@ -40,10 +40,13 @@ PROTOTYPES = {
     "mcs_plan": (c_int, [c_vp, c_vp, c_vp, c_int, c_int, c_int, c_int, c_int, c_int, c_float,
                          PMETA, c_vp, c_vp, c_size_t, c_vp]),
     "mcs_plan_group": (c_int, [c_vp, c_int, c_int, c_int, c_int, c_vp, c_vp, c_size_t, c_vp]),
-    "mcs_plan_select": (c_int, [c_vp, c_vp, c_vp, c_int, c_int, c_int, c_int, c_int, c_int, c_float,
-                                c_vp, c_vp, c_size_t, c_vp]),
+    "mcs_plan_stats": (c_int, [c_vp, c_vp, c_vp, c_int, c_int, c_int, c_int, c_int, c_int, c_float,
+                               c_vp, c_vp, c_size_t, c_vp]),
+    "mcs_plan_scores": (c_int, [c_vp, c_vp, c_vp, c_int, c_int, c_int, c_int, c_int, c_int, c_float,
+                                c_vp, c_size_t, c_vp]),
+    "mcs_plan_topk": (c_int, [c_int, c_int, c_int, c_int, c_int, c_int, c_vp, c_vp, c_size_t, c_vp]),
     "mcs_plan_residual": (c_int, [c_vp, c_vp, c_vp, c_vp, c_vp, c_int, c_int, c_int, c_int, c_int,
-                                  c_int, c_float, c_vp, c_vp, c_vp, c_size_t, c_vp]),
+                                  c_int, c_float, c_vp, c_vp, c_size_t, c_vp]),
     "mcs_sparse_step": (c_int, [c_vp, c_vp, c_vp, PMETA, c_float, c_vp, c_vp]),
     "mcs_dense": (c_int, [c_vp, c_vp, c_vp, c_int, c_int, c_int, c_int, c_float, c_vp, c_vp]),
     "mcs_validate_workspace_size": (c_size_t, [c_int, c_int, c_int]),

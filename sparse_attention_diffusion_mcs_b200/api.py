@@ -108,45 +108,84 @@ def plan(Q, K, V, G: int, k: int, scale: Optional[float] = None,
     return (meta, out_dense) if (return_dense or out_dense is not None) else meta
 
 
-def plan_group(Q, workspace: Optional[torch.Tensor] = None) -> torch.Tensor:
+def plan_group(Q, workspace: Optional[torch.Tensor] = None,
+               out: Optional[torch.Tensor] = None) -> torch.Tensor:
     """Step a1 alone: int32 perm [B, H, N]."""
     _check_qkv(Q)
     B, H, N, d = Q.shape
-    perm = torch.empty((B, H, N), dtype=torch.int32, device=Q.device)
+    perm = out if out is not None else torch.empty((B, H, N), dtype=torch.int32, device=Q.device)
     ws = _ws(workspace, B, H, N, d, 128, 1, Q.device)
     check(lib().mcs_plan_group(_ptr(Q), B, H, N, d, _ptr(perm), _ptr(ws), ws.numel(), _stream()),
           "mcs_plan_group")
     return perm
 
 
-def plan_select(Q, K, perm, G: int, k: int, scale: Optional[float] = None,
-                workspace: Optional[torch.Tensor] = None) -> torch.Tensor:
-    """Steps a2-a4 for a given grouping: int32 kv_idx [B, H, n_groups, min(k, N)]."""
+def plan_stats(Q, K, V, G: int, k: int, scale: Optional[float] = None,
+               workspace: Optional[torch.Tensor] = None, return_dense: bool = False,
+               out_dense: Optional[torch.Tensor] = None):
+    """Step a2 into the workspace (row statistics, fp32 dense output).
+    Returns the workspace, or (workspace, O_dense bf16)."""
+    _check_qkv(Q, K, V)
+    B, H, N, d = Q.shape
+    ws = _ws(workspace, B, H, N, d, G, k, Q.device)
+    od = out_dense if out_dense is not None else (torch.empty_like(Q) if return_dense else None)
+    check(lib().mcs_plan_stats(_ptr(Q), _ptr(K), _ptr(V), B, H, N, d, G, k, _scale(d, scale), _ptr(od),
+                               _ptr(ws), ws.numel(), _stream()), "mcs_plan_stats")
+    return (ws, od) if (return_dense or out_dense is not None) else ws
+
+
+def plan_scores(Q, K, perm, G: int, k: int, workspace: torch.Tensor,
+                scale: Optional[float] = None) -> None:
+    """Step a3 into the workspace (needs plan_stats on the same workspace)."""
     _check_qkv(Q, K)
     B, H, N, d = Q.shape
     perm = perm.to(torch.int32).contiguous()
+    check(lib().mcs_plan_scores(_ptr(Q), _ptr(K), _ptr(perm), B, H, N, d, G, k, _scale(d, scale),
+                                _ptr(workspace), workspace.numel(), _stream()), "mcs_plan_scores")
+
+
+def plan_topk(B: int, H: int, N: int, d: int, G: int, k: int, workspace: torch.Tensor,
+              out: Optional[torch.Tensor] = None) -> torch.Tensor:
+    """Step a4 (needs plan_scores on the same workspace): int32 kv_idx."""
     kk = min(int(k), N)
-    kv = torch.empty((B, H, -(-N // G), kk), dtype=torch.int32, device=Q.device)
-    ws = _ws(workspace, B, H, N, d, G, k, Q.device)
-    check(lib().mcs_plan_select(_ptr(Q), _ptr(K), _ptr(perm), B, H, N, d, G, k, _scale(d, scale),
-                                _ptr(kv), _ptr(ws), ws.numel(), _stream()), "mcs_plan_select")
-    return kv
+    if out is None:
+        out = torch.empty((B, H, -(-N // G), kk), dtype=torch.int32, device=workspace.device)
+    check(lib().mcs_plan_topk(B, H, N, d, G, k, _ptr(out), _ptr(workspace), workspace.numel(),
+                              _stream()), "mcs_plan_topk")
+    return out
+
+
+def plan_select(Q, K, perm, G: int, k: int, scale: Optional[float] = None,
+                workspace: Optional[torch.Tensor] = None) -> torch.Tensor:
+    """Steps a2-a4 for a given grouping: int32 kv_idx [B, H, n_groups, min(k, N)]."""
+    B, H, N, d = Q.shape
+    ws = plan_stats(Q, K, K, G, k, scale, workspace)
+    plan_scores(Q, K, perm, G, k, ws, scale)
+    return plan_topk(B, H, N, d, G, k, ws)
 
 
 def plan_residual(Q, K, V, perm, kv_idx, G: int, scale: Optional[float] = None,
-                  workspace: Optional[torch.Tensor] = None, return_dense: bool = False):
-    """Steps a2 and a5 for a given grouping and selection: float32 residual."""
+                  workspace: Optional[torch.Tensor] = None, stats_done: bool = False,
+                  return_dense: bool = False, out: Optional[torch.Tensor] = None):
+    """Step a5 (running a2 first unless stats_done): float32 residual."""
     _check_qkv(Q, K, V)
     B, H, N, d = Q.shape
     perm = perm.to(torch.int32).contiguous()
     kv_idx = kv_idx.to(torch.int32).contiguous()
     k = kv_idx.shape[-1]
-    res = torch.empty((B, H, N, d), dtype=torch.float32, device=Q.device)
-    od = torch.empty_like(Q) if return_dense else None
-    ws = _ws(workspace, B, H, N, d, G, k, Q.device)
+    od = None
+    if stats_done:
+        if workspace is None:
+            raise ValueError("stats_done needs the workspace plan_stats filled")
+        ws = workspace
+    elif return_dense:
+        ws, od = plan_stats(Q, K, V, G, k, scale, workspace, return_dense=True)
+    else:
+        ws = plan_stats(Q, K, V, G, k, scale, workspace)
+    res = out if out is not None else torch.empty((B, H, N, d), dtype=torch.float32, device=Q.device)
     check(lib().mcs_plan_residual(_ptr(Q), _ptr(K), _ptr(V), _ptr(perm), _ptr(kv_idx), B, H, N, d,
-                                  G, k, _scale(d, scale), _ptr(res), _ptr(od), _ptr(ws),
-                                  ws.numel(), _stream()), "mcs_plan_residual")
+                                  G, k, _scale(d, scale), _ptr(res), _ptr(ws), ws.numel(), _stream()),
+          "mcs_plan_residual")
     return (res, od) if return_dense else res
 
 

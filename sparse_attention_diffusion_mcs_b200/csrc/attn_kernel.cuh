@@ -1,4 +1,4 @@
-// attn_kernel.cuh -- one tcgen05 / TMEM flash-attention kernel, four uses.
+// attn_kernel.cuh -- one tcgen05 / TMEM / TMA flash-attention kernel, four uses.
 //
 //  kModeDense     O = softmax(scale Q K^T) V over all N keys, bf16 out.  The
 //                 dense baseline of the pages ("relative to dense attention",
@@ -22,7 +22,10 @@
 // CTA = 128 query rows x all KV tiles of 128 keys; 224 threads:
 //   warps 0-3  softmax + epilogue; thread t owns query row t = TMEM lane t
 //   warp  4    TMEM allocation and the single UMMA-issuing thread
-//   warps 5-6  gather: cp.async 16-byte vectors into 128B-swizzled tiles
+//   warp  5    Q and K producer (TMA), warp 6 V producer (TMA)
+// Rows listed by index (sparse modes) arrive through TMA tile::gather4, four
+// 128-byte rows per instruction; contiguous tiles (dense modes) through 3D
+// tile loads whose row bound is the head, so the ragged tail is zero-filled.
 // TMEM: S double buffer (2 x 128 fp32 columns) + O (D columns).
 // Synchronisation is mbarrier-only inside the loops; every wait is bounded.
 #pragma once
@@ -33,8 +36,8 @@ namespace mcs {
 
 enum AttnMode : int { kModeDense = 0, kModeStep = 1, kModePlanDense = 2, kModePlanResid = 3 };
 
-struct AttnArgs {
-  const bf16 *Q, *K, *V;   // [BH, N, D]
+struct alignas(64) AttnArgs {
+  CUtensorMap tmQ, tmK, tmV;   // gather maps (2D, box {64,1}) or tile maps (3D, box {64,128,1})
   int N;                   // tokens per head
   int G;                   // query group size (sparse modes)
   int k;                   // kept keys per group (sparse modes), <= N
@@ -57,29 +60,30 @@ struct AttnCfg {
   static constexpr int BM = 128, BN = 128;
   static constexpr bool kSparse = (MODE == kModeStep || MODE == kModePlanResid);
   static constexpr bool kSplit = (MODE == kModePlanDense || MODE == kModePlanResid);
-  static constexpr int NST = (D == 64) ? 3 : 2;             // K ring and V ring depth
+  static constexpr int NK = D == 64 ? (kSplit ? 4 : 5) : (kSplit ? 2 : 3);   // K ring depth
+  static constexpr int NV = D == 64 ? (kSplit ? 4 : 5) : 2;                  // V ring depth
   static constexpr int Q_BYTES = BM * D * 2;
   static constexpr int KV_BYTES = BN * D * 2;
   static constexpr int P_BYTES = BM * BN * 2;
   static constexpr int OFF_Q = 0;
   static constexpr int OFF_K = OFF_Q + Q_BYTES;
-  static constexpr int OFF_V = OFF_K + NST * KV_BYTES;
-  static constexpr int OFF_P = OFF_V + NST * KV_BYTES;
+  static constexpr int OFF_V = OFF_K + NK * KV_BYTES;
+  static constexpr int OFF_P = OFF_V + NV * KV_BYTES;
   static constexpr int OFF_BAR = OFF_P + (kSplit ? 2 : 1) * P_BYTES;
-  static constexpr int N_BAR = 1 + 4 * NST + 2 + 3;         // q, k/v full/empty, s_full[2], p, pv, drain
+  static constexpr int N_BAR = 1 + 2 * NK + 2 * NV + 2 + 3;   // q, k/v full/empty, s_full[2], p, pv, drain
   static constexpr int OFF_MISC = OFF_BAR + 8 * N_BAR;
-  static constexpr int SMEM = OFF_MISC + 16 + 1024;         // + slack to align the base to 1 KB
+  static constexpr int SMEM = OFF_MISC + 16 + 1024;          // + slack to align the base to 1 KB
   static constexpr int THREADS = 224;
   static constexpr uint32_t TMEM_COLS = 512;
   static constexpr uint32_t COL_S0 = 0, COL_S1 = 128, COL_O = 256;
 };
 
 template <int D, int MODE>
-__global__ void __launch_bounds__(224, 1) attn_kernel(const AttnArgs a) {
+__global__ void __launch_bounds__(224, 1) attn_kernel(const __grid_constant__ AttnArgs a) {
   using C = AttnCfg<D, MODE>;
-  constexpr int BM = C::BM, BN = C::BN, NST = C::NST;
-  constexpr int CPR = D / 8;           // 16-byte chunks per row
-  constexpr int RPP = 64 / CPR;        // rows covered per loader pass (64 loader threads)
+  constexpr int BM = C::BM, BN = C::BN, NK = C::NK, NV = C::NV;
+  constexpr int NDB = D / 64;                       // 64-column (128-byte) blocks per row
+  constexpr uint32_t TILE_TX = 128u * D * 2u;       // bytes of one 128-row tile
 
   extern __shared__ uint8_t smem_raw[];
   uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
@@ -90,27 +94,26 @@ __global__ void __launch_bounds__(224, 1) attn_kernel(const AttnArgs a) {
   const uint32_t sV0 = sbase + C::OFF_V;
   const uint32_t sP = sbase + C::OFF_P;
   const uint32_t bar0 = sbase + C::OFF_BAR;
-  // barrier addresses
   const uint32_t b_q = bar0;
   auto b_kfull = [&](int s) { return bar0 + 8 * (1 + s); };
-  auto b_kempty = [&](int s) { return bar0 + 8 * (1 + NST + s); };
-  auto b_vfull = [&](int s) { return bar0 + 8 * (1 + 2 * NST + s); };
-  auto b_vempty = [&](int s) { return bar0 + 8 * (1 + 3 * NST + s); };
-  const uint32_t b_sfull0 = bar0 + 8 * (1 + 4 * NST);
-  const uint32_t b_p = bar0 + 8 * (3 + 4 * NST);
-  const uint32_t b_pv = bar0 + 8 * (4 + 4 * NST);
-  const uint32_t b_drain = bar0 + 8 * (5 + 4 * NST);
+  auto b_kempty = [&](int s) { return bar0 + 8 * (1 + NK + s); };
+  auto b_vfull = [&](int s) { return bar0 + 8 * (1 + 2 * NK + s); };
+  auto b_vempty = [&](int s) { return bar0 + 8 * (1 + 2 * NK + NV + s); };
+  const uint32_t b_sfull0 = bar0 + 8 * (1 + 2 * NK + 2 * NV);
+  const uint32_t b_p = b_sfull0 + 16;
+  const uint32_t b_pv = b_sfull0 + 24;
+  const uint32_t b_drain = b_sfull0 + 32;
   uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem + C::OFF_MISC);
   volatile int *abort_flag = reinterpret_cast<volatile int *>(smem + C::OFF_MISC + 4);
 
   const int tid = threadIdx.x;
   const int warp = tid >> 5;
+  const int lane = tid & 31;
   const int tile = blockIdx.x;          // query tile (dense) or query group (sparse)
   const int bh = blockIdx.y;
   const int N = a.N;
   const size_t head = static_cast<size_t>(bh) * N;
 
-  // number of keys this CTA attends to, and KV tiles
   const int nkeys = C::kSparse ? a.k : N;
   const int T = (nkeys + BN - 1) / BN;
   const int32_t *kv_list =
@@ -134,11 +137,13 @@ __global__ void __launch_bounds__(224, 1) attn_kernel(const AttnArgs a) {
   };
 
   if (tid == 0) {
-    mbar_init(b_q, 64);
-    for (int s = 0; s < NST; ++s) {
-      mbar_init(b_kfull(s), 64);
-      mbar_init(b_vfull(s), 64);
+    mbar_init(b_q, 1);
+    for (int s = 0; s < NK; ++s) {
+      mbar_init(b_kfull(s), 1);
       mbar_init(b_kempty(s), 1);
+    }
+    for (int s = 0; s < NV; ++s) {
+      mbar_init(b_vfull(s), 1);
       mbar_init(b_vempty(s), 1);
     }
     mbar_init(b_sfull0, 1);
@@ -153,85 +158,113 @@ __global__ void __launch_bounds__(224, 1) attn_kernel(const AttnArgs a) {
     tmem_alloc(smem_u32(tmem_slot), C::TMEM_COLS);
     tmem_relinquish();
   }
+  if (warp == 5 && lane == 0) {
+    tma_prefetch_desc(&a.tmQ);
+    tma_prefetch_desc(&a.tmK);
+    tma_prefetch_desc(&a.tmV);
+  }
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
   const uint32_t tbase = *tmem_slot;
 
   if (warp >= 5) {
-    // ------------------------------------------------------------------ gather
-    const int lt = tid - 160;   // 0..63
-    const int c = lt % CPR;
-    const int r0 = lt / CPR;
-    // Q rows (through perm in the sparse modes)
-#pragma unroll 4
-    for (int i = 0; i < 128 / RPP; ++i) {
-      const int r = r0 + i * RPP;
-      const int q = q_token(r);
-      const bf16 *src = q >= 0 ? a.Q + (head + q) * D + c * 8 : a.Q;
-      cp_async16(sQ + sw128_offset(r, c, BM), src, q >= 0 ? 16u : 0u);
+    // ------------------------------------------------------------------ TMA producers
+    const bool is_k = (warp == 5);
+    const void *tm = is_k ? static_cast<const void *>(&a.tmK) : static_cast<const void *>(&a.tmV);
+    const int NS = is_k ? NK : NV;
+    const uint32_t ring = is_k ? sK0 : sV0;
+    bool ok = true;
+    if (is_k) {
+      // the Q tile, once
+      if (C::kSparse) {
+        int rows[4];
+        const int q0 = q_token(0);
+        const int fallback = q0 >= 0 ? q0 : 0;   // padding rows re-read a valid row
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+          const int q = q_token(4 * lane + i);
+          rows[i] = static_cast<int>(head) + (q >= 0 ? q : fallback);
+        }
+        if (lane == 0) mbar_arrive_expect_tx(b_q, TILE_TX);
+        __syncwarp();
+#pragma unroll
+        for (int db = 0; db < NDB; ++db)
+          tma_gather4(sQ + db * (BM * 128) + lane * 512, &a.tmQ, db * 64, rows[0], rows[1], rows[2], rows[3], b_q);
+      } else if (lane == 0) {
+        mbar_arrive_expect_tx(b_q, TILE_TX);
+#pragma unroll
+        for (int db = 0; db < NDB; ++db) tma_load_3d(sQ + db * (BM * 128), &a.tmQ, db * 64, tile * BM, bh, b_q);
+      }
     }
-    cp_async_arrive_noinc(b_q);
     if (MODE == kModeStep || MODE == kModePlanResid) {
       // warm L2 with the rows the epilogue will read
       const float *ep = MODE == kModeStep ? a.residual : a.O32_in;
+      const int lt = tid - 160;
       for (int i = lt; i < 128 * (D / 32); i += 64) {
-        const int r = i / (D / 32);
-        const int q = q_token(r);
-        if (q >= 0)
-          asm volatile("prefetch.global.L2 [%0];" ::"l"(ep + (head + q) * D + (i % (D / 32)) * 32));
+        const int q = q_token(i / (D / 32));
+        if (q >= 0) asm volatile("prefetch.global.L2 [%0];" ::"l"(ep + (head + q) * D + (i % (D / 32)) * 32));
       }
     }
-    bool ok = true;
-    for (int j = 0; j < T && ok; ++j) {
-      const int s = j % NST;
-      const uint32_t ph = (j / NST) & 1;
-      int key[128 / RPP];
+    int issued = 0;
+    for (int j = 0; j < T; ++j) {
+      const int s = j % NS;
+      int rows[4] = {0, 0, 0, 0};
+      if (C::kSparse) {
+        const int first = kv_list[0];
 #pragma unroll
-      for (int i = 0; i < 128 / RPP; ++i) {
-        const int pos = j * BN + r0 + i * RPP;
-        key[i] = pos < nkeys ? (C::kSparse ? kv_list[pos] : pos) : -1;
-        if (C::kSparse && key[i] >= N) {   // corrupt metadata: treat as padding, report
-          record_status(a.status, kStatusBadMeta);
-          key[i] = -1;
+        for (int i = 0; i < 4; ++i) {
+          const int pos = j * BN + 4 * lane + i;
+          int key = pos < nkeys ? kv_list[pos] : first;     // padding keys re-read a valid key (masked later)
+          if (static_cast<unsigned>(key) >= static_cast<unsigned>(N)) {   // corrupt metadata
+            record_status(a.status, kStatusBadMeta);
+            key = 0;
+          }
+          rows[i] = static_cast<int>(head) + key;
         }
       }
-      if (!mbar_wait(b_kempty(s), ph ^ 1, a.wait_ns, abort_flag)) { ok = false; break; }
-      const uint32_t dK = sK0 + s * C::KV_BYTES;
+      int got = 1;
+      if (lane == 0) got = mbar_wait(is_k ? b_kempty(s) : b_vempty(s), ((j / NS) & 1) ^ 1, a.wait_ns, abort_flag);
+      got = __shfl_sync(0xffffffffu, got, 0);
+      if (!got) { ok = false; break; }
+      const uint32_t full = is_k ? b_kfull(s) : b_vfull(s);
+      const uint32_t dst = ring + s * C::KV_BYTES;
+      if (C::kSparse) {
+        if (lane == 0) mbar_arrive_expect_tx(full, TILE_TX);
+        __syncwarp();
 #pragma unroll
-      for (int i = 0; i < 128 / RPP; ++i) {
-        const int r = r0 + i * RPP;
-        const bf16 *src = key[i] >= 0 ? a.K + (head + key[i]) * D + c * 8 : a.K;
-        cp_async16(dK + sw128_offset(r, c, BN), src, key[i] >= 0 ? 16u : 0u);
-      }
-      cp_async_arrive_noinc(b_kfull(s));
-      if (!mbar_wait(b_vempty(s), ph ^ 1, a.wait_ns, abort_flag)) { ok = false; break; }
-      const uint32_t dV = sV0 + s * C::KV_BYTES;
+        for (int db = 0; db < NDB; ++db)
+          tma_gather4(dst + db * (BN * 128) + lane * 512, tm, db * 64, rows[0], rows[1], rows[2], rows[3], full);
+      } else if (lane == 0) {
+        mbar_arrive_expect_tx(full, TILE_TX);
 #pragma unroll
-      for (int i = 0; i < 128 / RPP; ++i) {
-        const int r = r0 + i * RPP;
-        const bf16 *src = key[i] >= 0 ? a.V + (head + key[i]) * D + c * 8 : a.V;
-        cp_async16(dV + sw128_offset(r, c, BN), src, key[i] >= 0 ? 16u : 0u);
+        for (int db = 0; db < NDB; ++db) tma_load_3d(dst + db * (BN * 128), tm, db * 64, j * BN, bh, full);
       }
-      cp_async_arrive_noinc(b_vfull(s));
+      ++issued;
     }
-    if (!ok && !*abort_flag) {
+    if (!ok && lane == 0 && !*abort_flag) {
       *abort_flag = 1;
       record_status(a.status, kStatusTimeout);
     }
-    cp_async_wait_all();
+    // never leave the CTA with a copy still landing in its shared memory
+    if (lane == 0) {
+      volatile int never = 0;
+      for (int t = (issued > NS ? issued - NS : 0); t < issued; ++t)
+        mbar_wait(is_k ? b_kfull(t % NS) : b_vfull(t % NS), (t / NS) & 1, 2000000000ull, &never);
+      if (is_k) mbar_wait(b_q, 0, 2000000000ull, &never);
+    }
+    __syncwarp();
   } else if (warp == 4) {
     // ------------------------------------------------------------------ UMMA issue
-    if (tid == 128) {
+    if (lane == 0) {
       constexpr uint32_t idesc_qk = idesc_bf16_f32(BM, BN, 0);
       constexpr uint32_t idesc_pv = idesc_bf16_f32(BM, D, 1);
       const uint32_t tS0 = tbase + C::COL_S0, tS1 = tbase + C::COL_S1, tO = tbase + C::COL_O;
       bool ok = mbar_wait(b_q, 0, a.wait_ns, abort_flag);
       auto issue_qk = [&](int j) -> bool {
-        const int s = j % NST;
-        if (!mbar_wait(b_kfull(s), (j / NST) & 1, a.wait_ns, abort_flag)) return false;
+        const int s = j % NK;
+        if (!mbar_wait(b_kfull(s), (j / NK) & 1, a.wait_ns, abort_flag)) return false;
         tc_fence_after();
-        fence_proxy_async_smem();
         const uint32_t kb = sK0 + s * C::KV_BYTES;
         const uint32_t tS = (j & 1) ? tS1 : tS0;
 #pragma unroll
@@ -245,11 +278,10 @@ __global__ void __launch_bounds__(224, 1) attn_kernel(const AttnArgs a) {
         return true;
       };
       auto issue_pv = [&](int j) -> bool {
-        const int s = j % NST;
+        const int s = j % NV;
         if (!mbar_wait(b_p, j & 1, a.wait_ns, abort_flag)) return false;
-        if (!mbar_wait(b_vfull(s), (j / NST) & 1, a.wait_ns, abort_flag)) return false;
+        if (!mbar_wait(b_vfull(s), (j / NV) & 1, a.wait_ns, abort_flag)) return false;
         tc_fence_after();
-        fence_proxy_async_smem();
         const uint32_t vb = sV0 + s * C::KV_BYTES;
 #pragma unroll
         for (int kk = 0; kk < BN / 16; ++kk) {

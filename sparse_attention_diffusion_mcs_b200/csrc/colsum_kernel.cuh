@@ -10,15 +10,17 @@
 // lanes, the group's queries on columns), so each thread owns one key and the
 // sum over the group is a private loop over its TMEM row: no cross-thread
 // reduction.  CTA = one (head, group); loops over all N/128 key tiles.
-//   warps 0-3 reduce, warp 4 issues UMMA, warps 5-6 stream K tiles (cp.async).
+//   warps 0-3 reduce, warp 4 issues UMMA, warp 5 loads the group's queries
+//   (TMA tile::gather4) and streams K tiles (TMA 3D tiles), warp 6 idles.
 #pragma once
 
 #include "mcs_common.cuh"
 
 namespace mcs {
 
-struct ColsumArgs {
-  const bf16 *Q, *K;        // [BH, N, D]
+struct alignas(64) ColsumArgs {
+  CUtensorMap tmQ;          // gather map over [BH*N, D]
+  CUtensorMap tmK;          // tile map over [BH, N, D]
   const int32_t *perm;      // [BH, N]
   const float *row_m;       // [BH, N] (log2 domain)
   const float *row_l;       // [BH, N]
@@ -32,7 +34,7 @@ struct ColsumArgs {
 template <int D>
 struct ColsumCfg {
   static constexpr int BM = 128, BN = 128;   // BM keys per tile (MMA M), BN queries (MMA N)
-  static constexpr int NST = 4;
+  static constexpr int NST = D == 64 ? 8 : 4;
   static constexpr int Q_BYTES = BN * D * 2;
   static constexpr int K_BYTES = BM * D * 2;
   static constexpr int OFF_Q = 0;
@@ -46,11 +48,11 @@ struct ColsumCfg {
 };
 
 template <int D>
-__global__ void __launch_bounds__(224, 1) colsum_kernel(const ColsumArgs a) {
+__global__ void __launch_bounds__(224, 1) colsum_kernel(const __grid_constant__ ColsumArgs a) {
   using C = ColsumCfg<D>;
   constexpr int BM = C::BM, NST = C::NST;
-  constexpr int CPR = D / 8;
-  constexpr int RPP = 64 / CPR;         // rows per loader pass (64 loader threads)
+  constexpr int NDB = D / 64;
+  constexpr uint32_t TILE_TX = 128u * D * 2u;
 
   extern __shared__ uint8_t smem_raw[];
   uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
@@ -89,9 +91,9 @@ __global__ void __launch_bounds__(224, 1) colsum_kernel(const ColsumArgs a) {
   };
 
   if (tid == 0) {
-    mbar_init(b_q, 64);
+    mbar_init(b_q, 1);
     for (int s = 0; s < NST; ++s) {
-      mbar_init(b_kfull(s), 64);
+      mbar_init(b_kfull(s), 1);
       mbar_init(b_kempty(s), 1);
     }
     mbar_init(b_sfull0, 1);
@@ -119,37 +121,46 @@ __global__ void __launch_bounds__(224, 1) colsum_kernel(const ColsumArgs a) {
   tc_fence_after();
   const uint32_t tbase = *tmem_slot;
 
-  if (warp >= 5) {
-    const int lt = tid - 160;   // 0..63
-    const int c = lt % CPR;
-    const int r0 = lt / CPR;
-#pragma unroll 4
-    for (int i = 0; i < 128 / RPP; ++i) {
-      const int r = r0 + i * RPP;
-      const int q = q_token(r);
-      const bf16 *src = q >= 0 ? a.Q + (head + q) * D + c * 8 : a.Q;
-      cp_async16(sQ + sw128_offset(r, c, 128), src, q >= 0 ? 16u : 0u);
-    }
-    cp_async_arrive_noinc(b_q);
-    bool ok = true;
-    for (int j = 0; j < T; ++j) {
-      const int s = j % NST;
-      if (!mbar_wait(b_kempty(s), ((j / NST) & 1) ^ 1, a.wait_ns, abort_flag)) { ok = false; break; }
-      const uint32_t dK = sK0 + s * C::K_BYTES;
+  if (warp == 5) {
+    const int lane = tid & 31;
+    {
+      int rows[4];
+      const int q0 = q_token(0);
+      const int fallback = q0 >= 0 ? q0 : 0;   // padding queries re-read a valid row (their stats zero them)
 #pragma unroll
-      for (int i = 0; i < 128 / RPP; ++i) {
-        const int r = r0 + i * RPP;
-        const int key = j * BM + r;
-        const bf16 *src = key < N ? a.K + (head + key) * D + c * 8 : a.K;
-        cp_async16(dK + sw128_offset(r, c, BM), src, key < N ? 16u : 0u);
+      for (int i = 0; i < 4; ++i) {
+        const int q = q_token(4 * lane + i);
+        rows[i] = static_cast<int>(head) + (q >= 0 ? q : fallback);
       }
-      cp_async_arrive_noinc(b_kfull(s));
+      if (lane == 0) mbar_arrive_expect_tx(b_q, TILE_TX);
+      __syncwarp();
+#pragma unroll
+      for (int db = 0; db < NDB; ++db)
+        tma_gather4(sQ + db * (128 * 128) + lane * 512, &a.tmQ, db * 64, rows[0], rows[1], rows[2], rows[3], b_q);
     }
-    if (!ok && !*abort_flag) {
-      *abort_flag = 1;
-      record_status(a.status, kStatusTimeout);
+    bool ok = true;
+    int issued = 0;
+    if (lane == 0) {
+      for (int j = 0; j < T; ++j) {
+        const int s = j % NST;
+        if (!mbar_wait(b_kempty(s), ((j / NST) & 1) ^ 1, a.wait_ns, abort_flag)) { ok = false; break; }
+        const uint32_t dK = sK0 + s * C::K_BYTES;
+        mbar_arrive_expect_tx(b_kfull(s), TILE_TX);
+#pragma unroll
+        for (int db = 0; db < NDB; ++db) tma_load_3d(dK + db * (BM * 128), &a.tmK, db * 64, j * BM, bh, b_kfull(s));
+        ++issued;
+      }
+      if (!ok && !*abort_flag) {
+        *abort_flag = 1;
+        record_status(a.status, kStatusTimeout);
+      }
+      // never leave the CTA with a copy still landing in its shared memory
+      volatile int never = 0;
+      for (int t = (issued > NST ? issued - NST : 0); t < issued; ++t)
+        mbar_wait(b_kfull(t % NST), (t / NST) & 1, 2000000000ull, &never);
+      mbar_wait(b_q, 0, 2000000000ull, &never);
     }
-    cp_async_wait_all();
+    __syncwarp();
   } else if (warp == 4) {
     if (tid == 128) {
       constexpr uint32_t idesc = idesc_bf16_f32(BM, 128, 0);
@@ -183,7 +194,7 @@ __global__ void __launch_bounds__(224, 1) colsum_kernel(const ColsumArgs a) {
       volatile int never = 0;
       mbar_wait(b_drain, 0, 2000000000ull, &never);
     }
-  } else {
+  } else if (warp < 4) {
     const uint32_t lane_addr = static_cast<uint32_t>(warp * 32) << 16;
     const float sl2 = a.scale_log2;
     float *out = a.colsum + (static_cast<size_t>(bh) * a.n_groups + g) * N;

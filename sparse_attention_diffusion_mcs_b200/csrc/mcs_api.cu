@@ -1,5 +1,7 @@
 // mcs_api.cu -- host side of the C ABI declared in include/mcs.h: argument
 // checks, workspace carving and kernel launches on the caller's stream.
+#include <cudaTypedefs.h>
+
 #include <climits>
 #include <cstdint>
 #include <cstring>
@@ -42,11 +44,55 @@ bool shape_ok(int B, int H, int N, int d) {
   if (B < 1 || H < 1 || N < 1) return false;
   if (static_cast<long long>(B) * H > 65535) return false;
   if (N > (1 << 24)) return false;
+  if (static_cast<long long>(B) * H * N >= (1ll << 31)) return false;   // TMA row coordinates are int32
   (void)d;
   return true;
 }
 bool d_ok(int d) { return d == 64 || d == 128; }
 bool g_ok(int G) { return G == 64 || G == 128; }
+
+// ---------------------------------------------------------------- TMA tensor maps
+// cuTensorMapEncodeTiled is fetched through the runtime's driver entry point,
+// so the library does not link the driver and still loads on hosts without it.
+PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void *p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+  });
+  return fn;
+}
+
+// rows x D bf16 rows, box of one 64-column row (128 bytes): tile::gather4 source
+bool map_gather(CUtensorMap *m, const void *base, int D, size_t rows) {
+  auto fn = encode_fn();
+  if (!fn) return false;
+  const cuuint64_t dims[2] = {static_cast<cuuint64_t>(D), static_cast<cuuint64_t>(rows)};
+  const cuuint64_t strides[1] = {static_cast<cuuint64_t>(D) * 2};
+  const cuuint32_t box[2] = {64, 1};
+  const cuuint32_t es[2] = {1, 1};
+  return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void *>(base), dims, strides, box, es,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+// [BH, N, D] bf16, box of 128 rows x 64 columns of one head: rows past N read as zero
+bool map_tile(CUtensorMap *m, const void *base, int D, int N, int BH) {
+  auto fn = encode_fn();
+  if (!fn) return false;
+  const cuuint64_t dims[3] = {static_cast<cuuint64_t>(D), static_cast<cuuint64_t>(N),
+                              static_cast<cuuint64_t>(BH)};
+  const cuuint64_t strides[2] = {static_cast<cuuint64_t>(D) * 2, static_cast<cuuint64_t>(N) * D * 2};
+  const cuuint32_t box[3] = {64, 128, 1};
+  const cuuint32_t es[3] = {1, 1, 1};
+  return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void *>(base), dims, strides, box, es,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
 
 template <typename F>
 cudaError_t set_smem(F *fn, int bytes) {
@@ -54,10 +100,22 @@ cudaError_t set_smem(F *fn, int bytes) {
 }
 
 // ---------------------------------------------------------------- attention launches
+struct QKV {
+  const void *Q, *K, *V;
+};
+
 template <int D, int MODE>
-cudaError_t launch_attn(const AttnArgs &a, int grid_x, int BH, cudaStream_t s) {
+cudaError_t launch_attn(AttnArgs &a, const QKV &t, int grid_x, int BH, cudaStream_t s) {
   using C = AttnCfg<D, MODE>;
   static_assert(C::SMEM <= 232448, "shared memory budget");
+  bool ok;
+  if (C::kSparse) {
+    const size_t rows = static_cast<size_t>(BH) * a.N;
+    ok = map_gather(&a.tmQ, t.Q, D, rows) && map_gather(&a.tmK, t.K, D, rows) && map_gather(&a.tmV, t.V, D, rows);
+  } else {
+    ok = map_tile(&a.tmQ, t.Q, D, a.N, BH) && map_tile(&a.tmK, t.K, D, a.N, BH) && map_tile(&a.tmV, t.V, D, a.N, BH);
+  }
+  if (!ok) return cudaErrorInvalidValue;
   cudaError_t e = set_smem(attn_kernel<D, MODE>, C::SMEM);
   if (e != cudaSuccess) return e;
   attn_kernel<D, MODE><<<dim3(grid_x, BH), C::THREADS, C::SMEM, s>>>(a);
@@ -65,16 +123,13 @@ cudaError_t launch_attn(const AttnArgs &a, int grid_x, int BH, cudaStream_t s) {
 }
 
 template <int MODE>
-cudaError_t launch_attn_d(int d, const AttnArgs &a, int grid_x, int BH, cudaStream_t s) {
-  return d == 64 ? launch_attn<64, MODE>(a, grid_x, BH, s) : launch_attn<128, MODE>(a, grid_x, BH, s);
+cudaError_t launch_attn_d(int d, AttnArgs &a, const QKV &t, int grid_x, int BH, cudaStream_t s) {
+  return d == 64 ? launch_attn<64, MODE>(a, t, grid_x, BH, s) : launch_attn<128, MODE>(a, t, grid_x, BH, s);
 }
 
-AttnArgs base_args(const void *Q, const void *K, const void *V, int N, float scale) {
+AttnArgs base_args(int N, float scale) {
   AttnArgs a;
   std::memset(&a, 0, sizeof(a));
-  a.Q = static_cast<const bf16 *>(Q);
-  a.K = static_cast<const bf16 *>(K);
-  a.V = static_cast<const bf16 *>(V);
   a.N = N;
   a.scale_log2 = scale * 1.4426950408889634f;
   a.status = status_ptr();
@@ -151,20 +206,21 @@ cudaError_t run_group(const void *Q, int BH, int N, int32_t *perm, void *ws, con
 
 cudaError_t run_plan_dense(const void *Q, const void *K, const void *V, int BH, int N, int d, float scale,
                            void *O_dense, void *ws, const PlanWs &w, cudaStream_t s) {
-  AttnArgs a = base_args(Q, K, V, N, scale);
+  AttnArgs a = base_args(N, scale);
   a.O = static_cast<bf16 *>(O_dense);
   a.O32 = at<float>(ws, w.O32);
   a.row_m = at<float>(ws, w.row_m);
   a.row_l = at<float>(ws, w.row_l);
-  return launch_attn_d<kModePlanDense>(d, a, (N + 127) / 128, BH, s);
+  return launch_attn_d<kModePlanDense>(d, a, QKV{Q, K, V}, (N + 127) / 128, BH, s);
 }
 
-cudaError_t run_select(const void *Q, const void *K, const int32_t *perm, int BH, int N, int d, int G,
-                       int k, float scale, int32_t *kv_idx, void *ws, const PlanWs &w, cudaStream_t s) {
+cudaError_t run_scores(const void *Q, const void *K, const int32_t *perm, int BH, int N, int d, int G,
+                       float scale, void *ws, const PlanWs &w, cudaStream_t s) {
   const int ng = (N + G - 1) / G;
   ColsumArgs c;
-  c.Q = static_cast<const bf16 *>(Q);
-  c.K = static_cast<const bf16 *>(K);
+  std::memset(&c, 0, sizeof(c));
+  if (!map_gather(&c.tmQ, Q, d, static_cast<size_t>(BH) * N) || !map_tile(&c.tmK, K, d, N, BH))
+    return cudaErrorInvalidValue;
   c.perm = perm;
   c.row_m = at<float>(ws, w.row_m);
   c.row_l = at<float>(ws, w.row_l);
@@ -185,8 +241,12 @@ cudaError_t run_select(const void *Q, const void *K, const int32_t *perm, int BH
     if (e != cudaSuccess) return e;
     colsum_kernel<128><<<dim3(ng, BH), 224, ColsumCfg<128>::SMEM, s>>>(c);
   }
-  e = cudaGetLastError();
-  if (e != cudaSuccess) return e;
+  return cudaGetLastError();
+}
+
+cudaError_t run_topk(int BH, int N, int G, int k, int32_t *kv_idx, void *ws, const PlanWs &w,
+                     cudaStream_t s) {
+  const int ng = (N + G - 1) / G;
   topk_kernel<<<BH * ng, kTopkThreads, 0, s>>>(at<float>(ws, w.colsum), N, k, kv_idx);
   return cudaGetLastError();
 }
@@ -194,7 +254,7 @@ cudaError_t run_select(const void *Q, const void *K, const int32_t *perm, int BH
 cudaError_t run_residual(const void *Q, const void *K, const void *V, const int32_t *perm,
                          const int32_t *kv_idx, int BH, int N, int d, int G, int k, float scale,
                          float *residual, void *ws, const PlanWs &w, cudaStream_t s) {
-  AttnArgs a = base_args(Q, K, V, N, scale);
+  AttnArgs a = base_args(N, scale);
   a.G = G;
   a.k = k;
   a.n_groups = (N + G - 1) / G;
@@ -202,7 +262,7 @@ cudaError_t run_residual(const void *Q, const void *K, const void *V, const int3
   a.kv_idx = kv_idx;
   a.O32_in = at<float>(ws, w.O32);
   a.R_out = residual;
-  return launch_attn_d<kModePlanResid>(d, a, a.n_groups, BH, s);
+  return launch_attn_d<kModePlanResid>(d, a, QKV{Q, K, V}, a.n_groups, BH, s);
 }
 
 mcs_status check_common(const void *Q, const void *K, const void *V, int B, int H, int N, int d,
@@ -274,41 +334,54 @@ mcs_status mcs_plan_group(const void *Q, int B, int H, int N, int d, int32_t *pe
                              : run_group<128>(Q, BH, N, perm, workspace, w, s));
 }
 
-mcs_status mcs_plan_select(const void *Q, const void *K, const int32_t *perm, int B, int H, int N, int d,
-                           int G, int k, float scale, int32_t *kv_idx, void *workspace,
-                           size_t workspace_bytes, mcs_stream_t stream) {
-  mcs_status st = check_common(Q, K, K, B, H, N, d, scale);
+mcs_status mcs_plan_stats(const void *Q, const void *K, const void *V, int B, int H, int N, int d, int G,
+                          int k, float scale, void *O_dense, void *workspace, size_t workspace_bytes,
+                          mcs_stream_t stream) {
+  mcs_status st = check_common(Q, K, V, B, H, N, d, scale);
   if (st != MCS_OK) return st;
-  if (!perm || !kv_idx || k < 1) return MCS_ERR_INVALID_ARG;
+  if (k < 1 || (O_dense && !aligned16(O_dense))) return MCS_ERR_INVALID_ARG;
   if (!g_ok(G)) return MCS_ERR_UNSUPPORTED;
   const PlanWs w = plan_ws(B, H, N, d, G);
   if ((st = check_ws(workspace, workspace_bytes, w.total)) != MCS_OK) return st;
-  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
-  const int BH = B * H;
-  const int kk = k < N ? k : N;
-  // statistics pass needs V only for its (discarded) output: use K as V
-  cudaError_t e = run_plan_dense(Q, K, K, BH, N, d, scale, nullptr, workspace, w, s);
-  if (e == cudaSuccess) e = run_select(Q, K, perm, BH, N, d, G, kk, scale, kv_idx, workspace, w, s);
-  return cuda_status(e);
+  return cuda_status(run_plan_dense(Q, K, V, B * H, N, d, scale, O_dense, workspace, w,
+                                    reinterpret_cast<cudaStream_t>(stream)));
+}
+
+mcs_status mcs_plan_scores(const void *Q, const void *K, const int32_t *perm, int B, int H, int N, int d,
+                           int G, int k, float scale, void *workspace, size_t workspace_bytes,
+                           mcs_stream_t stream) {
+  mcs_status st = check_common(Q, K, K, B, H, N, d, scale);
+  if (st != MCS_OK) return st;
+  if (!perm || k < 1) return MCS_ERR_INVALID_ARG;
+  if (!g_ok(G)) return MCS_ERR_UNSUPPORTED;
+  const PlanWs w = plan_ws(B, H, N, d, G);
+  if ((st = check_ws(workspace, workspace_bytes, w.total)) != MCS_OK) return st;
+  return cuda_status(run_scores(Q, K, perm, B * H, N, d, G, scale, workspace, w,
+                                reinterpret_cast<cudaStream_t>(stream)));
+}
+
+mcs_status mcs_plan_topk(int B, int H, int N, int d, int G, int k, int32_t *kv_idx, void *workspace,
+                         size_t workspace_bytes, mcs_stream_t stream) {
+  if (!shape_ok(B, H, N, d) || !kv_idx || k < 1) return MCS_ERR_INVALID_ARG;
+  if (!d_ok(d) || !g_ok(G)) return MCS_ERR_UNSUPPORTED;
+  const PlanWs w = plan_ws(B, H, N, d, G);
+  mcs_status st = check_ws(workspace, workspace_bytes, w.total);
+  if (st != MCS_OK) return st;
+  return cuda_status(run_topk(B * H, N, G, k < N ? k : N, kv_idx, workspace, w,
+                              reinterpret_cast<cudaStream_t>(stream)));
 }
 
 mcs_status mcs_plan_residual(const void *Q, const void *K, const void *V, const int32_t *perm,
                              const int32_t *kv_idx, int B, int H, int N, int d, int G, int k, float scale,
-                             float *residual, void *O_dense, void *workspace, size_t workspace_bytes,
-                             mcs_stream_t stream) {
+                             float *residual, void *workspace, size_t workspace_bytes, mcs_stream_t stream) {
   mcs_status st = check_common(Q, K, V, B, H, N, d, scale);
   if (st != MCS_OK) return st;
-  if (!perm || !kv_idx || !residual || k < 1) return MCS_ERR_INVALID_ARG;
-  if (!aligned16(residual) || (O_dense && !aligned16(O_dense))) return MCS_ERR_INVALID_ARG;
+  if (!perm || !kv_idx || !residual || k < 1 || !aligned16(residual)) return MCS_ERR_INVALID_ARG;
   if (!g_ok(G)) return MCS_ERR_UNSUPPORTED;
   const PlanWs w = plan_ws(B, H, N, d, G);
   if ((st = check_ws(workspace, workspace_bytes, w.total)) != MCS_OK) return st;
-  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
-  const int BH = B * H;
-  const int kk = k < N ? k : N;
-  cudaError_t e = run_plan_dense(Q, K, V, BH, N, d, scale, O_dense, workspace, w, s);
-  if (e == cudaSuccess) e = run_residual(Q, K, V, perm, kv_idx, BH, N, d, G, kk, scale, residual, workspace, w, s);
-  return cuda_status(e);
+  return cuda_status(run_residual(Q, K, V, perm, kv_idx, B * H, N, d, G, k < N ? k : N, scale, residual,
+                                  workspace, w, reinterpret_cast<cudaStream_t>(stream)));
 }
 
 mcs_status mcs_plan(const void *Q, const void *K, const void *V, int B, int H, int N, int d, int G, int k,
@@ -326,8 +399,8 @@ mcs_status mcs_plan(const void *Q, const void *K, const void *V, int B, int H, i
   cudaError_t e = d == 64 ? run_group<64>(Q, BH, N, meta->perm, workspace, w, s)
                           : run_group<128>(Q, BH, N, meta->perm, workspace, w, s);
   if (e == cudaSuccess) e = run_plan_dense(Q, K, V, BH, N, d, scale, O_dense, workspace, w, s);
-  if (e == cudaSuccess)
-    e = run_select(Q, K, meta->perm, BH, N, d, G, meta->k, scale, meta->kv_idx, workspace, w, s);
+  if (e == cudaSuccess) e = run_scores(Q, K, meta->perm, BH, N, d, G, scale, workspace, w, s);
+  if (e == cudaSuccess) e = run_topk(BH, N, G, meta->k, meta->kv_idx, workspace, w, s);
   if (e == cudaSuccess)
     e = run_residual(Q, K, V, meta->perm, meta->kv_idx, BH, N, d, G, meta->k, scale, meta->residual,
                      workspace, w, s);
@@ -344,7 +417,7 @@ mcs_status mcs_sparse_step(const void *Q, const void *K, const void *V, const mc
   if (!g_ok(meta->G)) return MCS_ERR_UNSUPPORTED;
   if (meta->k < 1 || meta->k > meta->N || meta->n_groups != (meta->N + meta->G - 1) / meta->G)
     return MCS_ERR_INVALID_ARG;
-  AttnArgs a = base_args(Q, K, V, meta->N, scale);
+  AttnArgs a = base_args(meta->N, scale);
   a.G = meta->G;
   a.k = meta->k;
   a.n_groups = meta->n_groups;
@@ -353,7 +426,7 @@ mcs_status mcs_sparse_step(const void *Q, const void *K, const void *V, const mc
   a.residual = meta->residual;
   a.O = static_cast<bf16 *>(O);
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
-  return cuda_status(launch_attn_d<kModeStep>(meta->d, a, meta->n_groups, meta->B * meta->H, s));
+  return cuda_status(launch_attn_d<kModeStep>(meta->d, a, QKV{Q, K, V}, meta->n_groups, meta->B * meta->H, s));
 }
 
 mcs_status mcs_dense(const void *Q, const void *K, const void *V, int B, int H, int N, int d, float scale,
@@ -361,10 +434,10 @@ mcs_status mcs_dense(const void *Q, const void *K, const void *V, int B, int H, 
   mcs_status st = check_common(Q, K, V, B, H, N, d, scale);
   if (st != MCS_OK) return st;
   if (!O || !aligned16(O)) return MCS_ERR_INVALID_ARG;
-  AttnArgs a = base_args(Q, K, V, N, scale);
+  AttnArgs a = base_args(N, scale);
   a.O = static_cast<bf16 *>(O);
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
-  return cuda_status(launch_attn_d<kModeDense>(d, a, (N + 127) / 128, B * H, s));
+  return cuda_status(launch_attn_d<kModeDense>(d, a, QKV{Q, K, V}, (N + 127) / 128, B * H, s));
 }
 
 size_t mcs_validate_workspace_size(int B, int H, int N) {

@@ -90,9 +90,14 @@ def test_plan_argument_errors(L):
     m.residual = None
     assert L.mcs_plan(*args(FAKE, need)) == INVALID
     assert L.mcs_plan_group(None, 1, 1, 10, 64, FAKE, FAKE, 1 << 20, None) == INVALID
-    assert L.mcs_plan_select(FAKE, FAKE, None, 1, 1, 10, 64, 64, 4, 0.1, FAKE, FAKE, 1 << 20,
-                             None) == INVALID
-    assert L.mcs_plan_residual(FAKE, FAKE, FAKE, FAKE, FAKE, 1, 1, 10, 64, 64, 4, 0.1, None, None,
+    assert L.mcs_plan_stats(FAKE, FAKE, FAKE, 1, 1, 10, 64, 64, 4, 0.1, None, None, 1 << 20,
+                            None) == WORKSPACE
+    assert L.mcs_plan_stats(FAKE, FAKE, FAKE, 1, 1, 10, 64, 64, 4, 0.1, FAKE + 8, FAKE, 1 << 20,
+                            None) == INVALID
+    assert L.mcs_plan_scores(FAKE, FAKE, None, 1, 1, 10, 64, 64, 4, 0.1, FAKE, 1 << 20, None) == INVALID
+    assert L.mcs_plan_topk(1, 1, 10, 64, 64, 4, None, FAKE, 1 << 20, None) == INVALID
+    assert L.mcs_plan_topk(1, 1, 10, 64, 64, 4, FAKE, FAKE, 16, None) == WORKSPACE
+    assert L.mcs_plan_residual(FAKE, FAKE, FAKE, FAKE, FAKE, 1, 1, 10, 64, 64, 4, 0.1, None,
                                FAKE, 1 << 20, None) == INVALID
 
 
