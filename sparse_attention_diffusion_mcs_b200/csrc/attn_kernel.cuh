@@ -19,14 +19,21 @@
 //                 epilogue writes R = O_dense - O_sparse (the cached residual
 //                 "between dense and sparse attention outputs").
 //
-// CTA = 128 query rows x all KV tiles of 128 keys; 224 threads:
+// CTA = 128 query rows x all KV tiles of 128 keys:
 //   warps 0-3  softmax + epilogue; thread t owns query row t = TMEM lane t
 //   warp  4    TMEM allocation and the single UMMA-issuing thread
-//   warp  5    Q and K producer (TMA), warp 6 V producer (TMA)
+//   sparse modes (288 threads): warps 5-6 Q and K producers, 7-8 V producers
+//   dense modes  (224 threads): warp 5 Q and K producer, warp 6 V producer
 // Rows listed by index (sparse modes) arrive through TMA tile::gather4, four
-// 128-byte rows per instruction; contiguous tiles (dense modes) through 3D
-// tile loads whose row bound is the head, so the ragged tail is zero-filled.
-// TMEM: S double buffer (2 x 128 fp32 columns) + O (D columns).
+// 128-byte rows per instruction.  On B200 its throughput grows with the
+// number of issuing warps (measured 2.1 TB/s from one warp, 3.4 from two, 5
+// from four), so each ring has two issuing warps, each owning half of the
+// tile's gather4 operations.  Contiguous tiles (dense modes) arrive through
+// 3D tile loads whose row bound is the head, so the ragged tail is zero.
+// TMEM: S double buffer (2 x 128 fp32 columns) + O (D columns) + the lo part
+// of P (2 x 64 columns).  P's hi part (bf16 pairs) is written over its own S
+// buffer; P.V runs with A straight from TMEM, so shared memory holds only Q
+// and the K and V rings.
 // Synchronisation is mbarrier-only inside the loops; every wait is bounded.
 #pragma once
 
@@ -60,26 +67,27 @@ struct AttnCfg {
   static constexpr int BM = 128, BN = 128;
   static constexpr bool kSparse = (MODE == kModeStep || MODE == kModePlanResid);
   static constexpr bool kSplit = (MODE == kModePlanDense || MODE == kModePlanResid);
-  static constexpr int NK = D == 64 ? (kSplit ? 4 : 5) : (kSplit ? 2 : 3);   // K ring depth
-  static constexpr int NV = D == 64 ? (kSplit ? 4 : 5) : 2;                  // V ring depth
+  static constexpr int NK = D == 64 ? 6 : 3;   // K ring depth
+  static constexpr int NV = D == 64 ? 6 : 3;   // V ring depth
   static constexpr int Q_BYTES = BM * D * 2;
   static constexpr int KV_BYTES = BN * D * 2;
-  static constexpr int P_BYTES = BM * BN * 2;
   static constexpr int OFF_Q = 0;
   static constexpr int OFF_K = OFF_Q + Q_BYTES;
   static constexpr int OFF_V = OFF_K + NK * KV_BYTES;
-  static constexpr int OFF_P = OFF_V + NV * KV_BYTES;
-  static constexpr int OFF_BAR = OFF_P + (kSplit ? 2 : 1) * P_BYTES;
+  static constexpr int OFF_BAR = OFF_V + NV * KV_BYTES;
   static constexpr int N_BAR = 1 + 2 * NK + 2 * NV + 2 + 3;   // q, k/v full/empty, s_full[2], p, pv, drain
   static constexpr int OFF_MISC = OFF_BAR + 8 * N_BAR;
   static constexpr int SMEM = OFF_MISC + 16 + 1024;          // + slack to align the base to 1 KB
-  static constexpr int THREADS = 224;
+  static constexpr int THREADS = kSparse ? 288 : 224;
+  // dense modes keep the whole score row in registers (one TMEM pass); the
+  // 288-thread sparse CTA caps registers at 168, so it reads S twice
+  static constexpr bool kOnePass = !kSparse;
   static constexpr uint32_t TMEM_COLS = 512;
-  static constexpr uint32_t COL_S0 = 0, COL_S1 = 128, COL_O = 256;
+  static constexpr uint32_t COL_S0 = 0, COL_S1 = 128, COL_O = 256, COL_PLO = 384;
 };
 
 template <int D, int MODE>
-__global__ void __launch_bounds__(224, 1) attn_kernel(const __grid_constant__ AttnArgs a) {
+__global__ void __launch_bounds__(AttnCfg<D, MODE>::THREADS, 1) attn_kernel(const __grid_constant__ AttnArgs a) {
   using C = AttnCfg<D, MODE>;
   constexpr int BM = C::BM, BN = C::BN, NK = C::NK, NV = C::NV;
   constexpr int NDB = D / 64;                       // 64-column (128-byte) blocks per row
@@ -92,7 +100,6 @@ __global__ void __launch_bounds__(224, 1) attn_kernel(const __grid_constant__ At
   const uint32_t sQ = sbase + C::OFF_Q;
   const uint32_t sK0 = sbase + C::OFF_K;
   const uint32_t sV0 = sbase + C::OFF_V;
-  const uint32_t sP = sbase + C::OFF_P;
   const uint32_t bar0 = sbase + C::OFF_BAR;
   const uint32_t b_q = bar0;
   auto b_kfull = [&](int s) { return bar0 + 8 * (1 + s); };
@@ -170,77 +177,82 @@ __global__ void __launch_bounds__(224, 1) attn_kernel(const __grid_constant__ At
 
   if (warp >= 5) {
     // ------------------------------------------------------------------ TMA producers
-    const bool is_k = (warp == 5);
+    const int pw = warp - 5;                  // sparse: 0,1 K ring, 2,3 V ring; dense: 0 K, 1 V
+    const bool is_k = C::kSparse ? pw < 2 : pw == 0;
+    const int h = C::kSparse ? (pw & 1) : 0;  // which half of the tile's operations
     const void *tm = is_k ? static_cast<const void *>(&a.tmK) : static_cast<const void *>(&a.tmV);
     const int NS = is_k ? NK : NV;
     const uint32_t ring = is_k ? sK0 : sV0;
+    // sparse: one gather4 (4 rows x 128 bytes) per active lane and tile
+    constexpr int OPS = 16 * NDB;             // gather4 operations per warp per tile
+    const bool active = lane < OPS;
+    const int op = h * OPS + (active ? lane : 0);
+    const int quad = op % 32, dbk = op / 32;
     bool ok = true;
     if (is_k) {
       // the Q tile, once
       if (C::kSparse) {
-        int rows[4];
         const int q0 = q_token(0);
         const int fallback = q0 >= 0 ? q0 : 0;   // padding rows re-read a valid row
+        int rows[4];
 #pragma unroll
         for (int i = 0; i < 4; ++i) {
-          const int q = q_token(4 * lane + i);
+          const int q = q_token(4 * quad + i);
           rows[i] = static_cast<int>(head) + (q >= 0 ? q : fallback);
         }
-        if (lane == 0) mbar_arrive_expect_tx(b_q, TILE_TX);
+        if (h == 0 && lane == 0) mbar_arrive_expect_tx(b_q, TILE_TX);
         __syncwarp();
-#pragma unroll
-        for (int db = 0; db < NDB; ++db)
-          tma_gather4(sQ + db * (BM * 128) + lane * 512, &a.tmQ, db * 64, rows[0], rows[1], rows[2], rows[3], b_q);
-      } else if (lane == 0) {
+        if (active)
+          tma_gather4(sQ + dbk * (BM * 128) + quad * 512, &a.tmQ, dbk * 64, rows[0], rows[1], rows[2], rows[3], b_q);
+      } else if (h == 0 && lane == 0) {
         mbar_arrive_expect_tx(b_q, TILE_TX);
 #pragma unroll
         for (int db = 0; db < NDB; ++db) tma_load_3d(sQ + db * (BM * 128), &a.tmQ, db * 64, tile * BM, bh, b_q);
       }
     }
-    if (MODE == kModeStep || MODE == kModePlanResid) {
-      // warm L2 with the rows the epilogue will read
-      const float *ep = MODE == kModeStep ? a.residual : a.O32_in;
-      const int lt = tid - 160;
-      for (int i = lt; i < 128 * (D / 32); i += 64) {
-        const int q = q_token(i / (D / 32));
-        if (q >= 0) asm volatile("prefetch.global.L2 [%0];" ::"l"(ep + (head + q) * D + (i % (D / 32)) * 32));
-      }
-    }
-    int issued = 0;
-    for (int j = 0; j < T; ++j) {
-      const int s = j % NS;
-      int rows[4] = {0, 0, 0, 0};
-      if (C::kSparse) {
-        const int first = kv_list[0];
+    // global row indices of tile t for this lane's gather4 (sparse modes)
+    auto tile_rows = [&](int t, int (&rows)[4]) {
+      const int first = kv_list[0];
 #pragma unroll
-        for (int i = 0; i < 4; ++i) {
-          const int pos = j * BN + 4 * lane + i;
-          int key = pos < nkeys ? kv_list[pos] : first;     // padding keys re-read a valid key (masked later)
-          if (static_cast<unsigned>(key) >= static_cast<unsigned>(N)) {   // corrupt metadata
-            record_status(a.status, kStatusBadMeta);
-            key = 0;
-          }
-          rows[i] = static_cast<int>(head) + key;
+      for (int i = 0; i < 4; ++i) {
+        const int pos = t * BN + 4 * quad + i;
+        int key = pos < nkeys ? kv_list[pos] : first;     // padding keys re-read a valid key (masked later)
+        if (static_cast<unsigned>(key) >= static_cast<unsigned>(N)) {   // corrupt metadata
+          record_status(a.status, kStatusBadMeta);
+          key = 0;
         }
+        rows[i] = static_cast<int>(head) + key;
       }
-      int got = 1;
-      if (lane == 0) got = mbar_wait(is_k ? b_kempty(s) : b_vempty(s), ((j / NS) & 1) ^ 1, a.wait_ns, abort_flag);
-      got = __shfl_sync(0xffffffffu, got, 0);
-      if (!got) { ok = false; break; }
-      const uint32_t full = is_k ? b_kfull(s) : b_vfull(s);
-      const uint32_t dst = ring + s * C::KV_BYTES;
-      if (C::kSparse) {
-        if (lane == 0) mbar_arrive_expect_tx(full, TILE_TX);
-        __syncwarp();
+    };
+    const bool dense_idle = !C::kSparse && h == 1;   // dense tiles need one issuing lane per ring
+    int issued = 0;
+    if (!dense_idle) {
+      int rows[4] = {0, 0, 0, 0}, next[4] = {0, 0, 0, 0};
+      if (C::kSparse) tile_rows(0, rows);
+      for (int j = 0; j < T; ++j) {
+        const int s = j % NS;
+        if (C::kSparse && j + 1 < T) tile_rows(j + 1, next);   // in flight while we wait for the slot
+        int got = 1;
+        if (lane == 0) got = mbar_wait(is_k ? b_kempty(s) : b_vempty(s), ((j / NS) & 1) ^ 1, a.wait_ns, abort_flag);
+        got = __shfl_sync(0xffffffffu, got, 0);
+        if (!got) { ok = false; break; }
+        const uint32_t full = is_k ? b_kfull(s) : b_vfull(s);
+        const uint32_t dst = ring + s * C::KV_BYTES;
+        if (C::kSparse) {
+          // one expect-tx arrival per phase; the other warp's bytes may land first
+          if (h == 0 && lane == 0) mbar_arrive_expect_tx(full, TILE_TX);
+          __syncwarp();
+          if (active)
+            tma_gather4(dst + dbk * (BN * 128) + quad * 512, tm, dbk * 64, rows[0], rows[1], rows[2], rows[3], full);
 #pragma unroll
-        for (int db = 0; db < NDB; ++db)
-          tma_gather4(dst + db * (BN * 128) + lane * 512, tm, db * 64, rows[0], rows[1], rows[2], rows[3], full);
-      } else if (lane == 0) {
-        mbar_arrive_expect_tx(full, TILE_TX);
+          for (int i = 0; i < 4; ++i) rows[i] = next[i];
+        } else if (lane == 0) {
+          mbar_arrive_expect_tx(full, TILE_TX);
 #pragma unroll
-        for (int db = 0; db < NDB; ++db) tma_load_3d(dst + db * (BN * 128), tm, db * 64, j * BN, bh, full);
+          for (int db = 0; db < NDB; ++db) tma_load_3d(dst + db * (BN * 128), tm, db * 64, j * BN, bh, full);
+        }
+        ++issued;
       }
-      ++issued;
     }
     if (!ok && lane == 0 && !*abort_flag) {
       *abort_flag = 1;
@@ -283,19 +295,18 @@ __global__ void __launch_bounds__(224, 1) attn_kernel(const __grid_constant__ At
         if (!mbar_wait(b_vfull(s), (j / NV) & 1, a.wait_ns, abort_flag)) return false;
         tc_fence_after();
         const uint32_t vb = sV0 + s * C::KV_BYTES;
+        const uint32_t tP = (j & 1) ? tS1 : tS0;                              // hi part over S
+        const uint32_t tPlo = tbase + C::COL_PLO + (j & 1) * (BN / 2);        // lo part
 #pragma unroll
         for (int kk = 0; kk < BN / 16; ++kk) {
-          const uint32_t offp = (kk >> 2) * (128 * 128) + (kk & 3) * 32;
           const uint64_t bdesc = sdesc_sw128(vb + kk * 16 * 128, BN * 128, 1024);
-          umma_bf16_ss(tO, sdesc_sw128(sP + offp, 16, 1024), bdesc, idesc_pv,
-                       (j > 0 || kk > 0) ? 1u : 0u);
+          umma_bf16_ts(tO, tP + kk * 8, bdesc, idesc_pv, (j > 0 || kk > 0) ? 1u : 0u);
         }
         if (C::kSplit) {
 #pragma unroll
           for (int kk = 0; kk < BN / 16; ++kk) {
-            const uint32_t offp = (kk >> 2) * (128 * 128) + (kk & 3) * 32;
             const uint64_t bdesc = sdesc_sw128(vb + kk * 16 * 128, BN * 128, 1024);
-            umma_bf16_ss(tO, sdesc_sw128(sP + C::P_BYTES + offp, 16, 1024), bdesc, idesc_pv, 1u);
+            umma_bf16_ts(tO, tPlo + kk * 8, bdesc, idesc_pv, 1u);
           }
         }
         umma_commit(b_pv);
@@ -320,33 +331,87 @@ __global__ void __launch_bounds__(224, 1) attn_kernel(const __grid_constant__ At
   } else {
     // ------------------------------------------------------------------ softmax
     const int r = tid;                           // query row == TMEM lane
+    const int my_q = q_token(r);
+    if (MODE == kModeStep || MODE == kModePlanResid) {
+      // warm L2 with the row the epilogue will read
+      const float *ep = MODE == kModeStep ? a.residual : a.O32_in;
+      if (my_q >= 0) {
+#pragma unroll
+        for (int c = 0; c < D / 32; ++c)
+          asm volatile("prefetch.global.L2 [%0];" ::"l"(ep + (head + my_q) * D + c * 32));
+      }
+    }
     const uint32_t lane_addr = static_cast<uint32_t>(warp * 32) << 16;
     const float sl2 = a.scale_log2;
     float m_run = -INFINITY, l_run = 0.f;
     bool ok = true;
-    float s[BN];
     for (int j = 0; j < T; ++j) {
       if (!mbar_wait(b_sfull0 + 8 * (j & 1), (j >> 1) & 1, a.wait_ns, abort_flag)) { ok = false; break; }
       tc_fence_after();
       const uint32_t tS = tbase + lane_addr + ((j & 1) ? C::COL_S1 : C::COL_S0);
-#pragma unroll
-      for (int cc = 0; cc < BN / 32; ++cc) {
-        float tmp[32];
-        tmem_ld32(tS + cc * 32, tmp);
-#pragma unroll
-        for (int i = 0; i < 32; ++i) s[cc * 32 + i] = tmp[i];
-      }
-      tmem_wait_ld();
+      const uint32_t tPlo = tbase + lane_addr + C::COL_PLO + (j & 1) * (BN / 2);
       const int nvalid = nkeys - j * BN;   // >= 1
-      float mx = -INFINITY;
-#pragma unroll
-      for (int i = 0; i < BN; ++i) {
-        if (i >= nvalid) s[i] = -INFINITY;
-        mx = fmaxf(mx, s[i]);
-      }
-      mx *= sl2;
       float alpha = 1.f;
       bool resc = false;
+      float rs0 = 0.f, rs1 = 0.f;
+      if constexpr (C::kOnePass) {
+        float sv[BN];
+#pragma unroll
+        for (int cc = 0; cc < BN / 32; ++cc) {
+          float tmp[32];
+          tmem_ld32(tS + cc * 32, tmp);
+#pragma unroll
+          for (int i = 0; i < 32; ++i) sv[cc * 32 + i] = tmp[i];
+        }
+        tmem_wait_ld();
+        float mx = -INFINITY;
+#pragma unroll
+        for (int i = 0; i < BN; ++i) {
+          if (i >= nvalid) sv[i] = -INFINITY;
+          mx = fmaxf(mx, sv[i]);
+        }
+        mx *= sl2;
+        if (j == 0) {
+          m_run = mx;
+        } else if (mx > m_run + 8.f) {      // lazy rescale: only when the max grew by > 2^8
+          alpha = ex2_approx(m_run - mx);
+          m_run = mx;
+          resc = true;
+        }
+#pragma unroll
+        for (int i = 0; i < BN; ++i) {
+          sv[i] = ex2_approx(fmaf(sv[i], sl2, -m_run));
+          if (i & 1) rs1 += sv[i]; else rs0 += sv[i];
+        }
+        // P over this tile's own S columns (bf16 pairs); lo parts in their own columns
+#pragma unroll
+        for (int hh = 0; hh < BN / 64; ++hh) {
+          uint32_t pk[32];
+#pragma unroll
+          for (int i = 0; i < 32; ++i) pk[i] = pack_bf16x2(sv[hh * 64 + 2 * i], sv[hh * 64 + 2 * i + 1]);
+          tmem_st32u(tS + hh * 32, pk);
+          if (C::kSplit) {
+#pragma unroll
+            for (int i = 0; i < 32; ++i) {
+              const __nv_bfloat162 hb = *reinterpret_cast<const __nv_bfloat162 *>(&pk[i]);
+              const float2 hf = __bfloat1622float2(hb);
+              pk[i] = pack_bf16x2(sv[hh * 64 + 2 * i] - hf.x, sv[hh * 64 + 2 * i + 1] - hf.y);
+            }
+            tmem_st32u(tPlo + hh * 32, pk);
+          }
+        }
+      } else {
+      // pass 1: row max of this tile
+      float mx = -INFINITY;
+#pragma unroll
+      for (int cc = 0; cc < BN / 32; ++cc) {
+        float v[32];
+        tmem_ld32(tS + cc * 32, v);
+        tmem_wait_ld();
+#pragma unroll
+        for (int i = 0; i < 32; ++i) mx = fmaxf(mx, (cc * 32 + i < nvalid) ? v[i] : -INFINITY);
+      }
+      mx *= sl2;
       if (j == 0) {
         m_run = mx;
       } else if (mx > m_run + 8.f) {      // lazy rescale: only when the max grew by > 2^8
@@ -354,14 +419,36 @@ __global__ void __launch_bounds__(224, 1) attn_kernel(const __grid_constant__ At
         m_run = mx;
         resc = true;
       }
-      float rs = 0.f;
+      // pass 2: P = 2^(s*scale*log2e - m) as bf16 pairs over S (chunk cc lands on
+      // columns [16cc, 16cc+16), all already read), lo parts in their own columns
 #pragma unroll
-      for (int i = 0; i < BN; ++i) {
-        s[i] = ex2_approx(fmaf(s[i], sl2, -m_run));
-        rs += s[i];
+      for (int cc = 0; cc < BN / 32; ++cc) {
+        float v[32];
+        tmem_ld32(tS + cc * 32, v);
+        tmem_wait_ld();
+#pragma unroll
+        for (int i = 0; i < 32; ++i) {
+          v[i] = (cc * 32 + i < nvalid) ? ex2_approx(fmaf(v[i], sl2, -m_run)) : 0.f;
+          if (i & 1) rs1 += v[i]; else rs0 += v[i];
+        }
+        uint32_t pk[16];
+#pragma unroll
+        for (int i = 0; i < 16; ++i) pk[i] = pack_bf16x2(v[2 * i], v[2 * i + 1]);
+        tmem_st16u(tS + cc * 16, pk);
+        if (C::kSplit) {
+#pragma unroll
+          for (int i = 0; i < 16; ++i) {
+            const __nv_bfloat162 hb = *reinterpret_cast<const __nv_bfloat162 *>(&pk[i]);
+            const float2 hf = __bfloat1622float2(hb);
+            pk[i] = pack_bf16x2(v[2 * i] - hf.x, v[2 * i + 1] - hf.y);
+          }
+          tmem_st16u(tPlo + cc * 16, pk);
+        }
       }
-      l_run = fmaf(l_run, alpha, rs);
-      // P buffer and O are free once the previous P.V has completed
+      }
+      l_run = fmaf(l_run, alpha, rs0 + rs1);
+      tmem_wait_st();
+      // O is stable once the previous P.V has completed
       if (j > 0) {
         if (!mbar_wait(b_pv, (j - 1) & 1, a.wait_ns, abort_flag)) { ok = false; break; }
         tc_fence_after();
@@ -379,29 +466,6 @@ __global__ void __launch_bounds__(224, 1) attn_kernel(const __grid_constant__ At
           tmem_wait_st();
         }
       }
-      uint8_t *pP = smem + C::OFF_P;
-#pragma unroll
-      for (int c16 = 0; c16 < BN / 8; ++c16) {
-        uint4 hi;
-        hi.x = pack_bf16x2(s[c16 * 8 + 0], s[c16 * 8 + 1]);
-        hi.y = pack_bf16x2(s[c16 * 8 + 2], s[c16 * 8 + 3]);
-        hi.z = pack_bf16x2(s[c16 * 8 + 4], s[c16 * 8 + 5]);
-        hi.w = pack_bf16x2(s[c16 * 8 + 6], s[c16 * 8 + 7]);
-        const uint32_t off = sw128_offset(r, c16, BM);
-        *reinterpret_cast<uint4 *>(pP + off) = hi;
-        if (C::kSplit) {
-          const __nv_bfloat162 *h2 = reinterpret_cast<const __nv_bfloat162 *>(&hi);
-          uint4 lo;
-          uint32_t *lw = reinterpret_cast<uint32_t *>(&lo);
-#pragma unroll
-          for (int u = 0; u < 4; ++u) {
-            const float2 hf = __bfloat1622float2(h2[u]);
-            lw[u] = pack_bf16x2(s[c16 * 8 + 2 * u] - hf.x, s[c16 * 8 + 2 * u + 1] - hf.y);
-          }
-          *reinterpret_cast<uint4 *>(pP + C::P_BYTES + off) = lo;
-        }
-      }
-      fence_proxy_async_smem();
       tc_fence_before();
       mbar_arrive(b_p);
     }
@@ -416,7 +480,7 @@ __global__ void __launch_bounds__(224, 1) attn_kernel(const __grid_constant__ At
     } else {
       // ------------------------------------------------------------------ epilogue
       tc_fence_after();
-      const int q = q_token(r);
+      const int q = my_q;
       const float inv_l = 1.f / l_run;
       const uint32_t tO = tbase + lane_addr + C::COL_O;
       const size_t row = (head + (q >= 0 ? q : 0)) * D;
