@@ -51,7 +51,8 @@ typedef enum {
   MCS_ERR_WORKSPACE = 3,    /* workspace missing or smaller than required  */
   MCS_ERR_CUDA = 4,         /* a CUDA runtime call or launch failed        */
   MCS_ERR_TIMEOUT = 5,      /* a bounded device wait ran out               */
-  MCS_ERR_BAD_META = 6      /* metadata failed validation                  */
+  MCS_ERR_BAD_META = 6,     /* metadata failed validation                  */
+  MCS_ERR_TOO_LARGE = 7     /* shape exceeds a fixed, compiled-in capacity */
 } mcs_status;
 
 /* Cached metadata of one plan ("query groups, KV indices ... and residuals",
@@ -174,6 +175,30 @@ size_t mcs_validate_workspace_size(int B, int H, int N);
  */
 mcs_status mcs_validate_meta(const mcs_meta *meta, void *workspace, size_t workspace_bytes,
                              int *first_bad, mcs_stream_t stream);
+
+/*
+ * mcs_validate_meta_noalloc -- the same checks as mcs_validate_meta, for
+ * callers that cannot hand over a device workspace.  The pages describe no
+ * such call; it exists for users of this library whose code may not call
+ * cudaMalloc at the point of the check: code recorded into a CUDA graph
+ * capture (allocation is not a capturable operation), runtimes that forbid
+ * allocation after start-up, and plugins that only receive raw pointers from
+ * a host framework that owns all device memory.
+ *
+ * Scratch: a fixed array compiled into the library, one per device that
+ * loads it, held until the process exits: 256 bytes + one bit per token,
+ * MCS_NOALLOC_MAX_TOKENS tokens (B*H*N) at most; larger shapes return
+ * MCS_ERR_TOO_LARGE before anything is launched.  Nothing is allocated.
+ * The first call on a device looks up that device's address of the array
+ * (cudaGetSymbolAddress); make that first call before any stream capture.
+ * Every call clears the scratch it uses, so a call never sees an earlier
+ * call's contents, but calls that overlap on the GPU (two streams, or two
+ * host threads on one device) share the array and race.  Synchronous, like
+ * mcs_validate_meta; returns MCS_OK, MCS_ERR_BAD_META (with *first_bad) or
+ * an argument / CUDA error.
+ */
+#define MCS_NOALLOC_MAX_TOKENS (1u << 23)
+mcs_status mcs_validate_meta_noalloc(const mcs_meta *meta, int *first_bad, mcs_stream_t stream);
 
 /* Synchronise `stream`, then read and clear this device's status word.
  * Returns MCS_OK, or MCS_ERR_TIMEOUT if a kernel's bounded wait ran out

@@ -15,7 +15,7 @@ LIB_PATH = os.path.join(PKG_DIR, "libmcs.so")
 MCS_OK = 0
 STATUS_NAMES = {
     0: "MCS_OK", 1: "MCS_ERR_INVALID_ARG", 2: "MCS_ERR_UNSUPPORTED", 3: "MCS_ERR_WORKSPACE",
-    4: "MCS_ERR_CUDA", 5: "MCS_ERR_TIMEOUT", 6: "MCS_ERR_BAD_META",
+    4: "MCS_ERR_CUDA", 5: "MCS_ERR_TIMEOUT", 6: "MCS_ERR_BAD_META", 7: "MCS_ERR_TOO_LARGE",
 }
 
 # Every exported symbol and its prototype: (restype, argtypes).
@@ -51,6 +51,7 @@ PROTOTYPES = {
     "mcs_dense": (c_int, [c_vp, c_vp, c_vp, c_int, c_int, c_int, c_int, c_float, c_vp, c_vp]),
     "mcs_validate_workspace_size": (c_size_t, [c_int, c_int, c_int]),
     "mcs_validate_meta": (c_int, [PMETA, c_vp, c_size_t, ctypes.POINTER(c_int), c_vp]),
+    "mcs_validate_meta_noalloc": (c_int, [PMETA, ctypes.POINTER(c_int), c_vp]),
     "mcs_last_device_status": (c_int, [c_vp]),
     "mcs_selftest_wait_timeout": (c_int, [c_u64, c_vp]),
     "mcs_set_wait_limit_ns": (None, [c_u64]),

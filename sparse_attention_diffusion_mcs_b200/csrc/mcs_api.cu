@@ -280,6 +280,27 @@ mcs_status check_ws(void *ws, size_t bytes, size_t need) {
   return MCS_OK;
 }
 
+// ---------------------------------------------------------------- allocation-free validation scratch
+// Fixed scratch for mcs_validate_meta_noalloc: a 256-byte flag area followed
+// by one bit per token.  Host code may not pass the symbol itself to a kernel
+// (on the host it only names a stand-in); the device address comes from
+// cudaGetSymbolAddress, looked up once per device with that device current.
+constexpr size_t kNoAllocScratchBytes = 256 + (static_cast<size_t>(MCS_NOALLOC_MAX_TOKENS) + 7) / 8;
+static __device__ __align__(256) unsigned char g_noalloc_scratch[kNoAllocScratchBytes];
+unsigned char *g_noalloc_ptr[kMaxDevices];
+
+unsigned char *noalloc_scratch() {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return nullptr;
+  std::lock_guard<std::mutex> lk(g_mu);
+  if (!g_noalloc_ptr[dev]) {
+    void *p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || p == nullptr) return nullptr;
+    g_noalloc_ptr[dev] = static_cast<unsigned char *>(p);
+  }
+  return g_noalloc_ptr[dev];
+}
+
 }  // namespace
 
 // ============================================================================ C ABI
@@ -297,6 +318,7 @@ const char *mcs_status_string(mcs_status s) {
     case MCS_ERR_CUDA: return "MCS_ERR_CUDA";
     case MCS_ERR_TIMEOUT: return "MCS_ERR_TIMEOUT";
     case MCS_ERR_BAD_META: return "MCS_ERR_BAD_META";
+    case MCS_ERR_TOO_LARGE: return "MCS_ERR_TOO_LARGE";
   }
   return "MCS_ERR_UNKNOWN";
 }
@@ -471,6 +493,42 @@ mcs_status mcs_validate_meta(const mcs_meta *meta, void *workspace, size_t works
                                        static_cast<size_t>(BH) * meta->n_groups, bad);
   residual_check_kernel<<<grid, 256, 0, s>>>(meta->residual,
                                              static_cast<size_t>(BH) * meta->N * meta->d, bad);
+  if (cudaGetLastError() != cudaSuccess) return MCS_ERR_CUDA;
+  int h = INT_MAX;
+  e = cudaMemcpyAsync(&h, bad, sizeof(int), cudaMemcpyDeviceToHost, s);
+  if (e == cudaSuccess) e = cudaStreamSynchronize(s);
+  if (e != cudaSuccess) return MCS_ERR_CUDA;
+  if (h == INT_MAX) return MCS_OK;
+  if (first_bad) *first_bad = h;
+  return MCS_ERR_BAD_META;
+}
+
+mcs_status mcs_validate_meta_noalloc(const mcs_meta *meta, int *first_bad, mcs_stream_t stream) {
+  if (first_bad) *first_bad = 0;
+  if (!meta || !meta->perm || !meta->kv_idx || !meta->residual) return MCS_ERR_INVALID_ARG;
+  if (!shape_ok(meta->B, meta->H, meta->N, meta->d) || !d_ok(meta->d) || !g_ok(meta->G))
+    return MCS_ERR_INVALID_ARG;
+  if (meta->k < 1 || meta->k > meta->N || meta->n_groups != (meta->N + meta->G - 1) / meta->G)
+    return MCS_ERR_INVALID_ARG;
+  const size_t tokens = static_cast<size_t>(meta->B) * meta->H * meta->N;
+  if (tokens > MCS_NOALLOC_MAX_TOKENS) return MCS_ERR_TOO_LARGE;
+  unsigned char *scratch = noalloc_scratch();
+  if (!scratch) return MCS_ERR_CUDA;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  const int BH = meta->B * meta->H;
+  int *bad = reinterpret_cast<int *>(scratch);
+  unsigned *seen = reinterpret_cast<unsigned *>(scratch + 256);
+  const size_t bitmap_bytes = ((tokens + 31) / 32) * 4;
+  // the array keeps the previous call's contents: clear the flag and every bit this call reads
+  const int init = INT_MAX;
+  cudaError_t e = cudaMemcpyAsync(bad, &init, sizeof(int), cudaMemcpyHostToDevice, s);
+  if (e == cudaSuccess) e = cudaMemsetAsync(seen, 0, bitmap_bytes, s);
+  if (e != cudaSuccess) return MCS_ERR_CUDA;
+  const int grid = 148 * 8;
+  perm_mark_kernel<<<grid, 256, 0, s>>>(meta->perm, meta->N, BH, seen, bad);
+  kv_check_kernel<<<grid, 256, 0, s>>>(meta->kv_idx, meta->N, meta->k,
+                                       static_cast<size_t>(BH) * meta->n_groups, bad);
+  residual_check_kernel<<<grid, 256, 0, s>>>(meta->residual, tokens * meta->d, bad);
   if (cudaGetLastError() != cudaSuccess) return MCS_ERR_CUDA;
   int h = INT_MAX;
   e = cudaMemcpyAsync(&h, bad, sizeof(int), cudaMemcpyDeviceToHost, s);
