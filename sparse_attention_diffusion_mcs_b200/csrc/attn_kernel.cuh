@@ -23,13 +23,15 @@
 // CTA = 128 query rows x all KV tiles of 128 keys:
 //   warps 0-3  softmax + epilogue; thread t owns query row t = TMEM lane t
 //   warp  4    TMEM allocation and the single UMMA-issuing thread
-//   sparse modes (288 threads): warps 5-6 Q and K producers, 7-8 V producers
+//   sparse modes (384 threads): warps 5-8 Q and K producers, 9-11 V producers
 //   dense modes  (224 threads): warp 5 Q and K producer, warp 6 V producer
 // Rows listed by index (sparse modes) arrive through TMA tile::gather4, four
 // 128-byte rows per instruction.  On B200 its throughput grows with the
 // number of issuing warps (measured 2.1 TB/s from one warp, 3.4 from two, 5
-// from four), so each ring has two issuing warps, each owning half of the
-// tile's gather4 operations.  Contiguous tiles (dense modes) arrive through
+// from four, 6.4 from eight), so the K ring has four issuing warps and the V
+// ring three, each owning an interleaved share of the tile's gather4
+// operations.  (A 288-thread CTA is register-allocated like 384 threads, so
+// the extra warps cost no registers.)  Contiguous tiles (dense modes) arrive through
 // 3D tile loads whose row bound is the head, so the ragged tail is zero.
 // TMEM: S double buffer (2 x 128 fp32 columns) + O (D columns) + the lo part
 // of P (2 x 64 columns).  P's hi part (bf16 pairs) is written over its own S
@@ -37,6 +39,8 @@
 // and the K and V rings.
 // Synchronisation is mbarrier-only inside the loops; every wait is bounded.
 #pragma once
+
+#include <type_traits>
 
 #include "mcs_common.cuh"
 
@@ -82,9 +86,10 @@ struct AttnCfg {
   static constexpr int N_BAR = 1 + 2 * NK + 2 * NV + 2 + 3;   // q, k/v full/empty, s_full[2], p, pv, drain
   static constexpr int OFF_MISC = OFF_BAR + 8 * N_BAR;
   static constexpr int SMEM = OFF_MISC + 16 + 1024;          // + slack to align the base to 1 KB
-  static constexpr int THREADS = kSparse ? 288 : 224;
+  static constexpr int THREADS = kSparse ? 384 : 224;
+  static constexpr int KW = kSparse ? 4 : 1, VW = kSparse ? 3 : 1;   // issuing warps per ring
   // dense modes keep the whole score row in registers (one TMEM pass); the
-  // 288-thread sparse CTA caps registers at 168, so it reads S twice
+  // 384-thread sparse CTA caps registers at 168, so it reads S twice
   static constexpr bool kOnePass = !kSparse;
   static constexpr uint32_t TMEM_COLS = 512;
   static constexpr uint32_t COL_S0 = 0, COL_S1 = 128, COL_O = 256, COL_PLO = 384;
@@ -181,16 +186,19 @@ __global__ void __launch_bounds__(AttnCfg<D, MODE>::THREADS, 1) attn_kernel(cons
 
   if (warp >= 5) {
     // ------------------------------------------------------------------ TMA producers
-    const int pw = warp - 5;                  // sparse: 0,1 K ring, 2,3 V ring; dense: 0 K, 1 V
-    const bool is_k = C::kSparse ? pw < 2 : pw == 0;
-    const int h = C::kSparse ? (pw & 1) : 0;  // which half of the tile's operations
+    const int pw = warp - 5;                  // 0..KW-1: K ring, KW..KW+VW-1: V ring
+    const bool is_k = pw < C::KW;
+    const int NW = is_k ? C::KW : C::VW;      // issuing warps of this ring
+    const int h = is_k ? pw : pw - C::KW;     // this warp's share of the tile's operations
     const void *tm = is_k ? static_cast<const void *>(&a.tmK) : static_cast<const void *>(&a.tmV);
     const int NS = is_k ? NK : NV;
     const uint32_t ring = is_k ? sK0 : sV0;
-    // sparse: one gather4 (4 rows x 128 bytes) per active lane and tile
-    constexpr int OPS = 16 * NDB;             // gather4 operations per warp per tile
-    const bool active = lane < OPS;
-    const int op = h * OPS + (active ? lane : 0);
+    // sparse: gather4 operation o (4 rows x 128 bytes) of a tile belongs to
+    // warp o % NW, lane o / NW; a tile has 32 row quads x NDB column blocks
+    constexpr int OPS = 32 * NDB;
+    const int op_raw = h + NW * lane;
+    const bool active = op_raw < OPS;
+    const int op = active ? op_raw : h;
     const int quad = op % 32, dbk = op / 32;
     bool ok = true;
     if (is_k) {
@@ -228,7 +236,7 @@ __global__ void __launch_bounds__(AttnCfg<D, MODE>::THREADS, 1) attn_kernel(cons
         rows[i] = static_cast<int>(head) + key;
       }
     };
-    const bool dense_idle = !C::kSparse && h == 1;   // dense tiles need one issuing lane per ring
+    const bool dense_idle = false;            // dense: one warp per ring, lane 0 issues
     int issued = 0;
     if (!dense_idle) {
       int rows[4] = {0, 0, 0, 0}, next[4] = {0, 0, 0, 0};
@@ -354,26 +362,12 @@ __global__ void __launch_bounds__(AttnCfg<D, MODE>::THREADS, 1) attn_kernel(cons
       tc_fence_after();
       const uint32_t tS = tbase + lane_addr + ((j & 1) ? C::COL_S1 : C::COL_S0);
       const uint32_t tPlo = tbase + lane_addr + C::COL_PLO + (j & 1) * (BN / 2);
-      const int nvalid = nkeys - j * BN;   // >= 1
+      const int nvalid = nkeys - j * BN;   // >= 1; only the last tile can be partial
       float alpha = 1.f;
       bool resc = false;
       float rs0 = 0.f, rs1 = 0.f;
-      if constexpr (C::kOnePass) {
-        float sv[BN];
-#pragma unroll
-        for (int cc = 0; cc < BN / 32; ++cc) {
-          float tmp[32];
-          tmem_ld32(tS + cc * 32, tmp);
-#pragma unroll
-          for (int i = 0; i < 32; ++i) sv[cc * 32 + i] = tmp[i];
-        }
-        tmem_wait_ld();
-        float mx = -INFINITY;
-#pragma unroll
-        for (int i = 0; i < BN; ++i) {
-          if (i >= nvalid) sv[i] = -INFINITY;
-          mx = fmaxf(mx, sv[i]);
-        }
+      // new running max from this tile's max (scaled to the log2 domain)
+      auto update_max = [&](float mx) {
         mx *= sl2;
         if (j == 0) {
           m_run = mx;
@@ -382,74 +376,109 @@ __global__ void __launch_bounds__(AttnCfg<D, MODE>::THREADS, 1) attn_kernel(cons
           m_run = mx;
           resc = true;
         }
-#pragma unroll
-        for (int i = 0; i < BN; ++i) {
-          sv[i] = ex2_approx(fmaf(sv[i], sl2, -m_run));
-          if (i & 1) rs1 += sv[i]; else rs0 += sv[i];
-        }
-        // P over this tile's own S columns (bf16 pairs); lo parts in their own columns
-#pragma unroll
-        for (int hh = 0; hh < BN / 64; ++hh) {
+      };
+      // P as bf16 pairs over S; the lo parts (split modes) in their own columns
+      auto store_p = [&](const float *pv, int n32, uint32_t dst_hi, uint32_t dst_lo) {
+        // n32 = number of 32-bit columns (pairs) to write from pv
+        if (n32 == 32) {
           uint32_t pk[32];
 #pragma unroll
-          for (int i = 0; i < 32; ++i) pk[i] = pack_bf16x2(sv[hh * 64 + 2 * i], sv[hh * 64 + 2 * i + 1]);
-          tmem_st32u(tS + hh * 32, pk);
+          for (int i = 0; i < 32; ++i) pk[i] = pack_bf16x2(pv[2 * i], pv[2 * i + 1]);
+          tmem_st32u(dst_hi, pk);
           if (C::kSplit) {
 #pragma unroll
             for (int i = 0; i < 32; ++i) {
-              const __nv_bfloat162 hb = *reinterpret_cast<const __nv_bfloat162 *>(&pk[i]);
-              const float2 hf = __bfloat1622float2(hb);
-              pk[i] = pack_bf16x2(sv[hh * 64 + 2 * i] - hf.x, sv[hh * 64 + 2 * i + 1] - hf.y);
+              const float h0 = __uint_as_float(pk[i] << 16), h1 = __uint_as_float(pk[i] & 0xFFFF0000u);
+              pk[i] = pack_bf16x2(pv[2 * i] - h0, pv[2 * i + 1] - h1);
             }
-            tmem_st32u(tPlo + hh * 32, pk);
+            tmem_st32u(dst_lo, pk);
+          }
+        } else {
+          uint32_t pk[16];
+#pragma unroll
+          for (int i = 0; i < 16; ++i) pk[i] = pack_bf16x2(pv[2 * i], pv[2 * i + 1]);
+          tmem_st16u(dst_hi, pk);
+          if (C::kSplit) {
+#pragma unroll
+            for (int i = 0; i < 16; ++i) {
+              const float h0 = __uint_as_float(pk[i] << 16), h1 = __uint_as_float(pk[i] & 0xFFFF0000u);
+              pk[i] = pack_bf16x2(pv[2 * i] - h0, pv[2 * i + 1] - h1);
+            }
+            tmem_st16u(dst_lo, pk);
           }
         }
-      } else {
-      // pass 1: row max of this tile
-      float mx = -INFINITY;
+      };
+      auto tile_body = [&](auto masked_tag) {
+        constexpr bool kMask = decltype(masked_tag)::value;
+        auto val = [&](float x, int col) -> float {
+          if constexpr (kMask) return col < nvalid ? x : -INFINITY;
+          else return x;
+        };
+        if constexpr (C::kOnePass) {
+          float sv[BN];
 #pragma unroll
-      for (int cc = 0; cc < BN / 32; ++cc) {
-        float v[32];
-        tmem_ld32(tS + cc * 32, v);
-        tmem_wait_ld();
+          for (int cc = 0; cc < BN / 32; ++cc) {
+            float tmp[32];
+            tmem_ld32(tS + cc * 32, tmp);
 #pragma unroll
-        for (int i = 0; i < 32; ++i) mx = fmaxf(mx, (cc * 32 + i < nvalid) ? v[i] : -INFINITY);
-      }
-      mx *= sl2;
-      if (j == 0) {
-        m_run = mx;
-      } else if (mx > m_run + 8.f) {      // lazy rescale: only when the max grew by > 2^8
-        alpha = ex2_approx(m_run - mx);
-        m_run = mx;
-        resc = true;
-      }
-      // pass 2: P = 2^(s*scale*log2e - m) as bf16 pairs over S (chunk cc lands on
-      // columns [16cc, 16cc+16), all already read), lo parts in their own columns
-#pragma unroll
-      for (int cc = 0; cc < BN / 32; ++cc) {
-        float v[32];
-        tmem_ld32(tS + cc * 32, v);
-        tmem_wait_ld();
-#pragma unroll
-        for (int i = 0; i < 32; ++i) {
-          v[i] = (cc * 32 + i < nvalid) ? ex2_approx(fmaf(v[i], sl2, -m_run)) : 0.f;
-          if (i & 1) rs1 += v[i]; else rs0 += v[i];
-        }
-        uint32_t pk[16];
-#pragma unroll
-        for (int i = 0; i < 16; ++i) pk[i] = pack_bf16x2(v[2 * i], v[2 * i + 1]);
-        tmem_st16u(tS + cc * 16, pk);
-        if (C::kSplit) {
-#pragma unroll
-          for (int i = 0; i < 16; ++i) {
-            const __nv_bfloat162 hb = *reinterpret_cast<const __nv_bfloat162 *>(&pk[i]);
-            const float2 hf = __bfloat1622float2(hb);
-            pk[i] = pack_bf16x2(v[2 * i] - hf.x, v[2 * i + 1] - hf.y);
+            for (int i = 0; i < 32; ++i) sv[cc * 32 + i] = tmp[i];
           }
-          tmem_st16u(tPlo + cc * 16, pk);
+          tmem_wait_ld();
+          float m0 = -INFINITY, m1 = -INFINITY;
+#pragma unroll
+          for (int i = 0; i < BN; i += 4) {
+            sv[i] = val(sv[i], i);
+            sv[i + 1] = val(sv[i + 1], i + 1);
+            sv[i + 2] = val(sv[i + 2], i + 2);
+            sv[i + 3] = val(sv[i + 3], i + 3);
+            m0 = fmax3(m0, sv[i], sv[i + 1]);
+            m1 = fmax3(m1, sv[i + 2], sv[i + 3]);
+          }
+          update_max(fmaxf(m0, m1));
+#pragma unroll
+          for (int i = 0; i < BN; ++i) {
+            sv[i] = ex2_approx(fmaf(sv[i], sl2, -m_run));
+            if (i & 1) rs1 += sv[i]; else rs0 += sv[i];
+          }
+#pragma unroll
+          for (int hh = 0; hh < BN / 64; ++hh) store_p(sv + hh * 64, 32, tS + hh * 32, tPlo + hh * 32);
+        } else {
+          // pass 1: row max of this tile
+          float m0 = -INFINITY, m1 = -INFINITY;
+#pragma unroll
+          for (int cc = 0; cc < BN / 32; ++cc) {
+            float v[32];
+            tmem_ld32(tS + cc * 32, v);
+            tmem_wait_ld();
+#pragma unroll
+            for (int i = 0; i < 32; i += 4) {
+              m0 = fmax3(m0, val(v[i], cc * 32 + i), val(v[i + 1], cc * 32 + i + 1));
+              m1 = fmax3(m1, val(v[i + 2], cc * 32 + i + 2), val(v[i + 3], cc * 32 + i + 3));
+            }
+          }
+          update_max(fmaxf(m0, m1));
+          // pass 2: P = 2^(s*scale*log2e - m); chunk cc lands on columns [16cc, 16cc+16),
+          // all of them already read
+#pragma unroll
+          for (int cc = 0; cc < BN / 32; ++cc) {
+            float v[32];
+            tmem_ld32(tS + cc * 32, v);
+            tmem_wait_ld();
+#pragma unroll
+            for (int i = 0; i < 32; ++i) {
+              if constexpr (kMask) {
+                v[i] = (cc * 32 + i < nvalid) ? ex2_approx(fmaf(v[i], sl2, -m_run)) : 0.f;
+              } else {
+                v[i] = ex2_approx(fmaf(v[i], sl2, -m_run));
+              }
+              if (i & 1) rs1 += v[i]; else rs0 += v[i];
+            }
+            store_p(v, 16, tS + cc * 16, tPlo + cc * 16);
+          }
         }
-      }
-      }
+      };
+      if (nvalid >= BN) tile_body(std::false_type{});
+      else tile_body(std::true_type{});
       l_run = fmaf(l_run, alpha, rs0 + rs1);
       tmem_wait_st();
       // O is stable once the previous P.V has completed
