@@ -52,6 +52,23 @@ def parse_args():
     return ap.parse_args()
 
 
+# ----------------------------------------------------------------------------- ranks
+
+def rank_workload(w, rank: int):
+    """Weak scaling: every rank runs its own layer of the same shape, seeded
+    apart (heads are independent; nothing is exchanged on the data path)."""
+    return w.with_(seed=w.seed + rank)
+
+
+def max_over_ranks(t):
+    """Element-wise max of a float64 tensor over all ranks (the timing rule:
+    a multi-GPU number is the slowest rank's); identity without a process group."""
+    import torch.distributed as dist
+    if dist.is_available() and dist.is_initialized() and dist.get_world_size() > 1:
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return t
+
+
 # ----------------------------------------------------------------------------- inputs
 
 def _gen_head(args):
@@ -71,7 +88,8 @@ def make_inputs(w, rank: int):
     shape = (w.BH, w.N, w.d)
     s1 = [np.empty(shape, np.uint16) for _ in range(3)]
     s2 = [np.empty(shape, np.uint16) for _ in range(3)]
-    jobs = [(w.cfg_id, w.k, w.G, bh, w.seed + rank) for bh in range(w.BH)]
+    wr = rank_workload(w, rank)
+    jobs = [(w.cfg_id, w.k, w.G, bh, wr.seed) for bh in range(w.BH)]
     nproc = max(1, min(len(jobs), len(os.sched_getaffinity(0)), 16))
     with cf.ProcessPoolExecutor(nproc, mp_context=mp.get_context("spawn")) as ex:
         for bh, a, b in ex.map(_gen_head, jobs):
@@ -147,6 +165,33 @@ def measured_peaks():
     except Exception:
         return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0,
                 "source": "fallback"}
+
+
+def measured_traffic():
+    """{stage: bytes per launch} from profiles/traffic.txt, for stages whose
+    kernel sources still hash to what was profiled (else no entry)."""
+    import hashlib
+    csrc = os.path.join(ROOT, "sparse_attention_diffusion_mcs_b200", "csrc")
+    files = {"attn": ("mcs_common.cuh", "attn_kernel.cuh"), "colsum": ("mcs_common.cuh", "colsum_kernel.cuh")}
+    hashes = {}
+    for key, fs in files.items():
+        m = hashlib.sha256()
+        for f in fs:
+            with open(os.path.join(csrc, f), "rb") as fh:
+                m.update(fh.read())
+        hashes[key] = m.hexdigest()[:16]
+    out = {}
+    try:
+        for line in open(os.path.join(ROOT, "profiles", "traffic.txt")):
+            if line.startswith("#") or not line.strip():
+                continue
+            stage, kernel, hsh, rd, wr = line.split()
+            fam = "colsum" if kernel.startswith("colsum") else "attn"
+            if hashes.get(fam) == hsh:
+                out[stage] = int(rd) + int(wr)
+    except OSError:
+        pass
+    return out
 
 
 # ----------------------------------------------------------------------------- CPU baseline
@@ -326,9 +371,7 @@ def main():
     mean = {s: statistics.fmean(v) for s, v in per.items()}
 
     # max over ranks
-    vec = torch.tensor([total_ms] + [mean[s] for s in stages], dtype=torch.float64, device=dev)
-    if world > 1:
-        dist.all_reduce(vec, op=dist.ReduceOp.MAX)
+    vec = max_over_ranks(torch.tensor([total_ms] + [mean[s] for s in stages], dtype=torch.float64, device=dev))
     total_ms = float(vec[0])
     mean = {s: float(vec[1 + i]) for i, s in enumerate(stages)}
 
@@ -358,9 +401,7 @@ def main():
         b.record(stream)
         torch.cuda.synchronize()
         e2e_ms = a.elapsed_time(b) / args.steps
-        t = torch.tensor([e2e_ms], dtype=torch.float64, device=dev)
-        if world > 1:
-            dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        t = max_over_ranks(torch.tensor([e2e_ms], dtype=torch.float64, device=dev))
         e2e_ms = float(t[0])
         e2e = {"value": world * w.sparse_flops / (e2e_ms * 1e-3) / 1e12, "unit": "TFLOP/s",
                "ms_per_step": e2e_ms,
@@ -405,11 +446,13 @@ def main():
     kernels["step"]["hbm_frac"] = kernels["step"]["hbm_gbs"] / peaks["hbm_gbs"]
     kernels["step"]["gathered_kv_gbs"] = (BH * w.n_groups * 4.0 * kk * d) / (mean["step"] * 1e-3) / 1e9
 
+    traffic = measured_traffic()
+
     def roof(s):
         r = kernels[s]
         return {"kernel": s, "bound": r["bound"], "achieved": r["achieved"],
                 "peak": tc if r["bound"] == "tensor" else peaks["hbm_gbs"], "unit": r["unit"],
-                "frac": r["frac"], "traffic": None,
+                "frac": r["frac"], "traffic": traffic.get(s),
                 "peak_kind": f"{peaks['source']} bf16 sustained" if r["bound"] == "tensor"
                 else f"{peaks['source']} HBM copy"}
 
@@ -435,8 +478,8 @@ def main():
         "speedup_vs_dense": mean["dense"] / mean["step"],
         "amortized_speedup": S * mean["dense"] / (P * plan_ms + (S - P) * mean["step"]),
         "schedule": f"{S} denoising steps, plan at {list(w.plan_steps)}",
-        "roofline": roof("step"),
-        "roofline_dominant": roof(dom),
+        "roofline": roof(dom),
+        "roofline_reused_step": roof("step"),
         "kernels": kernels,
         "clocks": clk,
         "gpu_launches": KERNELS_PER_STEP * args.steps,
