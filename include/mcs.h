@@ -136,6 +136,17 @@ mcs_status mcs_plan_scores(const void *Q, const void *K, const int32_t *perm, in
 mcs_status mcs_plan_topk(int B, int H, int N, int d, int G, int k, int32_t *kv_idx,
                          void *workspace, size_t workspace_bytes, mcs_stream_t stream);
 
+/* a4 on caller-supplied scores: the selection mcs_plan_topk applies to the
+ * group probability sums (cctest.ai "Individual KV selection"), for any
+ * score matrix.  scores: float32 [rows, N] row-major on the device, meant to
+ * be >= 0 and finite (the sign bit is ignored, so -x ranks as x; NaN ranks
+ * above +inf).  kv_idx: int32 [rows, min(k,N)] on the device, caller-owned:
+ * per row the min(k,N) largest scores, ties to the lower index, ascending.
+ * rows == 0 is a no-op.  INVALID_ARG for null pointers, rows < 0, N < 1 or
+ * k < 1; CUDA for a launch failure.  Asynchronous on `stream`. */
+mcs_status mcs_select_topk(const float *scores, int rows, int N, int k, int32_t *kv_idx,
+                           mcs_stream_t stream);
+
 /* a5: residual float32 [B,H,N,d] = dense output (from mcs_plan_stats, same
  * Q, K, V) minus the output renormalised over each group's kept keys. */
 mcs_status mcs_plan_residual(const void *Q, const void *K, const void *V, const int32_t *perm,

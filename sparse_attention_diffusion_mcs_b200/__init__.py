@@ -16,6 +16,7 @@ from .api import (  # noqa: F401
     plan_select,
     plan_stats,
     plan_topk,
+    select_topk,
     selftest_wait_timeout,
     set_wait_limit_ns,
     sparse_step,

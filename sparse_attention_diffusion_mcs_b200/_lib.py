@@ -45,6 +45,7 @@ PROTOTYPES = {
     "mcs_plan_scores": (c_int, [c_vp, c_vp, c_vp, c_int, c_int, c_int, c_int, c_int, c_int, c_float,
                                 c_vp, c_size_t, c_vp]),
     "mcs_plan_topk": (c_int, [c_int, c_int, c_int, c_int, c_int, c_int, c_vp, c_vp, c_size_t, c_vp]),
+    "mcs_select_topk": (c_int, [c_vp, c_int, c_int, c_int, c_vp, c_vp]),
     "mcs_plan_residual": (c_int, [c_vp, c_vp, c_vp, c_vp, c_vp, c_int, c_int, c_int, c_int, c_int,
                                   c_int, c_float, c_vp, c_vp, c_size_t, c_vp]),
     "mcs_sparse_step": (c_int, [c_vp, c_vp, c_vp, PMETA, c_float, c_vp, c_vp]),

@@ -155,6 +155,23 @@ def plan_topk(B: int, H: int, N: int, d: int, G: int, k: int, workspace: torch.T
     return out
 
 
+def select_topk(scores: torch.Tensor, k: int, out: Optional[torch.Tensor] = None) -> torch.Tensor:
+    """Step a4 on any float32 score matrix [..., N]: int32 indices of the
+    min(k, N) largest per row, ties to the lower index, ascending."""
+    if scores.dtype != torch.float32 or not scores.is_cuda:
+        raise TypeError("scores must be a float32 CUDA tensor")
+    scores = scores.contiguous()
+    N = scores.shape[-1]
+    rows = scores.numel() // N if N else 0
+    kk = min(int(k), N)
+    if out is None:
+        out = torch.empty((*scores.shape[:-1], kk), dtype=torch.int32, device=scores.device)
+    if rows == 0:
+        return out
+    check(lib().mcs_select_topk(_ptr(scores), rows, N, int(k), _ptr(out), _stream()), "mcs_select_topk")
+    return out
+
+
 def plan_select(Q, K, perm, G: int, k: int, scale: Optional[float] = None,
                 workspace: Optional[torch.Tensor] = None) -> torch.Tensor:
     """Steps a2-a4 for a given grouping: int32 kv_idx [B, H, n_groups, min(k, N)]."""

@@ -1,6 +1,7 @@
 // colsum_kernel.cuh -- group probability sums, step a3 of the plan.
 //
 //   colsum[g, j] = sum_{i in group g} P_ij,  P_ij = 2^(s_ij*scale*log2e - m_i) / l_i
+//                                                = 2^(s_ij*scale*log2e - c_i),  c_i = m_i + log2(l_i)
 //
 // with (m_i, l_i) the exact row statistics from the dense pass ("KV indices
 // selected using exact attention probabilities", aiqbench.com abstract; the
@@ -39,7 +40,7 @@ struct ColsumCfg {
   static constexpr int K_BYTES = BM * D * 2;
   static constexpr int OFF_Q = 0;
   static constexpr int OFF_K = Q_BYTES;
-  static constexpr int OFF_STAT = OFF_K + NST * K_BYTES;     // float2 (m, 1/l) x 128
+  static constexpr int OFF_STAT = OFF_K + NST * K_BYTES;     // c_i = m_i + log2(l_i), 128 floats
   static constexpr int OFF_BAR = OFF_STAT + 128 * 8;
   static constexpr int N_BAR = 1 + 2 * NST + 5;              // q, k full/empty, s_full[2], s_free[2], drain
   static constexpr int OFF_MISC = OFF_BAR + 8 * N_BAR;
@@ -60,7 +61,7 @@ __global__ void __launch_bounds__(224, 1) colsum_kernel(const __grid_constant__ 
   const uint32_t sbase = smem_u32(smem);
   const uint32_t sQ = sbase + C::OFF_Q;
   const uint32_t sK0 = sbase + C::OFF_K;
-  float2 *stat = reinterpret_cast<float2 *>(smem + C::OFF_STAT);
+  float *stat = reinterpret_cast<float *>(smem + C::OFF_STAT);
   const uint32_t bar0 = sbase + C::OFF_BAR;
   const uint32_t b_q = bar0;
   auto b_kfull = [&](int s) { return bar0 + 8 * (1 + s); };
@@ -106,11 +107,8 @@ __global__ void __launch_bounds__(224, 1) colsum_kernel(const __grid_constant__ 
   }
   if (tid < 128) {
     const int q = q_token(tid);
-    if (q >= 0) {
-      stat[tid] = make_float2(a.row_m[head + q], 1.f / a.row_l[head + q]);
-    } else {
-      stat[tid] = make_float2(INFINITY, 0.f);   // padding query contributes 0
-    }
+    // fold the normaliser into the exponent; a padding query contributes 2^-inf = 0
+    stat[tid] = q >= 0 ? a.row_m[head + q] + log2f(a.row_l[head + q]) : INFINITY;
   }
   if (warp == 4) {
     tmem_alloc(smem_u32(tmem_slot), C::TMEM_COLS);
@@ -203,24 +201,28 @@ __global__ void __launch_bounds__(224, 1) colsum_kernel(const __grid_constant__ 
       const int b = j & 1;
       if (!mbar_wait(b_sfull0 + 8 * b, (j >> 1) & 1, a.wait_ns, abort_flag)) { ok = false; break; }
       tc_fence_after();
-      float acc0 = 0.f, acc1 = 0.f;
+      float acc0 = 0.f, acc1 = 0.f, acc2 = 0.f, acc3 = 0.f;
 #pragma unroll
       for (int cc = 0; cc < 4; ++cc) {
         float v[32];
         tmem_ld32(tbase + lane_addr + b * 128 + cc * 32, v);
         tmem_wait_ld();
+        const float4 *c4 = reinterpret_cast<const float4 *>(stat + cc * 32);
 #pragma unroll
-        for (int i = 0; i < 32; i += 2) {
-          const float2 s0 = stat[cc * 32 + i];
-          const float2 s1 = stat[cc * 32 + i + 1];
-          acc0 = fmaf(ex2_approx(fmaf(v[i], sl2, -s0.x)), s0.y, acc0);
-          acc1 = fmaf(ex2_approx(fmaf(v[i + 1], sl2, -s1.x)), s1.y, acc1);
+        for (int i = 0; i < 32; i += 4) {
+          const float4 c = c4[i / 4];     // same address in every lane: one broadcast read
+          acc0 += ex2_approx(fmaf(v[i], sl2, -c.x));
+          acc1 += ex2_approx(fmaf(v[i + 1], sl2, -c.y));
+          acc2 += ex2_approx(fmaf(v[i + 2], sl2, -c.z));
+          acc3 += ex2_approx(fmaf(v[i + 3], sl2, -c.w));
         }
       }
+      acc0 += acc1;
+      acc2 += acc3;
       tc_fence_before();
       mbar_arrive(b_sfree0 + 8 * b);
       const int key = j * BM + tid;
-      if (key < N) out[key] = acc0 + acc1;
+      if (key < N) out[key] = acc0 + acc2;
     }
     if (!ok && !*abort_flag) {
       *abort_flag = 1;

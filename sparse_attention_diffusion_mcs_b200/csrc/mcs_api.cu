@@ -244,11 +244,28 @@ cudaError_t run_scores(const void *Q, const void *K, const int32_t *perm, int BH
   return cudaGetLastError();
 }
 
+// top-k of `rows` rows of N scores each, k <= N
+cudaError_t launch_topk(const float *scores, int rows, int N, int k, int32_t *kv_idx, cudaStream_t s) {
+  if (rows == 0) return cudaSuccess;
+  const bool cache = static_cast<size_t>(N) * 4 <= static_cast<size_t>(kTopkRowCacheBytes);
+  const int smem = kTopkFixedSmem + (cache ? N * 4 : 0);
+  cudaError_t e;
+  if (N % 4 == 0 && aligned16(scores)) {
+    e = set_smem(topk_kernel<4>, smem);
+    if (e != cudaSuccess) return e;
+    topk_kernel<4><<<rows, kTopkThreads, smem, s>>>(scores, N, k, cache ? 1 : 0, kv_idx);
+  } else {
+    e = set_smem(topk_kernel<1>, smem);
+    if (e != cudaSuccess) return e;
+    topk_kernel<1><<<rows, kTopkThreads, smem, s>>>(scores, N, k, cache ? 1 : 0, kv_idx);
+  }
+  return cudaGetLastError();
+}
+
 cudaError_t run_topk(int BH, int N, int G, int k, int32_t *kv_idx, void *ws, const PlanWs &w,
                      cudaStream_t s) {
   const int ng = (N + G - 1) / G;
-  topk_kernel<<<BH * ng, kTopkThreads, 0, s>>>(at<float>(ws, w.colsum), N, k, kv_idx);
-  return cudaGetLastError();
+  return launch_topk(at<float>(ws, w.colsum), BH * ng, N, k, kv_idx, s);
 }
 
 cudaError_t run_residual(const void *Q, const void *K, const void *V, const int32_t *perm,
@@ -391,6 +408,13 @@ mcs_status mcs_plan_topk(int B, int H, int N, int d, int G, int k, int32_t *kv_i
   if (st != MCS_OK) return st;
   return cuda_status(run_topk(B * H, N, G, k < N ? k : N, kv_idx, workspace, w,
                               reinterpret_cast<cudaStream_t>(stream)));
+}
+
+mcs_status mcs_select_topk(const float *scores, int rows, int N, int k, int32_t *kv_idx,
+                           mcs_stream_t stream) {
+  if (!scores || !kv_idx || rows < 0 || N < 1 || k < 1) return MCS_ERR_INVALID_ARG;
+  return cuda_status(launch_topk(scores, rows, N, k < N ? k : N, kv_idx,
+                                 reinterpret_cast<cudaStream_t>(stream)));
 }
 
 mcs_status mcs_plan_residual(const void *Q, const void *K, const void *V, const int32_t *perm,

@@ -97,6 +97,12 @@ def test_plan_argument_errors(L):
     assert L.mcs_plan_scores(FAKE, FAKE, None, 1, 1, 10, 64, 64, 4, 0.1, FAKE, 1 << 20, None) == INVALID
     assert L.mcs_plan_topk(1, 1, 10, 64, 64, 4, None, FAKE, 1 << 20, None) == INVALID
     assert L.mcs_plan_topk(1, 1, 10, 64, 64, 4, FAKE, FAKE, 16, None) == WORKSPACE
+    assert L.mcs_select_topk(None, 4, 10, 3, FAKE, None) == INVALID
+    assert L.mcs_select_topk(FAKE, 4, 10, 3, None, None) == INVALID
+    assert L.mcs_select_topk(FAKE, -1, 10, 3, FAKE, None) == INVALID
+    assert L.mcs_select_topk(FAKE, 4, 0, 3, FAKE, None) == INVALID
+    assert L.mcs_select_topk(FAKE, 4, 10, 0, FAKE, None) == INVALID
+    assert L.mcs_select_topk(FAKE, 0, 10, 3, FAKE, None) == OK          # no rows: nothing launched
     assert L.mcs_plan_residual(FAKE, FAKE, FAKE, FAKE, FAKE, 1, 1, 10, 64, 64, 4, 0.1, None,
                                FAKE, 1 << 20, None) == INVALID
 
