@@ -10,7 +10,8 @@
 // the order of the exact projections up to fp64 rounding:
 //   mean_kernel       per (head, chunk of rows): column sums of Q
 //   cov_kernel        per (head, chunk): sum of (q - mu)(q - mu)^T
-//   eig_kernel        per head: combine chunks, top eigenvector by repeated
+//   cov_reduce_kernel per head: C = sum of the chunk partials / N
+//   eig_kernel        per head: top eigenvector of C by repeated
 //                     squaring + power iteration, sign fixed so the
 //                     largest-magnitude component is positive
 //   project_kernel    p_n = (q_n - mu) . v  -> order-preserving uint64 key
@@ -21,7 +22,7 @@
 
 namespace mcs {
 
-constexpr int kGroupChunk = 2048;     // rows per chunk of the mean / covariance passes
+constexpr int kGroupChunk = 1024;     // rows per chunk of the mean / covariance passes
 constexpr int kSortThreads = 1024;
 
 // ---------------------------------------------------------------- mean
@@ -58,72 +59,112 @@ __global__ void mean_finalize_kernel(const double *__restrict__ part, int N, int
 }
 
 // ---------------------------------------------------------------- covariance
-// 256 threads; thread (ti, tj) accumulates an RxR block of the DxD matrix in
-// fp64, R = D/16.  Rows are staged (centred) through shared memory.
+// 256 threads as a 16 x 16 grid; thread (ti, tj) accumulates C[ti + 16a][tj + 16b]
+// for a, b < R = D/16 in fp64 registers (columns interleaved so the shared
+// memory reads of one warp hit distinct banks).  Rows are centred and staged
+// through a double-buffered shared tile, the next tile's 16-byte loads in
+// flight while the current one is consumed.  The mirror entry C[j][i] is the
+// same sequence of fma(x_i, x_j, .) in the same row order, so the partial
+// matrices are exactly symmetric.
 template <int D>
 __global__ void __launch_bounds__(256) cov_kernel(const bf16 *__restrict__ Q, const double *__restrict__ mean,
                                                   int N, int n_chunks, double *__restrict__ part) {
   constexpr int R = D / 16;
   constexpr int ROWS = 16;
-  __shared__ double xs[ROWS][D + 1];
+  constexpr int VPR = D / 8;             // 16-byte vectors per row
+  constexpr int NV = ROWS * VPR;         // vectors per staged tile (<= 256)
+  __shared__ double xs[2][ROWS][D];
   const int chunk = blockIdx.x, bh = blockIdx.y;
   const int r0 = chunk * kGroupChunk;
   const int r1 = min(N, r0 + kGroupChunk);
-  const int ti = threadIdx.x / 16, tj = threadIdx.x % 16;
+  const int tid = threadIdx.x, ti = tid / 16, tj = tid % 16;
   const bf16 *q = Q + static_cast<size_t>(bh) * N * D;
   const double *mu = mean + bh * D;
+  const bool stager = tid < NV;
+  const int srow = tid / VPR, scol = (tid % VPR) * 8;
+  double mus[8];
+#pragma unroll
+  for (int e = 0; e < 8; ++e) mus[e] = stager ? mu[scol + e] : 0.0;
+  auto fetch = [&](int rb) -> uint4 {
+    const int r = rb + srow;
+    if (stager && r < r1) return __ldg(reinterpret_cast<const uint4 *>(q + static_cast<size_t>(r) * D + scol));
+    return make_uint4(0u, 0u, 0u, 0u);
+  };
+  auto stage = [&](int buf, int rb, uint4 v) {
+    if (!stager) return;
+    const bool live = rb + srow < r1;
+    const bf16 *h = reinterpret_cast<const bf16 *>(&v);
+#pragma unroll
+    for (int e = 0; e < 8; ++e)
+      xs[buf][srow][scol + e] = live ? static_cast<double>(__bfloat162float(h[e])) - mus[e] : 0.0;
+  };
   double acc[R][R];
 #pragma unroll
-  for (int i = 0; i < R; ++i)
+  for (int a = 0; a < R; ++a)
 #pragma unroll
-    for (int j = 0; j < R; ++j) acc[i][j] = 0.0;
+    for (int b = 0; b < R; ++b) acc[a][b] = 0.0;
+  int buf = 0;
+  stage(0, r0, fetch(r0));
+  __syncthreads();
   for (int rb = r0; rb < r1; rb += ROWS) {
-    __syncthreads();
-    for (int e = threadIdx.x; e < ROWS * D; e += 256) {
-      const int rr = e / D, c = e % D;
-      const int r = rb + rr;
-      xs[rr][c] = r < r1 ? static_cast<double>(__bfloat162float(q[static_cast<size_t>(r) * D + c])) - mu[c] : 0.0;
-    }
-    __syncthreads();
-#pragma unroll 2
+    const bool more = rb + ROWS < r1;
+    const uint4 nxt = more ? fetch(rb + ROWS) : make_uint4(0u, 0u, 0u, 0u);
+#pragma unroll 4
     for (int rr = 0; rr < ROWS; ++rr) {
       double xi[R], xj[R];
 #pragma unroll
-      for (int i = 0; i < R; ++i) {
-        xi[i] = xs[rr][ti * R + i];
-        xj[i] = xs[rr][tj * R + i];
+      for (int a = 0; a < R; ++a) {
+        xi[a] = xs[buf][rr][ti + 16 * a];
+        xj[a] = xs[buf][rr][tj + 16 * a];
       }
 #pragma unroll
-      for (int i = 0; i < R; ++i)
+      for (int a = 0; a < R; ++a)
 #pragma unroll
-        for (int j = 0; j < R; ++j) acc[i][j] = fma(xi[i], xj[j], acc[i][j]);
+        for (int b = 0; b < R; ++b) acc[a][b] = fma(xi[a], xj[b], acc[a][b]);
     }
+    if (more) stage(buf ^ 1, rb + ROWS, nxt);
+    __syncthreads();
+    buf ^= 1;
   }
   double *out = part + (static_cast<size_t>(bh) * n_chunks + chunk) * D * D;
 #pragma unroll
-  for (int i = 0; i < R; ++i)
+  for (int a = 0; a < R; ++a)
 #pragma unroll
-    for (int j = 0; j < R; ++j) out[(ti * R + i) * D + tj * R + j] = acc[i][j];
+    for (int b = 0; b < R; ++b) out[(ti + 16 * a) * D + tj + 16 * b] = acc[a][b];
+}
+
+// C = (sum of the chunk partials, in chunk order) / N; one thread per entry.
+template <int D>
+__global__ void __launch_bounds__(256) cov_reduce_kernel(const double *__restrict__ part, int N, int n_chunks,
+                                                         double *__restrict__ cov) {
+  const int bh = blockIdx.y;
+  const int e = blockIdx.x * 256 + threadIdx.x;
+  if (e >= D * D) return;
+  const double *p = part + static_cast<size_t>(bh) * n_chunks * D * D + e;
+  double sum = 0.0;
+  for (int i = 0; i < n_chunks; ++i) sum += p[static_cast<size_t>(i) * D * D];
+  cov[static_cast<size_t>(bh) * D * D + e] = sum / N;
 }
 
 // ---------------------------------------------------------------- eigenvector
-// One CTA of 256 threads per head.  C (fp64) and the squaring scratch live in
-// workspace (L2-resident, D*D doubles each); M, a normalised power of C
-// obtained by repeated squaring, lives in shared memory.  Squaring separates
-// the top eigenvector even for small spectral gaps; a few power iterations
-// with M and then with C itself give v.
+// One CTA of 256 threads per head.  M, a normalised power of C obtained by
+// repeated squaring, lives in shared memory; squaring separates the top
+// eigenvector even for small spectral gaps.  A few power iterations with M
+// and then with C itself (copied into the same shared buffer) give v.
+// M stays exactly symmetric (T[i][j] and T[j][i] are the same fma sequence),
+// so T = M.M is formed as sum_t M[t][i] M[t][j]: both operands are read from
+// row t, and thread (ti, tj) keeps its R x R block of T in registers.
 template <int D>
-__global__ void __launch_bounds__(256) eig_kernel(const double *__restrict__ part, int N, int n_chunks,
-                                                  double *__restrict__ cov, double *__restrict__ scratch,
-                                                  double *__restrict__ vdir, float *__restrict__ lambda) {
+__global__ void __launch_bounds__(256) eig_kernel(const double *__restrict__ cov, double *__restrict__ vdir,
+                                                  float *__restrict__ lambda) {
+  constexpr int R = D / 16;
   extern __shared__ double dsm[];
   double *M = dsm;               // D*D
   double *vec = M + D * D;       // D
-  double *tmp = vec + D;         // D
+  double *tmp = vec + D;         // 2*D
   __shared__ double red[256];
-  const int bh = blockIdx.x, tid = threadIdx.x;
-  double *Cm = cov + static_cast<size_t>(bh) * D * D;
-  double *T = scratch + static_cast<size_t>(bh) * D * D;
+  const int bh = blockIdx.x, tid = threadIdx.x, ti = tid / 16, tj = tid % 16;
+  const double *Cm = cov + static_cast<size_t>(bh) * D * D;
 
   auto block_sum = [&](double x) -> double {
     red[tid] = x;
@@ -137,12 +178,6 @@ __global__ void __launch_bounds__(256) eig_kernel(const double *__restrict__ par
     return r;
   };
 
-  for (int e = tid; e < D * D; e += 256) {
-    double sum = 0.0;
-    for (int i = 0; i < n_chunks; ++i) sum += part[(static_cast<size_t>(bh) * n_chunks + i) * D * D + e];
-    Cm[e] = sum / N;
-  }
-  __syncthreads();
   const double tr = block_sum(tid < D ? Cm[tid * D + tid] : 0.0);
   if (!(tr > 0.0)) {   // all queries identical: every direction is principal; take e_0
     if (tid < D) vdir[bh * D + tid] = tid == 0 ? 1.0 : 0.0;
@@ -152,15 +187,33 @@ __global__ void __launch_bounds__(256) eig_kernel(const double *__restrict__ par
   for (int e = tid; e < D * D; e += 256) M[e] = Cm[e] / tr;
   __syncthreads();
   for (int sq = 0; sq < 10; ++sq) {        // M <- M^2 / trace(M^2)  ->  C^(2^10), normalised
-    for (int e = tid; e < D * D; e += 256) {
-      const int i = e / D, j = e % D;
-      double acc = 0.0;
-      for (int t = 0; t < D; ++t) acc += M[i * D + t] * M[t * D + j];
-      T[e] = acc;
+    double acc[R][R];
+#pragma unroll
+    for (int a = 0; a < R; ++a)
+#pragma unroll
+      for (int b = 0; b < R; ++b) acc[a][b] = 0.0;
+#pragma unroll 2
+    for (int t = 0; t < D; ++t) {
+      double xi[R], xj[R];
+#pragma unroll
+      for (int a = 0; a < R; ++a) {
+        xi[a] = M[t * D + ti + 16 * a];
+        xj[a] = M[t * D + tj + 16 * a];
+      }
+#pragma unroll
+      for (int a = 0; a < R; ++a)
+#pragma unroll
+        for (int b = 0; b < R; ++b) acc[a][b] = fma(xi[a], xj[b], acc[a][b]);
     }
-    __syncthreads();
-    const double t2 = block_sum(tid < D ? T[tid * D + tid] : 0.0);
-    for (int e = tid; e < D * D; e += 256) M[e] = T[e] / t2;
+    double dsum = 0.0;
+    if (ti == tj)
+#pragma unroll
+      for (int a = 0; a < R; ++a) dsum += acc[a][a];
+    const double t2 = block_sum(dsum);     // its barriers also end every read of M
+#pragma unroll
+    for (int a = 0; a < R; ++a)
+#pragma unroll
+      for (int b = 0; b < R; ++b) M[(ti + 16 * a) * D + tj + 16 * b] = acc[a][b] / t2;
     __syncthreads();
   }
   // start from the column of M with the largest diagonal entry
@@ -175,20 +228,30 @@ __global__ void __launch_bounds__(256) eig_kernel(const double *__restrict__ par
   __syncthreads();
   if (tid < D) vec[tid] = M[tid * D + best];
   __syncthreads();
-  auto matvec_norm = [&](const double *A) {
-    if (tid < D) {
-      double acc = 0.0;
-      for (int t = 0; t < D; ++t) acc += A[tid * D + t] * vec[t];
-      tmp[tid] = acc;
+  // y = A v for the symmetric A in shared memory: y_i = sum_t A[t][i] v_t, the
+  // two halves of t on two threads, then normalise
+  auto matvec_norm = [&]() {
+    const int i = tid % D, h = tid / D;
+    if (h < 2) {
+      double a0 = 0.0, a1 = 0.0;
+      const int t0 = h * (D / 2);
+      for (int t = t0; t < t0 + D / 2; t += 2) {
+        a0 = fma(M[t * D + i], vec[t], a0);
+        a1 = fma(M[(t + 1) * D + i], vec[t + 1], a1);
+      }
+      tmp[h * D + i] = a0 + a1;
     }
     __syncthreads();
-    const double nn = block_sum(tid < D ? tmp[tid] * tmp[tid] : 0.0);
+    const double y = tid < D ? tmp[tid] + tmp[D + tid] : 0.0;
+    const double nn = block_sum(y * y);
     const double inv = nn > 0.0 ? 1.0 / sqrt(nn) : 0.0;
-    if (tid < D) vec[tid] = tmp[tid] * inv;
+    if (tid < D) vec[tid] = y * inv;
     __syncthreads();
   };
-  for (int it = 0; it < 8; ++it) matvec_norm(M);
-  for (int it = 0; it < 64; ++it) matvec_norm(Cm);
+  for (int it = 0; it < 8; ++it) matvec_norm();
+  for (int e = tid; e < D * D; e += 256) M[e] = Cm[e];
+  __syncthreads();
+  for (int it = 0; it < 64; ++it) matvec_norm();
   // sign: the first component of largest magnitude is positive
   if (tid == 0) {
     int im = 0;
@@ -199,9 +262,10 @@ __global__ void __launch_bounds__(256) eig_kernel(const double *__restrict__ par
   __syncthreads();
   const double sg = red[0];
   __syncthreads();
+  // Rayleigh quotient v.C.v for the eigenvalue
   if (tid < D) {
     double acc = 0.0;
-    for (int t = 0; t < D; ++t) acc += Cm[tid * D + t] * vec[t];
+    for (int t = 0; t < D; ++t) acc = fma(M[t * D + tid], vec[t], acc);
     tmp[tid] = acc * vec[tid];
   }
   __syncthreads();

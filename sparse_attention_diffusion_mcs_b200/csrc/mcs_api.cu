@@ -139,7 +139,7 @@ AttnArgs base_args(int N, float scale) {
 
 // ---------------------------------------------------------------- plan workspace
 struct PlanWs {
-  size_t mean_part, mean, cov_part, cov64, sq64, vdir, lambda, keys0, vals0, keys1, vals1;
+  size_t mean_part, mean, cov_part, cov64, vdir, lambda, keys0, vals0, keys1, vals1;
   size_t row_m, row_l, O32, colsum, total;
 };
 
@@ -158,7 +158,6 @@ PlanWs plan_ws(int B, int H, int N, int d, int G) {
   w.mean = take(BH * d * 8);
   w.cov_part = take(BH * nch * d * d * 8);
   w.cov64 = take(BH * d * d * 8);
-  w.sq64 = take(BH * d * d * 8);
   w.vdir = take(BH * d * 8);
   w.lambda = take(BH * 4);
   w.keys0 = take(BH * N * 8);
@@ -189,11 +188,12 @@ cudaError_t run_group(const void *Q, int BH, int N, int32_t *perm, void *ws, con
   mean_kernel<D><<<dim3(nch, BH), 256, 0, s>>>(q, N, nch, at<double>(ws, w.mean_part));
   mean_finalize_kernel<D><<<BH, D, 0, s>>>(at<double>(ws, w.mean_part), N, nch, at<double>(ws, w.mean));
   cov_kernel<D><<<dim3(nch, BH), 256, 0, s>>>(q, at<double>(ws, w.mean), N, nch, at<double>(ws, w.cov_part));
-  const int eig_smem = (D * D + 2 * D) * 8;
+  cov_reduce_kernel<D><<<dim3((D * D + 255) / 256, BH), 256, 0, s>>>(at<double>(ws, w.cov_part), N, nch,
+                                                                      at<double>(ws, w.cov64));
+  const int eig_smem = (D * D + 3 * D) * 8;
   cudaError_t e = set_smem(eig_kernel<D>, eig_smem);
   if (e != cudaSuccess) return e;
-  eig_kernel<D><<<BH, 256, eig_smem, s>>>(at<double>(ws, w.cov_part), N, nch, at<double>(ws, w.cov64),
-                                           at<double>(ws, w.sq64), at<double>(ws, w.vdir),
+  eig_kernel<D><<<BH, 256, eig_smem, s>>>(at<double>(ws, w.cov64), at<double>(ws, w.vdir),
                                            at<float>(ws, w.lambda));
   project_kernel<D><<<dim3((N + 7) / 8, BH), 256, 0, s>>>(q, at<double>(ws, w.mean), at<double>(ws, w.vdir), N,
                                                            at<unsigned long long>(ws, w.keys0),
