@@ -65,6 +65,7 @@ struct alignas(64) AttnArgs {
   float *row_m, *row_l;    // [BH, N]               kModePlanDense (log2 domain)
   unsigned *status;        // device status word
   uint64_t wait_ns;        // bound on any single wait
+  int BH;                  // heads; work items are (head, query tile or group) pairs
 };
 
 template <int D, int MODE>
@@ -83,7 +84,7 @@ struct AttnCfg {
   static constexpr int OFF_K = OFF_Q + Q_BYTES;
   static constexpr int OFF_V = OFF_K + NK * KV_BYTES;
   static constexpr int OFF_BAR = OFF_V + NV * KV_BYTES;
-  static constexpr int N_BAR = 1 + 2 * NK + 2 * NV + 2 + 3;   // q, k/v full/empty, s_full[2], p, pv, drain
+  static constexpr int N_BAR = 1 + 2 * NK + 2 * NV + 2 + 4;   // q, k/v full/empty, s_full[2], p, pv, drain, q_empty
   static constexpr int OFF_MISC = OFF_BAR + 8 * N_BAR;
   static constexpr int SMEM = OFF_MISC + 16 + 1024;          // + slack to align the base to 1 KB
   static constexpr int THREADS = kSparse ? 384 : 224;
@@ -119,35 +120,50 @@ __global__ void __launch_bounds__(AttnCfg<D, MODE>::THREADS, 1) attn_kernel(cons
   const uint32_t b_p = b_sfull0 + 16;
   const uint32_t b_pv = b_sfull0 + 24;
   const uint32_t b_drain = b_sfull0 + 32;
+  const uint32_t b_qempty = b_sfull0 + 40;
   uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem + C::OFF_MISC);
   volatile int *abort_flag = reinterpret_cast<volatile int *>(smem + C::OFF_MISC + 4);
 
   const int tid = threadIdx.x;
   const int warp = tid >> 5;
   const int lane = tid & 31;
-  const int tile = blockIdx.x;          // query tile (dense) or query group (sparse)
-  const int bh = blockIdx.y;
   const int N = a.N;
-  const size_t head = static_cast<size_t>(bh) * N;
-
+  // Work items are (head, query tile) pairs (dense modes) or (head, query
+  // group) pairs (sparse modes), head-major; CTA c takes items c, c + grid,
+  // c + 2 grid, ...  Every item has the same number of key tiles T, so the
+  // rings, S buffers and barrier phases run on one tile counter per CTA and
+  // the next item's loads and first Q.K^T overlap this item's epilogue.
+  const int per_head = C::kSparse ? a.n_groups : (N + BM - 1) / BM;
+  const int n_items = a.BH * per_head;
   const int nkeys = C::kSparse ? a.k : N;
   const int T = (nkeys + BN - 1) / BN;
-  const int32_t *kv_list =
-      C::kSparse ? a.kv_idx + (static_cast<size_t>(bh) * a.n_groups + tile) * a.k : nullptr;
+  struct Item {
+    int tile, bh;
+    size_t head;
+    const int32_t *kv_list;
+  };
+  auto item_at = [&](int item) -> Item {
+    Item w;
+    w.tile = item % per_head;
+    w.bh = item / per_head;
+    w.head = static_cast<size_t>(w.bh) * N;
+    w.kv_list = C::kSparse ? a.kv_idx + (static_cast<size_t>(w.bh) * a.n_groups + w.tile) * a.k : nullptr;
+    return w;
+  };
 
-  // query row r of this tile -> token index, or -1 when the row is padding
-  auto q_token = [&](int r) -> int {
+  // query row r of an item -> token index, or -1 when the row is padding
+  auto q_token = [&](const Item &w, int r) -> int {
     if (C::kSparse) {
-      const int gr = tile * a.G + r;
+      const int gr = w.tile * a.G + r;
       if (r >= a.G || gr >= N) return -1;
-      const int q = a.perm[head + gr];
+      const int q = a.perm[w.head + gr];
       if (static_cast<unsigned>(q) >= static_cast<unsigned>(N)) {   // corrupt metadata: never gather out of range
         record_status(a.status, kStatusBadMeta);
         return -1;
       }
       return q;
     } else {
-      const int q = tile * BM + r;
+      const int q = w.tile * BM + r;
       return q < N ? q : -1;
     }
   };
@@ -167,6 +183,7 @@ __global__ void __launch_bounds__(AttnCfg<D, MODE>::THREADS, 1) attn_kernel(cons
     mbar_init(b_p, 128);
     mbar_init(b_pv, 1);
     mbar_init(b_drain, 1);
+    mbar_init(b_qempty, 1);
     *abort_flag = 0;
     mbar_init_fence();
   }
@@ -201,57 +218,68 @@ __global__ void __launch_bounds__(AttnCfg<D, MODE>::THREADS, 1) attn_kernel(cons
     const int op = active ? op_raw : h;
     const int quad = op % 32, dbk = op / 32;
     bool ok = true;
-    if (is_k) {
-      // the Q tile, once
-      if (C::kSparse) {
-        const int q0 = q_token(0);
-        const int fallback = q0 >= 0 ? q0 : 0;   // padding rows re-read a valid row
-        int rows[4];
+    int issued = 0;                           // fills of this ring by this CTA
+    int nq = 0;                               // Q tiles loaded (K ring warps)
+    for (int item = blockIdx.x, it = 0; item < n_items && ok; item += gridDim.x, ++it) {
+      const Item w = item_at(item);
+      // global row indices of tile t for this lane's gather4 (sparse modes)
+      auto tile_rows = [&](int t, int (&rows)[4]) {
+        const int first = w.kv_list[0];
 #pragma unroll
         for (int i = 0; i < 4; ++i) {
-          const int q = q_token(4 * quad + i);
-          rows[i] = static_cast<int>(head) + (q >= 0 ? q : fallback);
+          const int pos = t * BN + 4 * quad + i;
+          int key = pos < nkeys ? w.kv_list[pos] : first;   // padding keys re-read a valid key (masked later)
+          if (static_cast<unsigned>(key) >= static_cast<unsigned>(N)) {   // corrupt metadata
+            record_status(a.status, kStatusBadMeta);
+            key = 0;
+          }
+          rows[i] = static_cast<int>(w.head) + key;
         }
-        if (h == 0 && lane == 0) mbar_arrive_expect_tx(b_q, TILE_TX);
-        __syncwarp();
-        if (active)
-          tma_gather4(sQ + dbk * (BM * 128) + quad * 512, &a.tmQ, dbk * 64, rows[0], rows[1], rows[2], rows[3], b_q);
-      } else if (h == 0 && lane == 0) {
-        mbar_arrive_expect_tx(b_q, TILE_TX);
-#pragma unroll
-        for (int db = 0; db < NDB; ++db) tma_load_3d(sQ + db * (BM * 128), &a.tmQ, db * 64, tile * BM, bh, b_q);
-      }
-    }
-    // global row indices of tile t for this lane's gather4 (sparse modes)
-    auto tile_rows = [&](int t, int (&rows)[4]) {
-      const int first = kv_list[0];
-#pragma unroll
-      for (int i = 0; i < 4; ++i) {
-        const int pos = t * BN + 4 * quad + i;
-        int key = pos < nkeys ? kv_list[pos] : first;     // padding keys re-read a valid key (masked later)
-        if (static_cast<unsigned>(key) >= static_cast<unsigned>(N)) {   // corrupt metadata
-          record_status(a.status, kStatusBadMeta);
-          key = 0;
-        }
-        rows[i] = static_cast<int>(head) + key;
-      }
-    };
-    const bool dense_idle = false;            // dense: one warp per ring, lane 0 issues
-    int issued = 0;
-    if (!dense_idle) {
+      };
       int rows[4] = {0, 0, 0, 0}, next[4] = {0, 0, 0, 0};
       if (C::kSparse) tile_rows(0, rows);
+      if (is_k) {
+        // the item's Q tile, once the previous item's last Q.K^T has read the buffer
+        if (it > 0) {
+          int got = 1;
+          if (lane == 0) got = mbar_wait(b_qempty, (it - 1) & 1, a.wait_ns, abort_flag);
+          got = __shfl_sync(0xffffffffu, got, 0);
+          if (!got) { ok = false; break; }
+        }
+        if (C::kSparse) {
+          const int q0 = q_token(w, 0);
+          const int fallback = q0 >= 0 ? q0 : 0;   // padding rows re-read a valid row
+          int qrows[4];
+#pragma unroll
+          for (int i = 0; i < 4; ++i) {
+            const int q = q_token(w, 4 * quad + i);
+            qrows[i] = static_cast<int>(w.head) + (q >= 0 ? q : fallback);
+          }
+          if (h == 0 && lane == 0) mbar_arrive_expect_tx(b_q, TILE_TX);
+          __syncwarp();
+          if (active)
+            tma_gather4(sQ + dbk * (BM * 128) + quad * 512, &a.tmQ, dbk * 64, qrows[0], qrows[1], qrows[2],
+                        qrows[3], b_q);
+        } else if (h == 0 && lane == 0) {
+          mbar_arrive_expect_tx(b_q, TILE_TX);
+#pragma unroll
+          for (int db = 0; db < NDB; ++db)
+            tma_load_3d(sQ + db * (BM * 128), &a.tmQ, db * 64, w.tile * BM, w.bh, b_q);
+        }
+        ++nq;
+      }
       for (int j = 0; j < T; ++j) {
-        const int s = j % NS;
+        const int s = issued % NS;
         if (C::kSparse && j + 1 < T) tile_rows(j + 1, next);   // in flight while we wait for the slot
         int got = 1;
-        if (lane == 0) got = mbar_wait(is_k ? b_kempty(s) : b_vempty(s), ((j / NS) & 1) ^ 1, a.wait_ns, abort_flag);
+        if (lane == 0)
+          got = mbar_wait(is_k ? b_kempty(s) : b_vempty(s), ((issued / NS) & 1) ^ 1, a.wait_ns, abort_flag);
         got = __shfl_sync(0xffffffffu, got, 0);
         if (!got) { ok = false; break; }
         const uint32_t full = is_k ? b_kfull(s) : b_vfull(s);
         const uint32_t dst = ring + s * C::KV_BYTES;
         if (C::kSparse) {
-          // one expect-tx arrival per phase; the other warp's bytes may land first
+          // one expect-tx arrival per phase; the other warps' bytes may land first
           if (h == 0 && lane == 0) mbar_arrive_expect_tx(full, TILE_TX);
           __syncwarp();
           if (active)
@@ -261,7 +289,7 @@ __global__ void __launch_bounds__(AttnCfg<D, MODE>::THREADS, 1) attn_kernel(cons
         } else if (lane == 0) {
           mbar_arrive_expect_tx(full, TILE_TX);
 #pragma unroll
-          for (int db = 0; db < NDB; ++db) tma_load_3d(dst + db * (BN * 128), tm, db * 64, j * BN, bh, full);
+          for (int db = 0; db < NDB; ++db) tma_load_3d(dst + db * (BN * 128), tm, db * 64, j * BN, w.bh, full);
         }
         ++issued;
       }
@@ -275,7 +303,7 @@ __global__ void __launch_bounds__(AttnCfg<D, MODE>::THREADS, 1) attn_kernel(cons
       volatile int never = 0;
       for (int t = (issued > NS ? issued - NS : 0); t < issued; ++t)
         mbar_wait(is_k ? b_kfull(t % NS) : b_vfull(t % NS), (t / NS) & 1, 2000000000ull, &never);
-      if (is_k) mbar_wait(b_q, 0, 2000000000ull, &never);
+      if (is_k && nq > 0) mbar_wait(b_q, (nq - 1) & 1, 2000000000ull, &never);
     }
     __syncwarp();
   } else if (warp == 4) {
@@ -284,31 +312,36 @@ __global__ void __launch_bounds__(AttnCfg<D, MODE>::THREADS, 1) attn_kernel(cons
       constexpr uint32_t idesc_qk = idesc_bf16_f32(BM, BN, 0);
       constexpr uint32_t idesc_pv = idesc_bf16_f32(BM, D, 1);
       const uint32_t tS0 = tbase + C::COL_S0, tS1 = tbase + C::COL_S1, tO = tbase + C::COL_O;
-      bool ok = mbar_wait(b_q, 0, a.wait_ns, abort_flag);
+      bool ok = true;
+      int g = 0;                               // this CTA's key tiles so far (all items)
+      // tile j of the current item is global tile g + j: ring slot, S buffer and phases
       auto issue_qk = [&](int j) -> bool {
-        const int s = j % NK;
-        if (!mbar_wait(b_kfull(s), (j / NK) & 1, a.wait_ns, abort_flag)) return false;
+        const int gj = g + j;
+        const int s = gj % NK;
+        if (!mbar_wait(b_kfull(s), (gj / NK) & 1, a.wait_ns, abort_flag)) return false;
         tc_fence_after();
         const uint32_t kb = sK0 + s * C::KV_BYTES;
-        const uint32_t tS = (j & 1) ? tS1 : tS0;
+        const uint32_t tS = (gj & 1) ? tS1 : tS0;
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) {
           const uint32_t off = (kk >> 2) * (128 * 128) + (kk & 3) * 32;
           umma_bf16_ss(tS, sdesc_sw128(sQ + off, 16, 1024), sdesc_sw128(kb + off, 16, 1024),
                        idesc_qk, kk > 0 ? 1u : 0u);
         }
-        umma_commit(b_sfull0 + 8 * (j & 1));
+        umma_commit(b_sfull0 + 8 * (gj & 1));
         umma_commit(b_kempty(s));
+        if (j == T - 1) umma_commit(b_qempty);   // the item's last read of Q
         return true;
       };
       auto issue_pv = [&](int j) -> bool {
-        const int s = j % NV;
-        if (!mbar_wait(b_p, j & 1, a.wait_ns, abort_flag)) return false;
-        if (!mbar_wait(b_vfull(s), (j / NV) & 1, a.wait_ns, abort_flag)) return false;
+        const int gj = g + j;
+        const int s = gj % NV;
+        if (!mbar_wait(b_p, gj & 1, a.wait_ns, abort_flag)) return false;
+        if (!mbar_wait(b_vfull(s), (gj / NV) & 1, a.wait_ns, abort_flag)) return false;
         tc_fence_after();
         const uint32_t vb = sV0 + s * C::KV_BYTES;
-        const uint32_t tP = (j & 1) ? tS1 : tS0;                              // hi part over S
-        const uint32_t tPlo = tbase + C::COL_PLO + (j & 1) * (BN / 2);        // lo part
+        const uint32_t tP = (gj & 1) ? tS1 : tS0;                              // hi part over S
+        const uint32_t tPlo = tbase + C::COL_PLO + (gj & 1) * (BN / 2);        // lo part
 #pragma unroll
         for (int kk = 0; kk < BN / 16; ++kk) {
           const uint64_t bdesc = sdesc_sw128(vb + kk * 16 * 128, BN * 128, 1024);
@@ -325,11 +358,17 @@ __global__ void __launch_bounds__(AttnCfg<D, MODE>::THREADS, 1) attn_kernel(cons
         umma_commit(b_vempty(s));
         return true;
       };
-      if (ok) ok = issue_qk(0);
-      if (ok && T > 1) ok = issue_qk(1);
-      for (int j = 0; j < T && ok; ++j) {
-        ok = issue_pv(j);
-        if (ok && j + 2 < T) ok = issue_qk(j + 2);
+      // the next item's first P.V (accumulate = 0) overwrites O only after its
+      // P is ready, which the softmax warps publish after reading this item's O
+      for (int item = blockIdx.x, it = 0; item < n_items && ok; item += gridDim.x, ++it) {
+        ok = mbar_wait(b_q, it & 1, a.wait_ns, abort_flag);
+        if (ok) ok = issue_qk(0);
+        if (ok && T > 1) ok = issue_qk(1);
+        for (int j = 0; j < T && ok; ++j) {
+          ok = issue_pv(j);
+          if (ok && j + 2 < T) ok = issue_qk(j + 2);
+        }
+        g += T;
       }
       if (!ok && !*abort_flag) {
         *abort_flag = 1;
@@ -343,7 +382,14 @@ __global__ void __launch_bounds__(AttnCfg<D, MODE>::THREADS, 1) attn_kernel(cons
   } else {
     // ------------------------------------------------------------------ softmax
     const int r = tid;                           // query row == TMEM lane
-    const int my_q = q_token(r);
+    const uint32_t lane_addr = static_cast<uint32_t>(warp * 32) << 16;
+    const float sl2 = a.scale_log2;
+    bool ok = true;
+    int g = 0;                                   // this CTA's key tiles so far (all items)
+    for (int item = blockIdx.x; item < n_items && ok; item += gridDim.x, g += T) {
+    const Item w = item_at(item);
+    const size_t head = w.head;
+    const int my_q = q_token(w, r);
     if (MODE == kModeStep || MODE == kModePlanResid) {
       // warm L2 with the row the epilogue will read
       const float *ep = MODE == kModeStep ? a.residual : a.O32_in;
@@ -353,15 +399,13 @@ __global__ void __launch_bounds__(AttnCfg<D, MODE>::THREADS, 1) attn_kernel(cons
           asm volatile("prefetch.global.L2 [%0];" ::"l"(ep + (head + my_q) * D + c * 32));
       }
     }
-    const uint32_t lane_addr = static_cast<uint32_t>(warp * 32) << 16;
-    const float sl2 = a.scale_log2;
     float m_run = -INFINITY, l_run = 0.f;
-    bool ok = true;
     for (int j = 0; j < T; ++j) {
-      if (!mbar_wait(b_sfull0 + 8 * (j & 1), (j >> 1) & 1, a.wait_ns, abort_flag)) { ok = false; break; }
+      const int gj = g + j;
+      if (!mbar_wait(b_sfull0 + 8 * (gj & 1), (gj >> 1) & 1, a.wait_ns, abort_flag)) { ok = false; break; }
       tc_fence_after();
-      const uint32_t tS = tbase + lane_addr + ((j & 1) ? C::COL_S1 : C::COL_S0);
-      const uint32_t tPlo = tbase + lane_addr + C::COL_PLO + (j & 1) * (BN / 2);
+      const uint32_t tS = tbase + lane_addr + ((gj & 1) ? C::COL_S1 : C::COL_S0);
+      const uint32_t tPlo = tbase + lane_addr + C::COL_PLO + (gj & 1) * (BN / 2);
       const int nvalid = nkeys - j * BN;   // >= 1; only the last tile can be partial
       float alpha = 1.f;
       bool resc = false;
@@ -483,7 +527,7 @@ __global__ void __launch_bounds__(AttnCfg<D, MODE>::THREADS, 1) attn_kernel(cons
       tmem_wait_st();
       // O is stable once the previous P.V has completed
       if (j > 0) {
-        if (!mbar_wait(b_pv, (j - 1) & 1, a.wait_ns, abort_flag)) { ok = false; break; }
+        if (!mbar_wait(b_pv, (gj - 1) & 1, a.wait_ns, abort_flag)) { ok = false; break; }
         tc_fence_after();
         if (__any_sync(0xffffffffu, resc)) {
           const uint32_t tO = tbase + lane_addr + C::COL_O;
@@ -503,14 +547,9 @@ __global__ void __launch_bounds__(AttnCfg<D, MODE>::THREADS, 1) attn_kernel(cons
       mbar_arrive(b_p);
     }
     if (ok && T > 0) {
-      if (!mbar_wait(b_pv, (T - 1) & 1, a.wait_ns, abort_flag)) ok = false;
+      if (!mbar_wait(b_pv, (g + T - 1) & 1, a.wait_ns, abort_flag)) ok = false;
     }
-    if (!ok) {
-      if (!*abort_flag) {
-        *abort_flag = 1;
-        record_status(a.status, kStatusTimeout);
-      }
-    } else {
+    if (ok) {
       // ------------------------------------------------------------------ epilogue
       tc_fence_after();
       const int q = my_q;
@@ -569,6 +608,11 @@ __global__ void __launch_bounds__(AttnCfg<D, MODE>::THREADS, 1) attn_kernel(cons
         a.row_m[head + q] = m_run;
         a.row_l[head + q] = l_run;
       }
+    }
+    }   // items
+    if (!ok && !*abort_flag) {
+      *abort_flag = 1;
+      record_status(a.status, kStatusTimeout);
     }
   }
 

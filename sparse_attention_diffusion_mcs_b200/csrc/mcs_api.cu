@@ -94,6 +94,14 @@ bool map_tile(CUtensorMap *m, const void *base, int D, int N, int BH) {
             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// SMs of the current device
+cudaError_t sm_count(int *n) {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  return cudaDeviceGetAttribute(n, cudaDevAttrMultiProcessorCount, dev);
+}
+
 template <typename F>
 cudaError_t set_smem(F *fn, int bytes) {
   return cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
@@ -118,7 +126,20 @@ cudaError_t launch_attn(AttnArgs &a, const QKV &t, int grid_x, int BH, cudaStrea
   if (!ok) return cudaErrorInvalidValue;
   cudaError_t e = set_smem(attn_kernel<D, MODE>, C::SMEM);
   if (e != cudaSuccess) return e;
-  attn_kernel<D, MODE><<<dim3(grid_x, BH), C::THREADS, C::SMEM, s>>>(a);
+  // Sparse modes run persistent, one CTA per SM (the kernel takes all of an
+  // SM's shared memory and TMEM) looping over (head, group) items, so each
+  // item's gathers and first Q.K^T overlap the previous item's epilogue.
+  // Dense modes (long items, small epilogues) launch one CTA per item.
+  a.BH = BH;
+  const long items = static_cast<long>(grid_x) * BH;
+  long grid = items;
+  if (C::kSparse) {
+    int sms = 0;
+    if ((e = sm_count(&sms)) != cudaSuccess) return e;
+    if (grid > sms) grid = sms;
+  }
+  if (grid == 0) return cudaSuccess;
+  attn_kernel<D, MODE><<<static_cast<unsigned>(grid), C::THREADS, C::SMEM, s>>>(a);
   return cudaGetLastError();
 }
 
