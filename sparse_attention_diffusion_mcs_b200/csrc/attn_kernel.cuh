@@ -92,6 +92,11 @@ struct AttnCfg {
   // dense modes keep the whole score row in registers (one TMEM pass); the
   // 384-thread sparse CTA caps registers at 168, so it reads S twice
   static constexpr bool kOnePass = !kSparse;
+  // The softmax reference max trails the true row max by up to 2^kRaise (log2
+  // units) before O and l are rescaled.  bf16 P and fp32 O, l keep their
+  // relative precision at any scale, so the only bound is range: P <= 2^32
+  // and l <= N 2^32 stay far from fp32 overflow for |V| < 2^64.
+  static constexpr float kRaise = 32.f;
   static constexpr uint32_t TMEM_COLS = 512;
   static constexpr uint32_t COL_S0 = 0, COL_S1 = 128, COL_O = 256, COL_PLO = 384;
 };
@@ -151,22 +156,26 @@ __global__ void __launch_bounds__(AttnCfg<D, MODE>::THREADS, 1) attn_kernel(cons
     return w;
   };
 
-  // query row r of an item -> token index, or -1 when the row is padding
-  auto q_token = [&](const Item &w, int r) -> int {
+  // query row r of an item -> token index, or -1 when the row is padding.
+  // q_raw only loads (so the load can be issued long before its use);
+  // q_check validates what it loaded.
+  auto q_raw = [&](const Item &w, int r) -> int {
     if (C::kSparse) {
       const int gr = w.tile * a.G + r;
-      if (r >= a.G || gr >= N) return -1;
-      const int q = a.perm[w.head + gr];
-      if (static_cast<unsigned>(q) >= static_cast<unsigned>(N)) {   // corrupt metadata: never gather out of range
-        record_status(a.status, kStatusBadMeta);
-        return -1;
-      }
-      return q;
+      return (r >= a.G || gr >= N) ? -1 : a.perm[w.head + gr];
     } else {
       const int q = w.tile * BM + r;
       return q < N ? q : -1;
     }
   };
+  auto q_check = [&](int q) -> int {
+    if (C::kSparse && q != -1 && static_cast<unsigned>(q) >= static_cast<unsigned>(N)) {
+      record_status(a.status, kStatusBadMeta);   // corrupt metadata: never gather out of range
+      return -1;
+    }
+    return q;
+  };
+  auto q_token = [&](const Item &w, int r) -> int { return q_check(q_raw(w, r)); };
 
   if (tid == 0) {
     mbar_init(b_q, 1);
@@ -386,23 +395,34 @@ __global__ void __launch_bounds__(AttnCfg<D, MODE>::THREADS, 1) attn_kernel(cons
     const float sl2 = a.scale_log2;
     bool ok = true;
     int g = 0;                                   // this CTA's key tiles so far (all items)
+    // the epilogue's second input (residual, or the dense output), read per row
+    constexpr bool kEpiIn = (MODE == kModeStep || MODE == kModePlanResid);
+    const float *ep_in = MODE == kModeStep ? a.residual : a.O32_in;
+    auto warm_row = [&](size_t head_, int q) {   // pull the row into L2 well before the epilogue
+      if (kEpiIn && q >= 0) {
+#pragma unroll
+        for (int c = 0; c < D / 32; ++c)
+          asm volatile("prefetch.global.L2 [%0];" ::"l"(ep_in + (head_ + q) * D + c * 32));
+      }
+    };
+    int my_q = -1;
+    if (static_cast<int>(blockIdx.x) < n_items) {
+      const Item w0 = item_at(blockIdx.x);
+      my_q = q_token(w0, r);
+      warm_row(w0.head, my_q);
+    }
     for (int item = blockIdx.x; item < n_items && ok; item += gridDim.x, g += T) {
     const Item w = item_at(item);
     const size_t head = w.head;
-    const int my_q = q_token(w, r);
-    if (MODE == kModeStep || MODE == kModePlanResid) {
-      // warm L2 with the row the epilogue will read
-      const float *ep = MODE == kModeStep ? a.residual : a.O32_in;
-      if (my_q >= 0) {
-#pragma unroll
-        for (int c = 0; c < D / 32; ++c)
-          asm volatile("prefetch.global.L2 [%0];" ::"l"(ep + (head + my_q) * D + c * 32));
-      }
-    }
+    // the next item's token, loaded now and used after this item's tiles
+    const int nitem = item + static_cast<int>(gridDim.x);
+    const bool has_next = nitem < n_items;
+    const Item wn = item_at(has_next ? nitem : item);
+    const int next_raw = has_next ? q_raw(wn, r) : -1;
     float m_run = -INFINITY, l_run = 0.f;
     for (int j = 0; j < T; ++j) {
       const int gj = g + j;
-      if (!mbar_wait(b_sfull0 + 8 * (gj & 1), (gj >> 1) & 1, a.wait_ns, abort_flag)) { ok = false; break; }
+      if (!mbar_wait_warp(b_sfull0 + 8 * (gj & 1), (gj >> 1) & 1, a.wait_ns, abort_flag)) { ok = false; break; }
       tc_fence_after();
       const uint32_t tS = tbase + lane_addr + ((gj & 1) ? C::COL_S1 : C::COL_S0);
       const uint32_t tPlo = tbase + lane_addr + C::COL_PLO + (gj & 1) * (BN / 2);
@@ -415,7 +435,7 @@ __global__ void __launch_bounds__(AttnCfg<D, MODE>::THREADS, 1) attn_kernel(cons
         mx *= sl2;
         if (j == 0) {
           m_run = mx;
-        } else if (mx > m_run + 8.f) {      // lazy rescale: only when the max grew by > 2^8
+        } else if (mx > m_run + C::kRaise) {   // lazy rescale: only when the max grew by > 2^kRaise
           alpha = ex2_approx(m_run - mx);
           m_run = mx;
           resc = true;
@@ -527,7 +547,7 @@ __global__ void __launch_bounds__(AttnCfg<D, MODE>::THREADS, 1) attn_kernel(cons
       tmem_wait_st();
       // O is stable once the previous P.V has completed
       if (j > 0) {
-        if (!mbar_wait(b_pv, (gj - 1) & 1, a.wait_ns, abort_flag)) { ok = false; break; }
+        if (!mbar_wait_warp(b_pv, (gj - 1) & 1, a.wait_ns, abort_flag)) { ok = false; break; }
         tc_fence_after();
         if (__any_sync(0xffffffffu, resc)) {
           const uint32_t tO = tbase + lane_addr + C::COL_O;
@@ -546,44 +566,57 @@ __global__ void __launch_bounds__(AttnCfg<D, MODE>::THREADS, 1) attn_kernel(cons
       tc_fence_before();
       mbar_arrive(b_p);
     }
+    const int q = my_q;
+    const size_t row = (head + (q >= 0 ? q : 0)) * D;
+    // the epilogue input of the first chunk is in flight while the last P.V runs
+    float4 ein[8];
+    if (kEpiIn && q >= 0) {
+      const float4 *src = reinterpret_cast<const float4 *>(ep_in + row);
+#pragma unroll
+      for (int u = 0; u < 8; ++u) ein[u] = __ldg(src + u);
+    }
+    if (ok) {
+      my_q = has_next ? q_check(next_raw) : -1;
+      warm_row(wn.head, my_q);
+    }
     if (ok && T > 0) {
-      if (!mbar_wait(b_pv, (g + T - 1) & 1, a.wait_ns, abort_flag)) ok = false;
+      if (!mbar_wait_warp(b_pv, (g + T - 1) & 1, a.wait_ns, abort_flag)) ok = false;
     }
     if (ok) {
       // ------------------------------------------------------------------ epilogue
       tc_fence_after();
-      const int q = my_q;
       const float inv_l = 1.f / l_run;
       const uint32_t tO = tbase + lane_addr + C::COL_O;
-      const size_t row = (head + (q >= 0 ? q : 0)) * D;
 #pragma unroll
       for (int cc = 0; cc < D / 32; ++cc) {
+        // next chunk's input in flight while this chunk is finished
+        float4 enx[8];
+        if (kEpiIn && q >= 0 && cc + 1 < D / 32) {
+          const float4 *src = reinterpret_cast<const float4 *>(ep_in + row + (cc + 1) * 32);
+#pragma unroll
+          for (int u = 0; u < 8; ++u) enx[u] = __ldg(src + u);
+        }
         float o[32];
         tmem_ld32(tO + cc * 32, o);
         tmem_wait_ld();
-        if (q < 0) continue;
+        if (q >= 0) {
 #pragma unroll
         for (int i = 0; i < 32; ++i) o[i] *= inv_l;
         if (MODE == kModeStep) {
-          const float4 *rp = reinterpret_cast<const float4 *>(a.residual + row + cc * 32);
 #pragma unroll
           for (int u = 0; u < 8; ++u) {
-            const float4 rv = __ldg(rp + u);
-            o[4 * u + 0] += rv.x;
-            o[4 * u + 1] += rv.y;
-            o[4 * u + 2] += rv.z;
-            o[4 * u + 3] += rv.w;
+            o[4 * u + 0] += ein[u].x;
+            o[4 * u + 1] += ein[u].y;
+            o[4 * u + 2] += ein[u].z;
+            o[4 * u + 3] += ein[u].w;
           }
         }
         if (MODE == kModePlanResid) {
-          const float4 *dp = reinterpret_cast<const float4 *>(a.O32_in + row + cc * 32);
           float4 *rp = reinterpret_cast<float4 *>(a.R_out + row + cc * 32);
 #pragma unroll
-          for (int u = 0; u < 8; ++u) {
-            const float4 dv = __ldg(dp + u);
-            rp[u] = make_float4(dv.x - o[4 * u], dv.y - o[4 * u + 1], dv.z - o[4 * u + 2],
-                                dv.w - o[4 * u + 3]);
-          }
+          for (int u = 0; u < 8; ++u)
+            rp[u] = make_float4(ein[u].x - o[4 * u], ein[u].y - o[4 * u + 1], ein[u].z - o[4 * u + 2],
+                                ein[u].w - o[4 * u + 3]);
         }
         if (MODE == kModePlanDense) {
           float4 *op = reinterpret_cast<float4 *>(a.O32 + row + cc * 32);
@@ -602,6 +635,11 @@ __global__ void __launch_bounds__(AttnCfg<D, MODE>::THREADS, 1) attn_kernel(cons
             w.w = pack_bf16x2(o[8 * u + 6], o[8 * u + 7]);
             op[u] = w;
           }
+        }
+        }   // q >= 0
+        if (kEpiIn && cc + 1 < D / 32) {
+#pragma unroll
+          for (int u = 0; u < 8; ++u) ein[u] = enx[u];
         }
       }
       if (MODE == kModePlanDense && q >= 0) {

@@ -199,7 +199,7 @@ __global__ void __launch_bounds__(224, 1) colsum_kernel(const __grid_constant__ 
     bool ok = true;
     for (int j = 0; j < T; ++j) {
       const int b = j & 1;
-      if (!mbar_wait(b_sfull0 + 8 * b, (j >> 1) & 1, a.wait_ns, abort_flag)) { ok = false; break; }
+      if (!mbar_wait_warp(b_sfull0 + 8 * b, (j >> 1) & 1, a.wait_ns, abort_flag)) { ok = false; break; }
       tc_fence_after();
       float acc0 = 0.f, acc1 = 0.f, acc2 = 0.f, acc3 = 0.f;
 #pragma unroll

@@ -15,10 +15,11 @@ from .dit_inputs import (
     drift_layer,
     random_metadata_head,
     random_qkv,
+    rising_qkv,
 )
 
 __all__ = [
     "CONFIGS", "Workload", "workload", "sweep_points",
     "bf16_round", "head_tensors", "layer_tensors", "drift_head", "drift_layer",
-    "random_metadata_head", "random_qkv",
+    "random_metadata_head", "random_qkv", "rising_qkv",
 ]

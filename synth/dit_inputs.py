@@ -186,3 +186,16 @@ def random_qkv(B: int, H: int, N: int, d: int, seed: int = 0, q_std: float = 1.0
     k = rng.standard_normal((B, H, N, d), dtype=np.float32)
     v = rng.standard_normal((B, H, N, d), dtype=np.float32)
     return bf16_round(q), bf16_round(k), bf16_round(v)
+
+
+def rising_qkv(B: int, H: int, N: int, d: int, seed: int = 0, q_std: float = 2.0, growth: float = 8.0):
+    """Gaussian Q, V and keys whose scale grows with the key index,
+    K_j ~ (1 + growth (j/N)^2) N(0, 1), so attention scores rise steeply along
+    any ascending key list: row maxima jump by many powers of two between,
+    and inside, 128-key tiles.  bf16 bit patterns [B, H, N, d]."""
+    rng = np.random.default_rng(np.random.SeedSequence(entropy=seed, spawn_key=(98, B, H, N, d)))
+    q = (q_std * rng.standard_normal((B, H, N, d))).astype(np.float32)
+    scale = (1.0 + growth * (np.arange(N) / N) ** 2).astype(np.float32)
+    k = rng.standard_normal((B, H, N, d), dtype=np.float32) * scale[:, None]
+    v = rng.standard_normal((B, H, N, d), dtype=np.float32)
+    return bf16_round(q), bf16_round(k), bf16_round(v)

@@ -17,6 +17,10 @@ from tests.gpu_util import (assert_out_close, assert_residual_close, dev_bf16, h
 
 pytestmark = pytest.mark.gpu
 
+# how far (log2 units) the sparse softmax lets a row's reference max trail the
+# running max before it rescales what it has written
+RAISE_LOG2 = 32
+
 
 def _shape_workload(N, d, G, k):
     return synth.CONFIGS[1].with_(grid=(1, 1, N), d=d, G=G, k=k)
@@ -38,6 +42,18 @@ def test_dense_random_shapes(B, H, N, d, qs):
         for h in range(H):
             ref = orc.dense_attention(Q[b, h], K[b, h], V[b, h], 1 / np.sqrt(d))
             assert_out_close(out[b, h], ref, f"dense b{b} h{h}")
+
+
+@pytest.mark.parametrize("N,d", [(1000, 128), (777, 64)])
+def test_dense_rising_scores(N, d):
+    """Keys whose scale grows with the index: row maxima jump by more than
+    2^RAISE_LOG2 between key tiles, so O and l are rescaled mid-row."""
+    Q, K, V = synth.rising_qkv(1, 1, N, d, seed=6, growth=40.0)
+    out = host(mcs.dense(dev_bf16(Q), dev_bf16(K), dev_bf16(V)))
+    torch.cuda.synchronize()
+    assert mcs.last_device_status() == 0
+    ref = orc.dense_attention(Q[0, 0], K[0, 0], V[0, 0], 1 / np.sqrt(d))
+    assert_out_close(out[0, 0], ref, f"dense rising N{N} d{d}")
 
 
 def test_dense_tiny_workload():
@@ -67,6 +83,35 @@ def test_sparse_step_random_metadata(N, d, G, k):
     assert mcs.last_device_status() == 0
     ref = orc.reused_step_head(Q[0, 0], K[0, 0], V[0, 0], w.scale, perm, kv, res, G)
     assert_out_close(out[0, 0], ref, f"step N{N} d{d} G{G} k{k}")
+
+
+@pytest.mark.parametrize("N,d,G,k", [(1000, 128, 128, 300), (1000, 64, 64, 600), (700, 128, 128, 700)])
+def test_sparse_step_rising_scores(N, d, G, k):
+    """Scores that rise steeply along each group's ascending key list: the
+    running max is raised by more than 2^RAISE_LOG2 between tiles and inside
+    them, so the P chunks a tile has already written get rescaled in place."""
+    w = _shape_workload(N, d, G, k)
+    Q, K, V = synth.rising_qkv(1, 1, N, d, seed=5, growth=40.0)
+    perm, kv, res = synth.random_metadata_head(w, 0)
+    # the inputs really do take the rescaling path: for the first group, some
+    # 32-key chunk that is not the first of its 128-key tile has a max above
+    # every earlier chunk's by more than 2^RAISE_LOG2
+    s = orc.scores(Q[0, 0][perm[:G]], K[0, 0], w.scale) * np.log2(np.e)
+    row = s[:, kv[0]]
+    nch = -(-row.shape[1] // 32)
+    padded = np.full((G, nch * 32), -np.inf)
+    padded[:, :row.shape[1]] = row
+    chunk_max = padded.reshape(G, nch, 32).max(axis=2)
+    raised = chunk_max[:, 1:] > np.maximum.accumulate(chunk_max, axis=1)[:, :-1] + RAISE_LOG2
+    assert raised[:, np.arange(1, nch) % 4 != 0].any()
+    meta = mcs.Meta.from_tensors(torch.from_numpy(perm)[None, None].cuda(),
+                                 torch.from_numpy(kv)[None, None].cuda(),
+                                 torch.from_numpy(res)[None, None].cuda(), G)
+    out = host(mcs.sparse_step(dev_bf16(Q), dev_bf16(K), dev_bf16(V), meta))
+    torch.cuda.synchronize()
+    assert mcs.last_device_status() == 0
+    ref = orc.reused_step_head(Q[0, 0], K[0, 0], V[0, 0], w.scale, perm, kv, res, G)
+    assert_out_close(out[0, 0], ref, f"rising step N{N} d{d} G{G} k{k}")
 
 
 def test_sparse_step_on_oracle_plan_with_drift():
