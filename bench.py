@@ -34,7 +34,7 @@ import numpy as np  # noqa: E402
 
 import synth  # noqa: E402
 
-KERNELS_PER_STEP = 12   # grouping 6, stats 1, scores 1, top-k 1, residual 1, step 1, dense 1
+KERNELS_PER_STEP = 13   # grouping 7, stats 1, scores 1, top-k 1, residual 1, step 1, dense 1
 
 
 def parse_args():
@@ -46,6 +46,8 @@ def parse_args():
     ap.add_argument("--config", type=int, default=3, help="workload id (default: 32K-token video layer)")
     ap.add_argument("--k", type=int, default=None, help="override keys per group")
     ap.add_argument("--G", type=int, default=None, help="override group size")
+    ap.add_argument("--heads", type=int, default=None,
+                    help="run only the first H heads of the layer (smaller profiling captures)")
     ap.add_argument("--cpu-seconds", type=float, default=12.0, help="CPU baseline budget")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
@@ -172,7 +174,8 @@ def measured_traffic():
     kernel sources still hash to what was profiled (else no entry)."""
     import hashlib
     csrc = os.path.join(ROOT, "sparse_attention_diffusion_mcs_b200", "csrc")
-    files = {"attn": ("mcs_common.cuh", "attn_kernel.cuh"), "colsum": ("mcs_common.cuh", "colsum_kernel.cuh")}
+    files = {"attn": ("mcs_common.cuh", "attn_kernel.cuh"), "colsum": ("mcs_common.cuh", "colsum_kernel.cuh"),
+             "topk": ("mcs_common.cuh", "topk_kernel.cuh")}
     hashes = {}
     for key, fs in files.items():
         m = hashlib.sha256()
@@ -186,7 +189,7 @@ def measured_traffic():
             if line.startswith("#") or not line.strip():
                 continue
             stage, kernel, hsh, rd, wr = line.split()
-            fam = "colsum" if kernel.startswith("colsum") else "attn"
+            fam = kernel.split("_")[0] if kernel.split("_")[0] in files else "attn"
             if hashes.get(fam) == hsh:
                 out[stage] = int(rd) + int(wr)
     except OSError:
@@ -289,6 +292,8 @@ def main():
     rank = int(os.environ.get("RANK", "0"))
     local = int(os.environ.get("LOCAL_RANK", "0"))
     w = synth.workload(args.config, k=args.k, G=args.G)
+    if args.heads:
+        w = w.with_(H=min(args.heads, w.H))
     # host inputs first (process pool before any CUDA work)
     s1, s2 = make_inputs(w, rank)
 
