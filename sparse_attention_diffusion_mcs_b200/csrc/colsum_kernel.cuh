@@ -13,6 +13,11 @@
 // reduction.  CTA = one (head, group); loops over all N/128 key tiles.
 //   warps 0-3 reduce, warp 4 issues UMMA, warp 5 loads the group's queries
 //   (TMA tile::gather4) and streams K tiles (TMA 3D tiles), warp 6 idles.
+// Two CTAs share an SM (256 TMEM columns and < 114 KB of shared memory each),
+// so each SM sub-partition has two reducing warps to hide TMEM and MUFU
+// latency.  The reducers keep the next 32-column chunk's TMEM load in flight,
+// and compute a quarter of the exponentials on the FMA pipe (ex2_fma) so that
+// the MUFU pipe, which bounds this kernel, carries three quarters.
 #pragma once
 
 #include "mcs_common.cuh"
@@ -32,10 +37,36 @@ struct alignas(64) ColsumArgs {
   uint64_t wait_ns;
 };
 
+// 2^x on the FMA and ALU pipes, for x <= 1/2 (here x = s*scale*log2e - c_i
+// <= 0 up to rounding): x = n + f with n = rint(x) by the 1.5*2^23 shift,
+// p(f) ~ 2^f on [-1/2, 1/2] by a degree-5 minimax polynomial (max relative
+// error 7.5e-8; coefficients from fit_exp2_poly.py), n added to p's exponent
+// bits.  Results below 2^-126 are 0, as the MUFU ex2.approx.ftz gives.
+__device__ __forceinline__ float ex2_fma(float x) {
+  const float xc = fmaxf(x, -126.f);
+  const float y = xc + 12582912.f;            // 1.5 * 2^23: rounds xc to an integer
+  const float f = xc - (y - 12582912.f);      // in [-1/2, 1/2]
+  float p = fmaf(1.327647245e-03f, f, 9.675540961e-03f);
+  p = fmaf(p, f, 5.550713092e-02f);
+  p = fmaf(p, f, 2.402212024e-01f);
+  p = fmaf(p, f, 6.931469440e-01f);
+  p = fmaf(p, f, 1.000000119e+00f);
+  // bits(y) = bits(1.5 * 2^23) + n, and bits(1.5 * 2^23) << 23 vanishes mod 2^32
+  const uint32_t r = __float_as_uint(p) + (__float_as_uint(y) << 23);
+  return x >= -126.f ? __uint_as_float(r) : 0.f;
+}
+
+// which of every 8 consecutive exponentials run on the FMA pipe (bit i: column
+// i mod 8); the rest use the MUFU ex2
+#ifndef MCS_COLSUM_FMA_EXP_MASK
+#define MCS_COLSUM_FMA_EXP_MASK 0x88u
+#endif
+constexpr unsigned kFmaExpMask = MCS_COLSUM_FMA_EXP_MASK;
+
 template <int D>
 struct ColsumCfg {
   static constexpr int BM = 128, BN = 128;   // BM keys per tile (MMA M), BN queries (MMA N)
-  static constexpr int NST = D == 64 ? 8 : 4;
+  static constexpr int NST = D == 64 ? 4 : 2;   // K ring depth (two CTAs per SM)
   static constexpr int Q_BYTES = BN * D * 2;
   static constexpr int K_BYTES = BM * D * 2;
   static constexpr int OFF_Q = 0;
@@ -49,7 +80,7 @@ struct ColsumCfg {
 };
 
 template <int D>
-__global__ void __launch_bounds__(224, 1) colsum_kernel(const __grid_constant__ ColsumArgs a) {
+__global__ void __launch_bounds__(224, 2) colsum_kernel(const __grid_constant__ ColsumArgs a) {
   using C = ColsumCfg<D>;
   constexpr int BM = C::BM, NST = C::NST;
   constexpr int NDB = D / 64;
@@ -202,19 +233,28 @@ __global__ void __launch_bounds__(224, 1) colsum_kernel(const __grid_constant__ 
       if (!mbar_wait_warp(b_sfull0 + 8 * b, (j >> 1) & 1, a.wait_ns, abort_flag)) { ok = false; break; }
       tc_fence_after();
       float acc0 = 0.f, acc1 = 0.f, acc2 = 0.f, acc3 = 0.f;
+      float v[2][32];
+      tmem_ld32(tbase + lane_addr + b * 128, v[0]);
 #pragma unroll
       for (int cc = 0; cc < 4; ++cc) {
-        float v[32];
-        tmem_ld32(tbase + lane_addr + b * 128 + cc * 32, v);
+        float (&cur)[32] = v[cc & 1];
         tmem_wait_ld();
+        if (cc + 1 < 4) tmem_ld32(tbase + lane_addr + b * 128 + (cc + 1) * 32, v[(cc + 1) & 1]);
         const float4 *c4 = reinterpret_cast<const float4 *>(stat + cc * 32);
 #pragma unroll
         for (int i = 0; i < 32; i += 4) {
           const float4 c = c4[i / 4];     // same address in every lane: one broadcast read
-          acc0 += ex2_approx(fmaf(v[i], sl2, -c.x));
-          acc1 += ex2_approx(fmaf(v[i + 1], sl2, -c.y));
-          acc2 += ex2_approx(fmaf(v[i + 2], sl2, -c.z));
-          acc3 += ex2_approx(fmaf(v[i + 3], sl2, -c.w));
+          const float cv[4] = {c.x, c.y, c.z, c.w};
+          float e[4];
+#pragma unroll
+          for (int u = 0; u < 4; ++u) {
+            const float x = fmaf(cur[i + u], sl2, -cv[u]);
+            e[u] = ((kFmaExpMask >> ((i + u) & 7)) & 1u) ? ex2_fma(x) : ex2_approx(x);
+          }
+          acc0 += e[0];
+          acc1 += e[1];
+          acc2 += e[2];
+          acc3 += e[3];
         }
       }
       acc0 += acc1;
