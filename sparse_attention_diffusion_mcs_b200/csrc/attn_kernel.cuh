@@ -84,7 +84,7 @@ struct AttnCfg {
   static constexpr int OFF_K = OFF_Q + Q_BYTES;
   static constexpr int OFF_V = OFF_K + NK * KV_BYTES;
   static constexpr int OFF_BAR = OFF_V + NV * KV_BYTES;
-  static constexpr int N_BAR = 1 + 2 * NK + 2 * NV + 2 + 4;   // q, k/v full/empty, s_full[2], p, pv, drain, q_empty
+  static constexpr int N_BAR = 1 + 2 * NK + 2 * NV + 8;   // q, k/v full/empty, s_full[2], p[2], pv[2], drain, q_empty
   static constexpr int OFF_MISC = OFF_BAR + 8 * N_BAR;
   static constexpr int SMEM = OFF_MISC + 16 + 1024;          // + slack to align the base to 1 KB
   static constexpr int THREADS = kSparse ? 384 : 224;
@@ -122,10 +122,17 @@ __global__ void __launch_bounds__(AttnCfg<D, MODE>::THREADS, 1) attn_kernel(cons
   auto b_vfull = [&](int s) { return bar0 + 8 * (1 + 2 * NK + s); };
   auto b_vempty = [&](int s) { return bar0 + 8 * (1 + 2 * NK + NV + s); };
   const uint32_t b_sfull0 = bar0 + 8 * (1 + 2 * NK + 2 * NV);
-  const uint32_t b_p = b_sfull0 + 16;
-  const uint32_t b_pv = b_sfull0 + 24;
-  const uint32_t b_drain = b_sfull0 + 32;
-  const uint32_t b_qempty = b_sfull0 + 40;
+  // "P ready" and "P.V done" alternate between two barriers each by tile
+  // parity.  The softmax warps wait on P.V only now and then (a rescale, the
+  // epilogue) and may publish P two tiles in a row before the MMA thread has
+  // looked, so up to two completions of each kind can be outstanding; with
+  // one barrier per parity each has at most one, and a parity wait cannot
+  // alias (P of tile j+2 needs S of tile j+2, whose Q.K^T is issued after
+  // the P.V of tile j, which needs P of tile j)
+  auto b_p = [&](int gj) { return b_sfull0 + 16 + 8 * (gj & 1); };
+  auto b_pv = [&](int gj) { return b_sfull0 + 32 + 8 * (gj & 1); };
+  const uint32_t b_drain = b_sfull0 + 48;
+  const uint32_t b_qempty = b_sfull0 + 56;
   uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem + C::OFF_MISC);
   volatile int *abort_flag = reinterpret_cast<volatile int *>(smem + C::OFF_MISC + 4);
 
@@ -189,8 +196,10 @@ __global__ void __launch_bounds__(AttnCfg<D, MODE>::THREADS, 1) attn_kernel(cons
     }
     mbar_init(b_sfull0, 1);
     mbar_init(b_sfull0 + 8, 1);
-    mbar_init(b_p, 128);
-    mbar_init(b_pv, 1);
+    mbar_init(b_p(0), 128);
+    mbar_init(b_p(1), 128);
+    mbar_init(b_pv(0), 1);
+    mbar_init(b_pv(1), 1);
     mbar_init(b_drain, 1);
     mbar_init(b_qempty, 1);
     *abort_flag = 0;
@@ -345,7 +354,7 @@ __global__ void __launch_bounds__(AttnCfg<D, MODE>::THREADS, 1) attn_kernel(cons
       auto issue_pv = [&](int j) -> bool {
         const int gj = g + j;
         const int s = gj % NV;
-        if (!mbar_wait(b_p, gj & 1, a.wait_ns, abort_flag)) return false;
+        if (!mbar_wait(b_p(gj), (gj >> 1) & 1, a.wait_ns, abort_flag)) return false;
         if (!mbar_wait(b_vfull(s), (gj / NV) & 1, a.wait_ns, abort_flag)) return false;
         tc_fence_after();
         const uint32_t vb = sV0 + s * C::KV_BYTES;
@@ -363,7 +372,7 @@ __global__ void __launch_bounds__(AttnCfg<D, MODE>::THREADS, 1) attn_kernel(cons
             umma_bf16_ts(tO, tPlo + kk * 8, bdesc, idesc_pv, 1u);
           }
         }
-        umma_commit(b_pv);
+        umma_commit(b_pv(gj));
         umma_commit(b_vempty(s));
         return true;
       };
@@ -507,9 +516,11 @@ __global__ void __launch_bounds__(AttnCfg<D, MODE>::THREADS, 1) attn_kernel(cons
 #pragma unroll
           for (int hh = 0; hh < BN / 64; ++hh) store_p(sv + hh * 64, 32, tS + hh * 32, tPlo + hh * 32);
         } else {
-          // pass 1: row max of this tile
+          // pass 1: row max of this tile.  Both passes stay rolled: unrolled
+          // over the four chunks they need more than the 168 registers a
+          // thread of this CTA has, and the spills cost more than the loop.
           float m0 = -INFINITY, m1 = -INFINITY;
-#pragma unroll
+#pragma unroll 1
           for (int cc = 0; cc < BN / 32; ++cc) {
             float v[32];
             tmem_ld32(tS + cc * 32, v);
@@ -523,7 +534,7 @@ __global__ void __launch_bounds__(AttnCfg<D, MODE>::THREADS, 1) attn_kernel(cons
           update_max(fmaxf(m0, m1));
           // pass 2: P = 2^(s*scale*log2e - m); chunk cc lands on columns [16cc, 16cc+16),
           // all of them already read
-#pragma unroll
+#pragma unroll 1
           for (int cc = 0; cc < BN / 32; ++cc) {
             float v[32];
             tmem_ld32(tS + cc * 32, v);
@@ -545,26 +556,27 @@ __global__ void __launch_bounds__(AttnCfg<D, MODE>::THREADS, 1) attn_kernel(cons
       else tile_body(std::true_type{});
       l_run = fmaf(l_run, alpha, rs0 + rs1);
       tmem_wait_st();
-      // O is stable once the previous P.V has completed
-      if (j > 0) {
-        if (!mbar_wait_warp(b_pv, (gj - 1) & 1, a.wait_ns, abort_flag)) { ok = false; break; }
+      // Only a warp with a row whose max moved by more than 2^kRaise waits for
+      // the previous P.V (O then holds exactly the tiles before this one) and
+      // rescales O; otherwise P is published at once and the P.V of this
+      // tile queues behind the previous one in the tensor pipe.
+      if (j > 0 && __any_sync(0xffffffffu, resc)) {
+        if (!mbar_wait_warp(b_pv(gj - 1), ((gj - 1) >> 1) & 1, a.wait_ns, abort_flag)) { ok = false; break; }
         tc_fence_after();
-        if (__any_sync(0xffffffffu, resc)) {
-          const uint32_t tO = tbase + lane_addr + C::COL_O;
+        const uint32_t tO = tbase + lane_addr + C::COL_O;
 #pragma unroll
-          for (int cc = 0; cc < D / 32; ++cc) {
-            float o[32];
-            tmem_ld32(tO + cc * 32, o);
-            tmem_wait_ld();
+        for (int cc = 0; cc < D / 32; ++cc) {
+          float o[32];
+          tmem_ld32(tO + cc * 32, o);
+          tmem_wait_ld();
 #pragma unroll
-            for (int i = 0; i < 32; ++i) o[i] *= alpha;
-            tmem_st32(tO + cc * 32, o);
-          }
-          tmem_wait_st();
+          for (int i = 0; i < 32; ++i) o[i] *= alpha;
+          tmem_st32(tO + cc * 32, o);
         }
+        tmem_wait_st();
       }
       tc_fence_before();
-      mbar_arrive(b_p);
+      mbar_arrive(b_p(gj));
     }
     const int q = my_q;
     const size_t row = (head + (q >= 0 ? q : 0)) * D;
@@ -579,9 +591,10 @@ __global__ void __launch_bounds__(AttnCfg<D, MODE>::THREADS, 1) attn_kernel(cons
       my_q = has_next ? q_check(next_raw) : -1;
       warm_row(wn.head, my_q);
     }
-    if (ok && T > 0) {
-      if (!mbar_wait_warp(b_pv, (g + T - 1) & 1, a.wait_ns, abort_flag)) ok = false;
-    }
+    // O is final once the item's last two P.V have completed (the earlier
+    // ones completed before the last Q.K^T this thread has seen)
+    for (int t = T >= 2 ? T - 2 : 0; t < T && ok; ++t)
+      if (!mbar_wait_warp(b_pv(g + t), ((g + t) >> 1) & 1, a.wait_ns, abort_flag)) ok = false;
     if (ok) {
       // ------------------------------------------------------------------ epilogue
       tc_fence_after();

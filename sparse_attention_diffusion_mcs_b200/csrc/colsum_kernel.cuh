@@ -37,25 +37,6 @@ struct alignas(64) ColsumArgs {
   uint64_t wait_ns;
 };
 
-// 2^x on the FMA and ALU pipes, for x <= 1/2 (here x = s*scale*log2e - c_i
-// <= 0 up to rounding): x = n + f with n = rint(x) by the 1.5*2^23 shift,
-// p(f) ~ 2^f on [-1/2, 1/2] by a degree-5 minimax polynomial (max relative
-// error 7.5e-8; coefficients from fit_exp2_poly.py), n added to p's exponent
-// bits.  Results below 2^-126 are 0, as the MUFU ex2.approx.ftz gives.
-__device__ __forceinline__ float ex2_fma(float x) {
-  const float xc = fmaxf(x, -126.f);
-  const float y = xc + 12582912.f;            // 1.5 * 2^23: rounds xc to an integer
-  const float f = xc - (y - 12582912.f);      // in [-1/2, 1/2]
-  float p = fmaf(1.327647245e-03f, f, 9.675540961e-03f);
-  p = fmaf(p, f, 5.550713092e-02f);
-  p = fmaf(p, f, 2.402212024e-01f);
-  p = fmaf(p, f, 6.931469440e-01f);
-  p = fmaf(p, f, 1.000000119e+00f);
-  // bits(y) = bits(1.5 * 2^23) + n, and bits(1.5 * 2^23) << 23 vanishes mod 2^32
-  const uint32_t r = __float_as_uint(p) + (__float_as_uint(y) << 23);
-  return x >= -126.f ? __uint_as_float(r) : 0.f;
-}
-
 // which of every 8 consecutive exponentials run on the FMA pipe (bit i: column
 // i mod 8); the rest use the MUFU ex2
 #ifndef MCS_COLSUM_FMA_EXP_MASK

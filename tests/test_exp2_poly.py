@@ -1,4 +1,4 @@
-"""The FMA-pipe exponential of the group-scores kernel, checked on the CPU.
+"""The FMA-pipe exponential of the attention and group-scores kernels, checked on the CPU.
 
 The kernel computes 2^x for x <= 1/2 as: clamp at -126, split x = n + f with
 n = rint(x) through the 1.5*2^23 shift, a degree-5 polynomial p(f) ~ 2^f on
@@ -17,7 +17,7 @@ import numpy as np
 from sparse_attention_diffusion_mcs_b200 import fit_exp2_poly
 
 SRC = os.path.join(os.path.dirname(__file__), "..", "sparse_attention_diffusion_mcs_b200", "csrc",
-                   "colsum_kernel.cuh")
+                   "mcs_common.cuh")
 
 
 def _kernel_coeffs():
