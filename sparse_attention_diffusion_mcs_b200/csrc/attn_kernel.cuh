@@ -87,8 +87,8 @@ struct AttnCfg {
   static constexpr int N_BAR = 1 + 2 * NK + 2 * NV + 8;   // q, k/v full/empty, s_full[2], p[2], pv[2], drain, q_empty
   static constexpr int OFF_MISC = OFF_BAR + 8 * N_BAR;
   static constexpr int SMEM = OFF_MISC + 16 + 1024;          // + slack to align the base to 1 KB
-  static constexpr int THREADS = kSparse ? 384 : 224;
   static constexpr int KW = kSparse ? 4 : 1, VW = kSparse ? 3 : 1;   // issuing warps per ring
+  static constexpr int THREADS = (5 + KW + VW) * 32;   // softmax 0-3, MMA 4, then the K and V warps
   // dense modes keep the whole score row in registers (one TMEM pass); the
   // 384-thread sparse CTA caps registers at 168, so it reads S twice
   static constexpr bool kOnePass = !kSparse;
