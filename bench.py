@@ -51,6 +51,10 @@ def parse_args():
     ap.add_argument("--cpu-seconds", type=float, default=12.0, help="CPU baseline budget")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--sweep", action="store_true",
+                    help="sparsity sweep on the 131K-token layer: one JSON line per (G, k) point "
+                         "(plan, reused step and dense times, roofline fraction, speedup)")
+    ap.add_argument("--sweep-reps", type=int, default=5, help="timed repetitions per sweep point")
     return ap.parse_args()
 
 
@@ -283,10 +287,71 @@ def workload_config(w, n):
 
 # ----------------------------------------------------------------------------- main arm
 
+def run_sweep(args):
+    """Sparsity sweep of the 131K-token video layer (B=1, H=24, N=131072,
+    d=128): for G in {64, 128} and k = floor(p N) with p in {1, 2, 5, 10, 25} %,
+    time the plan (all five stages), the reused step on drifted inputs and
+    dense attention with CUDA events, after one warm-up of each, and print one
+    JSON line per point.  The inputs do not depend on G or k, so they are made
+    once.  Not the contract line: the driver never passes --sweep."""
+    import torch
+    import sparse_attention_diffusion_mcs_b200 as mcs
+    base = synth.workload(5)
+    if args.heads:
+        base = base.with_(H=min(args.heads, base.H))
+    s1, s2 = make_inputs(base, 0)
+    dev = torch.device("cuda", 0)
+    up = lambda a: torch.from_numpy(a.view(np.int16)).view(torch.bfloat16).to(dev)
+    Q1, K1, V1 = (up(x) for x in s1)
+    Q2, K2, V2 = (up(x) for x in s2)
+    del s1, s2
+    peaks = measured_peaks()
+    tc = peaks["bf16_tflops_sustained"]
+    stream = torch.cuda.current_stream()
+
+    def timed(fn, reps):
+        fn()
+        torch.cuda.synchronize()
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        for _ in range(reps):
+            fn()
+        b.record(stream)
+        torch.cuda.synchronize()
+        return a.elapsed_time(b) / reps
+
+    O = torch.empty_like(Q2)
+    dense_ms = timed(lambda: mcs.dense(Q2, K2, V2, base.scale, out=O), args.sweep_reps)
+    for G in (64, 128):
+        for pct in (1, 2, 5, 10, 25):
+            k = (pct * base.N) // 100
+            w = synth.workload(5, k=k, G=G).with_(H=base.H)
+            ws = mcs.alloc_workspace(w.B, w.H, w.N, w.d, G, k, dev)
+            meta = mcs.Meta.empty(w.B, w.H, w.N, w.d, G, k, dev)
+            plan_ms = timed(lambda: mcs.plan(Q1, K1, V1, G, k, w.scale, workspace=ws, meta=meta),
+                            max(1, args.sweep_reps // 2))
+            step_ms = timed(lambda: mcs.sparse_step(Q2, K2, V2, meta, w.scale, out=O), args.sweep_reps)
+            status = mcs.last_device_status()
+            tf = w.sparse_flops / (step_ms * 1e-3) / 1e12
+            print(json.dumps({
+                "sweep": "video 131K-token layer: B=1 H=%d N=%d d=%d" % (w.H, w.N, w.d),
+                "G": G, "k": k, "k_pct": pct, "plan_ms": plan_ms, "reused_step_ms": step_ms,
+                "dense_ms": dense_ms, "speedup_vs_dense": dense_ms / step_ms,
+                "step_tflops": tf, "step_frac_of_sustained_bf16": tf / tc,
+                "gathered_kv_gbs": (w.BH * w.n_groups * 4.0 * min(k, w.N) * w.d) / (step_ms * 1e-3) / 1e9,
+                "one_plan_one_step_speedup": 2 * dense_ms / (plan_ms + step_ms),
+                "device_status": status}), flush=True)
+            del ws, meta
+            torch.cuda.empty_cache()
+    return 0
+
+
 def main():
     args = parse_args()
     if args.impl == "reference":
         return run_reference(args)
+    if args.sweep:
+        return run_sweep(args)
 
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
