@@ -513,8 +513,21 @@ __global__ void __launch_bounds__(AttnCfg<D, MODE>::THREADS, 1) attn_kernel(cons
             sv[i] = ex2_approx(fmaf(sv[i], sl2, -m_run));
             if (i & 1) rs1 += sv[i]; else rs0 += sv[i];
           }
+          {
+            // P as one 64-column store of bf16 pairs (and one of the lo parts)
+            uint32_t pk[64];
 #pragma unroll
-          for (int hh = 0; hh < BN / 64; ++hh) store_p(sv + hh * 64, 32, tS + hh * 32, tPlo + hh * 32);
+            for (int i = 0; i < 64; ++i) pk[i] = pack_bf16x2(sv[2 * i], sv[2 * i + 1]);
+            tmem_st64u(tS, pk);
+            if (C::kSplit) {
+#pragma unroll
+              for (int i = 0; i < 64; ++i) {
+                const float h0 = __uint_as_float(pk[i] << 16), h1 = __uint_as_float(pk[i] & 0xFFFF0000u);
+                pk[i] = pack_bf16x2(sv[2 * i] - h0, sv[2 * i + 1] - h1);
+              }
+              tmem_st64u(tPlo, pk);
+            }
+          }
         } else {
           // pass 1: row max of this tile.  Both passes stay rolled: unrolled
           // over the four chunks they need more than the 168 registers a
