@@ -490,11 +490,11 @@ __global__ void __launch_bounds__(AttnCfg<D, MODE>::THREADS, 1) attn_kernel(cons
         if constexpr (C::kOnePass) {
           float sv[BN];
 #pragma unroll
-          for (int cc = 0; cc < BN / 32; ++cc) {
-            float tmp[32];
-            tmem_ld32(tS + cc * 32, tmp);
+          for (int cc = 0; cc < BN / 64; ++cc) {
+            float tmp[64];
+            tmem_ld64(tS + cc * 64, tmp);
 #pragma unroll
-            for (int i = 0; i < 32; ++i) sv[cc * 32 + i] = tmp[i];
+            for (int i = 0; i < 64; ++i) sv[cc * 64 + i] = tmp[i];
           }
           tmem_wait_ld();
           float m0 = -INFINITY, m1 = -INFINITY;
@@ -534,14 +534,14 @@ __global__ void __launch_bounds__(AttnCfg<D, MODE>::THREADS, 1) attn_kernel(cons
           // thread of this CTA has, and the spills cost more than the loop.
           float m0 = -INFINITY, m1 = -INFINITY;
 #pragma unroll 1
-          for (int cc = 0; cc < BN / 32; ++cc) {
-            float v[32];
-            tmem_ld32(tS + cc * 32, v);
+          for (int ch = 0; ch < BN / 64; ++ch) {
+            float v[64];
+            tmem_ld64(tS + ch * 64, v);
             tmem_wait_ld();
 #pragma unroll
-            for (int i = 0; i < 32; i += 4) {
-              m0 = fmax3(m0, val(v[i], cc * 32 + i), val(v[i + 1], cc * 32 + i + 1));
-              m1 = fmax3(m1, val(v[i + 2], cc * 32 + i + 2), val(v[i + 3], cc * 32 + i + 3));
+            for (int i = 0; i < 64; i += 4) {
+              m0 = fmax3(m0, val(v[i], ch * 64 + i), val(v[i + 1], ch * 64 + i + 1));
+              m1 = fmax3(m1, val(v[i + 2], ch * 64 + i + 2), val(v[i + 3], ch * 64 + i + 3));
             }
           }
           update_max(fmaxf(m0, m1));
