@@ -385,7 +385,20 @@ def main():
 
     stages = ["group", "stats", "scores", "topk", "residual", "step", "dense"]
 
+    # The timed step: the whole plan in one mcs_plan call, the reused step,
+    # dense attention.
     def one_step(ev):
+        ev[0].record(stream)
+        mcs.plan(Q1, K1, V1, G, k, w.scale, workspace=ws, meta=meta, out_dense=O_dense_plan)
+        ev[1].record(stream)
+        mcs.sparse_step(Q2, K2, V2, meta, w.scale, out=O_step)
+        ev[2].record(stream)
+        mcs.dense(Q2, K2, V2, w.scale, out=O_dense)
+        ev[3].record(stream)
+
+    # Per-stage times for the kernel table: the same work through the
+    # stage-by-stage entry points, each stage alone on the stream.
+    def staged_step(ev):
         ev[0].record(stream)
         mcs.plan_group(Q1, ws, out=meta.perm)
         ev[1].record(stream)
@@ -406,6 +419,7 @@ def main():
     mk = lambda: [torch.cuda.Event(enable_timing=True) for _ in range(8)]
     for _ in range(args.warmup):
         one_step(mk())
+        staged_step(mk())
     torch.cuda.synchronize()
     if mcs.last_device_status() != 0:
         raise RuntimeError("device status after warm-up is not OK")
@@ -434,16 +448,30 @@ def main():
     clk = clocks.stop()
     status = mcs.last_device_status()
     total_ms = t_start.elapsed_time(t_end)
-    per = {s: [] for s in stages}
+    whole = {"plan": [], "step": [], "dense": []}
     for ev in evs:
+        for i, s in enumerate(whole):
+            whole[s].append(ev[i].elapsed_time(ev[i + 1]))
+    whole = {s: statistics.fmean(v) for s, v in whole.items()}
+    # stage breakdown, outside the timed region
+    sevs = [mk() for _ in range(max(3, args.steps // 2))]
+    for ev in sevs:
+        staged_step(ev)
+    torch.cuda.synchronize()
+    per = {s: [] for s in stages}
+    for ev in sevs:
         for i, s in enumerate(stages):
             per[s].append(ev[i].elapsed_time(ev[i + 1]))
     mean = {s: statistics.fmean(v) for s, v in per.items()}
+    # the timed region's own reused-step and dense times
+    mean["step"], mean["dense"] = whole["step"], whole["dense"]
 
     # max over ranks
-    vec = max_over_ranks(torch.tensor([total_ms] + [mean[s] for s in stages], dtype=torch.float64, device=dev))
+    vec = max_over_ranks(torch.tensor([total_ms, whole["plan"]] + [mean[s] for s in stages],
+                                      dtype=torch.float64, device=dev))
     total_ms = float(vec[0])
-    mean = {s: float(vec[1 + i]) for i, s in enumerate(stages)}
+    plan_whole_ms = float(vec[1])
+    mean = {s: float(vec[2 + i]) for i, s in enumerate(stages)}
 
     # ------------------------------------------------------------- e2e through the public API
     e2e = None
@@ -562,7 +590,7 @@ def main():
                 "peak_kind": f"{peaks['source']} bf16 sustained" if r["bound"] == "tensor"
                 else f"{peaks['source']} HBM copy"}
 
-    plan_ms = sum(mean[s] for s in ["group", "stats", "scores", "topk", "residual"])
+    plan_ms = plan_whole_ms
     S, P = w.steps, len(w.plan_steps)
     line = {
         "metric": "reused-step sparse attention effective TFLOP/s (4*B*H*N*k*d per step), 1xB200 per rank",
@@ -580,6 +608,7 @@ def main():
         "config": workload_config(w, world),
         "reused_step_ms": mean["step"],
         "plan_ms": plan_ms,
+        "plan_stages_sum_ms": sum(mean[s] for s in ["group", "stats", "scores", "topk", "residual"]),
         "dense_ms": mean["dense"],
         "speedup_vs_dense": mean["dense"] / mean["step"],
         "amortized_speedup": S * mean["dense"] / (P * plan_ms + (S - P) * mean["step"]),
