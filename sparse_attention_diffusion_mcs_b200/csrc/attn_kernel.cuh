@@ -497,22 +497,31 @@ __global__ void __launch_bounds__(AttnCfg<D, MODE>::THREADS, 1) attn_kernel(cons
             for (int i = 0; i < 64; ++i) sv[cc * 64 + i] = tmp[i];
           }
           tmem_wait_ld();
-          float m0 = -INFINITY, m1 = -INFINITY;
+          // eight independent max and sum chains: the row reductions are
+          // latency chains, not throughput
+          float mx[8];
 #pragma unroll
-          for (int i = 0; i < BN; i += 4) {
-            sv[i] = val(sv[i], i);
-            sv[i + 1] = val(sv[i + 1], i + 1);
-            sv[i + 2] = val(sv[i + 2], i + 2);
-            sv[i + 3] = val(sv[i + 3], i + 3);
-            m0 = fmax3(m0, sv[i], sv[i + 1]);
-            m1 = fmax3(m1, sv[i + 2], sv[i + 3]);
+          for (int u = 0; u < 8; ++u) mx[u] = -INFINITY;
+#pragma unroll
+          for (int i = 0; i < BN; i += 16) {
+#pragma unroll
+            for (int u = 0; u < 8; ++u) {
+              sv[i + 2 * u] = val(sv[i + 2 * u], i + 2 * u);
+              sv[i + 2 * u + 1] = val(sv[i + 2 * u + 1], i + 2 * u + 1);
+              mx[u] = fmax3(mx[u], sv[i + 2 * u], sv[i + 2 * u + 1]);
+            }
           }
-          update_max(fmaxf(m0, m1));
+          update_max(fmaxf(fmax3(mx[0], mx[1], mx[2]), fmax3(mx[3], mx[4], fmax3(mx[5], mx[6], mx[7]))));
+          float rsv[8];
+#pragma unroll
+          for (int u = 0; u < 8; ++u) rsv[u] = 0.f;
 #pragma unroll
           for (int i = 0; i < BN; ++i) {
             sv[i] = ex2_approx(fmaf(sv[i], sl2, -m_run));
-            if (i & 1) rs1 += sv[i]; else rs0 += sv[i];
+            rsv[i & 7] += sv[i];
           }
+          rs0 = (rsv[0] + rsv[1]) + (rsv[2] + rsv[3]);
+          rs1 = (rsv[4] + rsv[5]) + (rsv[6] + rsv[7]);
           {
             // P as one 64-column store of bf16 pairs (and one of the lo parts)
             uint32_t pk[64];
