@@ -1,5 +1,5 @@
 // mcs_common.cuh -- sm_100a building blocks shared by the MC-Sparse kernels:
-// mbarriers with bounded waits, cp.async gathers, tcgen05 (TMEM alloc, UMMA
+// mbarriers with bounded waits, TMA tile and gather4 loads, tcgen05 (TMEM alloc, UMMA
 // issue, commit, TMEM load/store, fences) and shared-memory descriptors.
 #pragma once
 
@@ -158,25 +158,7 @@ __device__ __forceinline__ void tma_load_3d(uint32_t dst, const void *tmap, int 
       : "memory");
 }
 
-// ---------------------------------------------------------------------------
-// cp.async (16-byte vectors, zero fill when src_bytes == 0)
-// ---------------------------------------------------------------------------
-__device__ __forceinline__ void cp_async16(uint32_t dst, const void *src, uint32_t src_bytes) {
-  asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(dst), "l"(src),
-               "r"(src_bytes)
-               : "memory");
-}
-
-// Arrive on `bar` once every cp.async this thread issued so far has landed.
-// The barrier's expected count must include this thread (no increment).
-__device__ __forceinline__ void cp_async_arrive_noinc(uint32_t bar) {
-  asm volatile("cp.async.mbarrier.arrive.noinc.shared::cta.b64 [%0];" ::"r"(bar) : "memory");
-}
-
-__device__ __forceinline__ void cp_async_wait_all() {
-  asm volatile("cp.async.wait_all;" ::: "memory");
-}
-
+// order generic-proxy shared-memory writes before async-proxy (TMA / UMMA) reads
 __device__ __forceinline__ void fence_proxy_async_smem() {
   asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
 }
@@ -336,33 +318,9 @@ __device__ __forceinline__ void tmem_st32(uint32_t taddr, const float (&v)[32]) 
 __device__ __forceinline__ void tmem_wait_ld() {
   asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
 }
-// Wait for this thread's TMEM loads with v tied to the wait, so that no use
-// of v (the destination of an earlier, asynchronous tcgen05.ld) can be
-// scheduled above it.
-__device__ __forceinline__ void tmem_wait_ld_into(float (&v)[32]) {
-  asm volatile("tcgen05.wait::ld.sync.aligned;"
-               : "+f"(v[0]), "+f"(v[1]), "+f"(v[2]), "+f"(v[3]), "+f"(v[4]), "+f"(v[5]), "+f"(v[6]), "+f"(v[7]), "+f"(v[8]), "+f"(v[9]), "+f"(v[10]), "+f"(v[11]), "+f"(v[12]), "+f"(v[13]), "+f"(v[14]), "+f"(v[15]), "+f"(v[16]), "+f"(v[17]), "+f"(v[18]), "+f"(v[19]), "+f"(v[20]), "+f"(v[21]), "+f"(v[22]), "+f"(v[23]), "+f"(v[24]), "+f"(v[25]), "+f"(v[26]), "+f"(v[27]), "+f"(v[28]), "+f"(v[29]), "+f"(v[30]), "+f"(v[31])
-               :
-               : "memory");
-}
-__device__ __forceinline__ void tmem_ld16u(uint32_t taddr, uint32_t (&r)[16]) {
-  asm volatile("tcgen05.ld.sync.aligned.32x32b.x16.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15}, [%16];"
-               : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15])
-               : "r"(taddr));
-}
 __device__ __forceinline__ void tmem_wait_st() {
   asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
 }
 
-// ---------------------------------------------------------------------------
-// 128-byte-swizzled tile addressing.  A tile of R rows by C bf16 columns is
-// stored as C/64 column blocks of R rows x 128 bytes; inside a 1024-byte
-// aligned block the 16-byte chunk c of row r sits at chunk (c ^ (r & 7)).
-// ---------------------------------------------------------------------------
-__device__ __forceinline__ uint32_t sw128_offset(int row, int chunk16, int rows_per_block) {
-  const int blk = chunk16 >> 3;
-  const int c = chunk16 & 7;
-  return static_cast<uint32_t>(blk * rows_per_block * 128 + row * 128 + ((c ^ (row & 7)) << 4));
-}
 
 }  // namespace mcs
