@@ -10,7 +10,7 @@ PKG_DIR = os.path.dirname(os.path.abspath(__file__))
 CSRC = os.path.join(PKG_DIR, "csrc")
 LIB_PATH = os.path.join(PKG_DIR, "libmcs.so")
 SOURCES = ["mcs_api.cu"]
-HEADERS = ["mcs_common.cuh", "attn_kernel.cuh", "colsum_kernel.cuh", "topk_kernel.cuh",
+HEADERS = ["mcs_common.cuh", "attn_kernel.cuh", "attn_dual_kernel.cuh", "colsum_kernel.cuh", "topk_kernel.cuh",
            "group_kernels.cuh", "validate_kernels.cuh"]
 NVCC_FLAGS = [
     "-gencode", "arch=compute_100a,code=sm_100a",

@@ -8,6 +8,7 @@
 #include <mutex>
 
 #include "../../include/mcs.h"
+#include "attn_dual_kernel.cuh"
 #include "attn_kernel.cuh"
 #include "colsum_kernel.cuh"
 #include "group_kernels.cuh"
@@ -124,22 +125,27 @@ cudaError_t launch_attn(AttnArgs &a, const QKV &t, int grid_x, int BH, cudaStrea
     ok = map_tile(&a.tmQ, t.Q, D, a.N, BH) && map_tile(&a.tmK, t.K, D, a.N, BH) && map_tile(&a.tmV, t.V, D, a.N, BH);
   }
   if (!ok) return cudaErrorInvalidValue;
-  cudaError_t e = set_smem(attn_kernel<D, MODE>, C::SMEM);
-  if (e != cudaSuccess) return e;
-  // Sparse modes run persistent, one CTA per SM (the kernel takes all of an
-  // SM's shared memory and TMEM) looping over (head, group) items, so each
-  // item's gathers and first Q.K^T overlap the previous item's epilogue.
-  // Dense modes (long items, small epilogues) launch one CTA per item.
   a.BH = BH;
   const long items = static_cast<long>(grid_x) * BH;
-  long grid = items;
-  if (C::kSparse) {
+  if (items == 0) return cudaSuccess;
+  cudaError_t e;
+  if constexpr (!C::kSparse) {
+    // Dense modes (long items, small epilogues): one CTA per (head, query
+    // tile), two softmax warpgroups taking alternate key tiles.
+    using H = DualCfg<D, MODE>;
+    static_assert(H::SMEM <= 232448, "shared memory budget");
+    if ((e = set_smem(attn_dual_kernel<D, MODE>, H::SMEM)) != cudaSuccess) return e;
+    attn_dual_kernel<D, MODE><<<static_cast<unsigned>(items), H::THREADS, H::SMEM, s>>>(a);
+  } else {
+    // Sparse modes run persistent, one CTA per SM (the kernel takes all of an
+    // SM's shared memory and TMEM) looping over (head, group) items, so each
+    // item's gathers and first Q.K^T overlap the previous item's epilogue.
+    if ((e = set_smem(attn_kernel<D, MODE>, C::SMEM)) != cudaSuccess) return e;
     int sms = 0;
     if ((e = sm_count(&sms)) != cudaSuccess) return e;
-    if (grid > sms) grid = sms;
+    const long grid = items < sms ? items : sms;
+    attn_kernel<D, MODE><<<static_cast<unsigned>(grid), C::THREADS, C::SMEM, s>>>(a);
   }
-  if (grid == 0) return cudaSuccess;
-  attn_kernel<D, MODE><<<static_cast<unsigned>(grid), C::THREADS, C::SMEM, s>>>(a);
   return cudaGetLastError();
 }
 

@@ -171,6 +171,30 @@ def test_plan_select_on_oracle_grouping(cfg, G, k):
     assert ndiff <= 2 * w.H * w.n_groups
 
 
+@pytest.mark.parametrize("N,d,G,k", [(1000, 128, 128, 100), (777, 64, 64, 50), (129, 128, 64, 16),
+                                     (100, 64, 64, 10)])
+def test_plan_stats_rising_scores(N, d, G, k):
+    """Statistics pass on keys whose scale grows with the index, so row maxima
+    jump by more than 2^RAISE_LOG2 inside and between key tiles (m, l, the
+    output accumulators and P already written are rescaled): its dense output
+    and the selection it drives match the oracle."""
+    Q, K, V = synth.rising_qkv(1, 1, N, d, seed=7, growth=40.0)
+    q, kd, v = dev_bf16(Q), dev_bf16(K), dev_bf16(V)
+    scale = 1 / np.sqrt(d)
+    perm = orc.group_queries(Q[0, 0]).astype(np.int32)
+    ws, od = mcs.plan_stats(q, kd, v, G, k, return_dense=True)
+    mcs.plan_scores(q, kd, torch.from_numpy(perm[None, None].copy()).cuda(), G, k, ws)
+    kv = mcs.plan_topk(1, 1, N, d, G, k, ws).cpu().numpy()
+    torch.cuda.synchronize()
+    assert mcs.last_device_status() == 0
+    ref = orc.dense_attention(Q[0, 0], K[0, 0], V[0, 0], scale)
+    assert_out_close(host(od)[0, 0], ref, f"plan dense rising N{N} d{d}")
+    # the steepest rows put most keys' probabilities below fp32's range
+    c = orc.group_prob_sums(Q[0, 0], K[0, 0], scale, perm, G)
+    for g in range(c.shape[0]):
+        kv_sets_agree(kv[0, 0, g], c[g], k, G=G)
+
+
 # ----------------------------------------------------------------------------- residual (a5)
 
 @pytest.mark.parametrize("cfg,G,k", [(1, 64, 128), (1, 128, 200)])
