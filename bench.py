@@ -178,8 +178,10 @@ def measured_traffic():
     kernel sources still hash to what was profiled (else no entry)."""
     import hashlib
     csrc = os.path.join(ROOT, "sparse_attention_diffusion_mcs_b200", "csrc")
-    files = {"attn": ("mcs_common.cuh", "attn_kernel.cuh"), "colsum": ("mcs_common.cuh", "colsum_kernel.cuh"),
-             "topk": ("mcs_common.cuh", "topk_kernel.cuh")}
+    files = {"attn_kernel": ("mcs_common.cuh", "attn_kernel.cuh"),
+             "attn_dual_kernel": ("mcs_common.cuh", "attn_kernel.cuh", "attn_dual_kernel.cuh"),
+             "colsum_kernel": ("mcs_common.cuh", "colsum_kernel.cuh"),
+             "topk_kernel": ("mcs_common.cuh", "topk_kernel.cuh")}
     hashes = {}
     for key, fs in files.items():
         m = hashlib.sha256()
@@ -193,8 +195,7 @@ def measured_traffic():
             if line.startswith("#") or not line.strip():
                 continue
             stage, kernel, hsh, rd, wr = line.split()
-            fam = kernel.split("_")[0] if kernel.split("_")[0] in files else "attn"
-            if hashes.get(fam) == hsh:
+            if hashes.get(kernel.split("<")[0]) == hsh:
                 out[stage] = int(rd) + int(wr)
     except OSError:
         pass

@@ -1,8 +1,7 @@
-// attn_kernel.cuh -- one tcgen05 / TMEM / TMA flash-attention kernel, four uses.
+// attn_kernel.cuh -- the sparse tcgen05 / TMEM / TMA flash-attention kernel
+// (two uses) and the argument block it shares with the dense kernel of
+// attn_dual_kernel.cuh.
 //
-//  kModeDense     O = softmax(scale Q K^T) V over all N keys, bf16 out.  The
-//                 dense baseline of the pages ("relative to dense attention",
-//                 aiqbench.com abstract).
 //  kModeStep      the reused denoising step (split-precision P, like the plan
 //                 passes): each CTA owns one query group
 //                 (rows gathered through perm), attends only to the group's
@@ -12,27 +11,24 @@
 //                 groups, KV indices and residuals "reused across subsequent
 //                 denoising steps"; cnshai.top post, section "MC-Sparse:
 //                 three failure modes, one fix").
-//  kModePlanDense dense pass of the metadata plan: exact row statistics
-//                 (m, l) of the softmax over all keys plus the dense output in
-//                 fp32.  P is split into bf16 hi + lo parts, two MMAs, so the
-//                 fp32 output carries ~2^-17 relative error instead of 2^-9.
-//  kModePlanResid sparse pass of the plan with the same split precision;
-//                 epilogue writes R = O_dense - O_sparse (the cached residual
-//                 "between dense and sparse attention outputs").
+//  kModePlanResid sparse pass of the plan with split-precision P (bf16 hi +
+//                 lo parts, two P.V MMAs, ~2^-17 relative error instead of
+//                 2^-9); the epilogue writes R = O_dense - O_sparse (the cached
+//                 residual "between dense and sparse attention outputs").
+// (kModeDense and kModePlanDense, the dense passes, run in attn_dual_kernel.cuh.)
 //
-// CTA = 128 query rows x all KV tiles of 128 keys:
+// A persistent CTA per SM takes (head, query group) items; per item, 128
+// query rows x all of the group's key tiles of 128 keys:
 //   warps 0-3  softmax + epilogue; thread t owns query row t = TMEM lane t
 //   warp  4    TMEM allocation and the single UMMA-issuing thread
-//   sparse modes (384 threads): warps 5-8 Q and K producers, 9-11 V producers
-//   dense modes  (224 threads): warp 5 Q and K producer, warp 6 V producer
-// Rows listed by index (sparse modes) arrive through TMA tile::gather4, four
+//   warps 5-8  Q and K producers, 9-11 V producers (384 threads)
+// Rows listed by index arrive through TMA tile::gather4, four
 // 128-byte rows per instruction.  On B200 its throughput grows with the
 // number of issuing warps (measured 2.1 TB/s from one warp, 3.4 from two, 5
 // from four, 6.4 from eight), so the K ring has four issuing warps and the V
 // ring three, each owning an interleaved share of the tile's gather4
 // operations.  (A 288-thread CTA is register-allocated like 384 threads, so
-// the extra warps cost no registers.)  Contiguous tiles (dense modes) arrive through
-// 3D tile loads whose row bound is the head, so the ragged tail is zero.
+// the extra warps cost no registers.)
 // TMEM: S double buffer (2 x 128 fp32 columns) + O (D columns) + the lo part
 // of P (2 x 64 columns).  P's hi part (bf16 pairs) is written over its own S
 // buffer; P.V runs with A straight from TMEM, so shared memory holds only Q
@@ -47,6 +43,8 @@
 namespace mcs {
 
 enum AttnMode : int { kModeDense = 0, kModeStep = 1, kModePlanDense = 2, kModePlanResid = 3 };
+
+constexpr bool is_sparse_mode(int mode) { return mode == kModeStep || mode == kModePlanResid; }
 
 struct alignas(64) AttnArgs {
   CUtensorMap tmQ, tmK, tmV;   // gather maps (2D, box {64,1}) or tile maps (3D, box {64,128,1})
@@ -70,12 +68,11 @@ struct alignas(64) AttnArgs {
 
 template <int D, int MODE>
 struct AttnCfg {
+  static_assert(is_sparse_mode(MODE), "sparse modes only");
   static constexpr int BM = 128, BN = 128;
-  static constexpr bool kSparse = (MODE == kModeStep || MODE == kModePlanResid);
-  // split-precision P (bf16 hi + lo, two P.V MMAs) everywhere except the dense
-  // baseline: the reused step adds a residual that can nearly cancel the
-  // sparse output, so the sparse output needs more than bf16's 2^-9
-  static constexpr bool kSplit = (MODE != kModeDense);
+  // split-precision P (bf16 hi + lo, two P.V MMAs): the reused step adds a
+  // residual that can nearly cancel the sparse output, so the sparse output
+  // needs more than bf16's 2^-9
   static constexpr int NK = D == 64 ? 6 : 3;   // K ring depth
   static constexpr int NV = D == 64 ? 6 : 3;   // V ring depth
   static constexpr int Q_BYTES = BM * D * 2;
@@ -87,11 +84,8 @@ struct AttnCfg {
   static constexpr int N_BAR = 1 + 2 * NK + 2 * NV + 8;   // q, k/v full/empty, s_full[2], p[2], pv[2], drain, q_empty
   static constexpr int OFF_MISC = OFF_BAR + 8 * N_BAR;
   static constexpr int SMEM = OFF_MISC + 16 + 1024;          // + slack to align the base to 1 KB
-  static constexpr int KW = kSparse ? 4 : 1, VW = kSparse ? 3 : 1;   // issuing warps per ring
+  static constexpr int KW = 4, VW = 3;   // issuing warps per ring
   static constexpr int THREADS = (5 + KW + VW) * 32;   // softmax 0-3, MMA 4, then the K and V warps
-  // dense modes keep the whole score row in registers (one TMEM pass); the
-  // 384-thread sparse CTA caps registers at 168, so it reads S twice
-  static constexpr bool kOnePass = !kSparse;
   // The softmax reference max trails the true row max by up to 2^kRaise (log2
   // units) before O and l are rescaled.  bf16 P and fp32 O, l keep their
   // relative precision at any scale, so the only bound is range: P <= 2^32
@@ -140,14 +134,13 @@ __global__ void __launch_bounds__(AttnCfg<D, MODE>::THREADS, 1) attn_kernel(cons
   const int warp = tid >> 5;
   const int lane = tid & 31;
   const int N = a.N;
-  // Work items are (head, query tile) pairs (dense modes) or (head, query
-  // group) pairs (sparse modes), head-major; CTA c takes items c, c + grid,
+  // Work items are (head, query group) pairs, head-major; CTA c takes items c, c + grid,
   // c + 2 grid, ...  Every item has the same number of key tiles T, so the
   // rings, S buffers and barrier phases run on one tile counter per CTA and
   // the next item's loads and first Q.K^T overlap this item's epilogue.
-  const int per_head = C::kSparse ? a.n_groups : (N + BM - 1) / BM;
+  const int per_head = a.n_groups;
   const int n_items = a.BH * per_head;
-  const int nkeys = C::kSparse ? a.k : N;
+  const int nkeys = a.k;
   const int T = (nkeys + BN - 1) / BN;
   struct Item {
     int tile, bh;
@@ -159,7 +152,7 @@ __global__ void __launch_bounds__(AttnCfg<D, MODE>::THREADS, 1) attn_kernel(cons
     w.tile = item % per_head;
     w.bh = item / per_head;
     w.head = static_cast<size_t>(w.bh) * N;
-    w.kv_list = C::kSparse ? a.kv_idx + (static_cast<size_t>(w.bh) * a.n_groups + w.tile) * a.k : nullptr;
+    w.kv_list = a.kv_idx + (static_cast<size_t>(w.bh) * a.n_groups + w.tile) * a.k;
     return w;
   };
 
@@ -167,16 +160,11 @@ __global__ void __launch_bounds__(AttnCfg<D, MODE>::THREADS, 1) attn_kernel(cons
   // q_raw only loads (so the load can be issued long before its use);
   // q_check validates what it loaded.
   auto q_raw = [&](const Item &w, int r) -> int {
-    if (C::kSparse) {
-      const int gr = w.tile * a.G + r;
-      return (r >= a.G || gr >= N) ? -1 : a.perm[w.head + gr];
-    } else {
-      const int q = w.tile * BM + r;
-      return q < N ? q : -1;
-    }
+    const int gr = w.tile * a.G + r;
+    return (r >= a.G || gr >= N) ? -1 : a.perm[w.head + gr];
   };
   auto q_check = [&](int q) -> int {
-    if (C::kSparse && q != -1 && static_cast<unsigned>(q) >= static_cast<unsigned>(N)) {
+    if (q != -1 && static_cast<unsigned>(q) >= static_cast<unsigned>(N)) {
       record_status(a.status, kStatusBadMeta);   // corrupt metadata: never gather out of range
       return -1;
     }
@@ -228,7 +216,7 @@ __global__ void __launch_bounds__(AttnCfg<D, MODE>::THREADS, 1) attn_kernel(cons
     const void *tm = is_k ? static_cast<const void *>(&a.tmK) : static_cast<const void *>(&a.tmV);
     const int NS = is_k ? NK : NV;
     const uint32_t ring = is_k ? sK0 : sV0;
-    // sparse: gather4 operation o (4 rows x 128 bytes) of a tile belongs to
+    // gather4 operation o (4 rows x 128 bytes) of a tile belongs to
     // warp o % NW, lane o / NW; a tile has 32 row quads x NDB column blocks
     constexpr int OPS = 32 * NDB;
     const int op_raw = h + NW * lane;
@@ -240,7 +228,7 @@ __global__ void __launch_bounds__(AttnCfg<D, MODE>::THREADS, 1) attn_kernel(cons
     int nq = 0;                               // Q tiles loaded (K ring warps)
     for (int item = blockIdx.x, it = 0; item < n_items && ok; item += gridDim.x, ++it) {
       const Item w = item_at(item);
-      // global row indices of tile t for this lane's gather4 (sparse modes)
+      // global row indices of tile t for this lane's gather4
       auto tile_rows = [&](int t, int (&rows)[4]) {
         const int first = w.kv_list[0];
 #pragma unroll
@@ -255,7 +243,7 @@ __global__ void __launch_bounds__(AttnCfg<D, MODE>::THREADS, 1) attn_kernel(cons
         }
       };
       int rows[4] = {0, 0, 0, 0}, next[4] = {0, 0, 0, 0};
-      if (C::kSparse) tile_rows(0, rows);
+      tile_rows(0, rows);
       if (is_k) {
         // the item's Q tile, once the previous item's last Q.K^T has read the buffer
         if (it > 0) {
@@ -264,31 +252,24 @@ __global__ void __launch_bounds__(AttnCfg<D, MODE>::THREADS, 1) attn_kernel(cons
           got = __shfl_sync(0xffffffffu, got, 0);
           if (!got) { ok = false; break; }
         }
-        if (C::kSparse) {
-          const int q0 = q_token(w, 0);
-          const int fallback = q0 >= 0 ? q0 : 0;   // padding rows re-read a valid row
-          int qrows[4];
+        const int q0 = q_token(w, 0);
+        const int fallback = q0 >= 0 ? q0 : 0;   // padding rows re-read a valid row
+        int qrows[4];
 #pragma unroll
-          for (int i = 0; i < 4; ++i) {
-            const int q = q_token(w, 4 * quad + i);
-            qrows[i] = static_cast<int>(w.head) + (q >= 0 ? q : fallback);
-          }
-          if (h == 0 && lane == 0) mbar_arrive_expect_tx(b_q, TILE_TX);
-          __syncwarp();
-          if (active)
-            tma_gather4(sQ + dbk * (BM * 128) + quad * 512, &a.tmQ, dbk * 64, qrows[0], qrows[1], qrows[2],
-                        qrows[3], b_q);
-        } else if (h == 0 && lane == 0) {
-          mbar_arrive_expect_tx(b_q, TILE_TX);
-#pragma unroll
-          for (int db = 0; db < NDB; ++db)
-            tma_load_3d(sQ + db * (BM * 128), &a.tmQ, db * 64, w.tile * BM, w.bh, b_q);
+        for (int i = 0; i < 4; ++i) {
+          const int q = q_token(w, 4 * quad + i);
+          qrows[i] = static_cast<int>(w.head) + (q >= 0 ? q : fallback);
         }
+        if (h == 0 && lane == 0) mbar_arrive_expect_tx(b_q, TILE_TX);
+        __syncwarp();
+        if (active)
+          tma_gather4(sQ + dbk * (BM * 128) + quad * 512, &a.tmQ, dbk * 64, qrows[0], qrows[1], qrows[2],
+                      qrows[3], b_q);
         ++nq;
       }
       for (int j = 0; j < T; ++j) {
         const int s = issued % NS;
-        if (C::kSparse && j + 1 < T) tile_rows(j + 1, next);   // in flight while we wait for the slot
+        if (j + 1 < T) tile_rows(j + 1, next);   // in flight while we wait for the slot
         int got = 1;
         if (lane == 0)
           got = mbar_wait(is_k ? b_kempty(s) : b_vempty(s), ((issued / NS) & 1) ^ 1, a.wait_ns, abort_flag);
@@ -296,19 +277,13 @@ __global__ void __launch_bounds__(AttnCfg<D, MODE>::THREADS, 1) attn_kernel(cons
         if (!got) { ok = false; break; }
         const uint32_t full = is_k ? b_kfull(s) : b_vfull(s);
         const uint32_t dst = ring + s * C::KV_BYTES;
-        if (C::kSparse) {
-          // one expect-tx arrival per phase; the other warps' bytes may land first
-          if (h == 0 && lane == 0) mbar_arrive_expect_tx(full, TILE_TX);
-          __syncwarp();
-          if (active)
-            tma_gather4(dst + dbk * (BN * 128) + quad * 512, tm, dbk * 64, rows[0], rows[1], rows[2], rows[3], full);
+        // one expect-tx arrival per phase; the other warps' bytes may land first
+        if (h == 0 && lane == 0) mbar_arrive_expect_tx(full, TILE_TX);
+        __syncwarp();
+        if (active)
+          tma_gather4(dst + dbk * (BN * 128) + quad * 512, tm, dbk * 64, rows[0], rows[1], rows[2], rows[3], full);
 #pragma unroll
-          for (int i = 0; i < 4; ++i) rows[i] = next[i];
-        } else if (lane == 0) {
-          mbar_arrive_expect_tx(full, TILE_TX);
-#pragma unroll
-          for (int db = 0; db < NDB; ++db) tma_load_3d(dst + db * (BN * 128), tm, db * 64, j * BN, w.bh, full);
-        }
+        for (int i = 0; i < 4; ++i) rows[i] = next[i];
         ++issued;
       }
     }
@@ -365,12 +340,10 @@ __global__ void __launch_bounds__(AttnCfg<D, MODE>::THREADS, 1) attn_kernel(cons
           const uint64_t bdesc = sdesc_sw128(vb + kk * 16 * 128, BN * 128, 1024);
           umma_bf16_ts(tO, tP + kk * 8, bdesc, idesc_pv, (j > 0 || kk > 0) ? 1u : 0u);
         }
-        if (C::kSplit) {
 #pragma unroll
-          for (int kk = 0; kk < BN / 16; ++kk) {
-            const uint64_t bdesc = sdesc_sw128(vb + kk * 16 * 128, BN * 128, 1024);
-            umma_bf16_ts(tO, tPlo + kk * 8, bdesc, idesc_pv, 1u);
-          }
+        for (int kk = 0; kk < BN / 16; ++kk) {
+          const uint64_t bdesc = sdesc_sw128(vb + kk * 16 * 128, BN * 128, 1024);
+          umma_bf16_ts(tO, tPlo + kk * 8, bdesc, idesc_pv, 1u);
         }
         umma_commit(b_pv(gj));
         umma_commit(b_vempty(s));
@@ -405,10 +378,9 @@ __global__ void __launch_bounds__(AttnCfg<D, MODE>::THREADS, 1) attn_kernel(cons
     bool ok = true;
     int g = 0;                                   // this CTA's key tiles so far (all items)
     // the epilogue's second input (residual, or the dense output), read per row
-    constexpr bool kEpiIn = (MODE == kModeStep || MODE == kModePlanResid);
     const float *ep_in = MODE == kModeStep ? a.residual : a.O32_in;
     auto warm_row = [&](size_t head_, int q) {   // pull the row into L2 well before the epilogue
-      if (kEpiIn && q >= 0) {
+      if (q >= 0) {
 #pragma unroll
         for (int c = 0; c < D / 32; ++c)
           asm volatile("prefetch.global.L2 [%0];" ::"l"(ep_in + (head_ + q) * D + c * 32));
@@ -450,36 +422,18 @@ __global__ void __launch_bounds__(AttnCfg<D, MODE>::THREADS, 1) attn_kernel(cons
           resc = true;
         }
       };
-      // P as bf16 pairs over S; the lo parts (split modes) in their own columns
-      auto store_p = [&](const float *pv, int n32, uint32_t dst_hi, uint32_t dst_lo) {
-        // n32 = number of 32-bit columns (pairs) to write from pv
-        if (n32 == 32) {
-          uint32_t pk[32];
+      // P of 32 keys as 16 bf16 pairs over S; their lo parts in their own columns
+      auto store_p = [&](const float (&pv)[32], uint32_t dst_hi, uint32_t dst_lo) {
+        uint32_t pk[16];
 #pragma unroll
-          for (int i = 0; i < 32; ++i) pk[i] = pack_bf16x2(pv[2 * i], pv[2 * i + 1]);
-          tmem_st32u(dst_hi, pk);
-          if (C::kSplit) {
+        for (int i = 0; i < 16; ++i) pk[i] = pack_bf16x2(pv[2 * i], pv[2 * i + 1]);
+        tmem_st16u(dst_hi, pk);
 #pragma unroll
-            for (int i = 0; i < 32; ++i) {
-              const float h0 = __uint_as_float(pk[i] << 16), h1 = __uint_as_float(pk[i] & 0xFFFF0000u);
-              pk[i] = pack_bf16x2(pv[2 * i] - h0, pv[2 * i + 1] - h1);
-            }
-            tmem_st32u(dst_lo, pk);
-          }
-        } else {
-          uint32_t pk[16];
-#pragma unroll
-          for (int i = 0; i < 16; ++i) pk[i] = pack_bf16x2(pv[2 * i], pv[2 * i + 1]);
-          tmem_st16u(dst_hi, pk);
-          if (C::kSplit) {
-#pragma unroll
-            for (int i = 0; i < 16; ++i) {
-              const float h0 = __uint_as_float(pk[i] << 16), h1 = __uint_as_float(pk[i] & 0xFFFF0000u);
-              pk[i] = pack_bf16x2(pv[2 * i] - h0, pv[2 * i + 1] - h1);
-            }
-            tmem_st16u(dst_lo, pk);
-          }
+        for (int i = 0; i < 16; ++i) {
+          const float h0 = __uint_as_float(pk[i] << 16), h1 = __uint_as_float(pk[i] & 0xFFFF0000u);
+          pk[i] = pack_bf16x2(pv[2 * i] - h0, pv[2 * i + 1] - h1);
         }
+        tmem_st16u(dst_lo, pk);
       };
       auto tile_body = [&](auto masked_tag) {
         constexpr bool kMask = decltype(masked_tag)::value;
@@ -487,91 +441,39 @@ __global__ void __launch_bounds__(AttnCfg<D, MODE>::THREADS, 1) attn_kernel(cons
           if constexpr (kMask) return col < nvalid ? x : -INFINITY;
           else return x;
         };
-        if constexpr (C::kOnePass) {
-          float sv[BN];
-#pragma unroll
-          for (int cc = 0; cc < BN / 64; ++cc) {
-            float tmp[64];
-            tmem_ld64(tS + cc * 64, tmp);
-#pragma unroll
-            for (int i = 0; i < 64; ++i) sv[cc * 64 + i] = tmp[i];
-          }
+        // pass 1: row max of this tile.  Both passes stay rolled: unrolled
+        // over the four chunks they need more than the 168 registers a
+        // thread of this CTA has, and the spills cost more than the loop.
+        float m0 = -INFINITY, m1 = -INFINITY;
+#pragma unroll 1
+        for (int ch = 0; ch < BN / 64; ++ch) {
+          float v[64];
+          tmem_ld64(tS + ch * 64, v);
           tmem_wait_ld();
-          // eight independent max and sum chains: the row reductions are
-          // latency chains, not throughput
-          float mx[8];
 #pragma unroll
-          for (int u = 0; u < 8; ++u) mx[u] = -INFINITY;
-#pragma unroll
-          for (int i = 0; i < BN; i += 16) {
-#pragma unroll
-            for (int u = 0; u < 8; ++u) {
-              sv[i + 2 * u] = val(sv[i + 2 * u], i + 2 * u);
-              sv[i + 2 * u + 1] = val(sv[i + 2 * u + 1], i + 2 * u + 1);
-              mx[u] = fmax3(mx[u], sv[i + 2 * u], sv[i + 2 * u + 1]);
-            }
+          for (int i = 0; i < 64; i += 4) {
+            m0 = fmax3(m0, val(v[i], ch * 64 + i), val(v[i + 1], ch * 64 + i + 1));
+            m1 = fmax3(m1, val(v[i + 2], ch * 64 + i + 2), val(v[i + 3], ch * 64 + i + 3));
           }
-          update_max(fmaxf(fmax3(mx[0], mx[1], mx[2]), fmax3(mx[3], mx[4], fmax3(mx[5], mx[6], mx[7]))));
-          float rsv[8];
-#pragma unroll
-          for (int u = 0; u < 8; ++u) rsv[u] = 0.f;
-#pragma unroll
-          for (int i = 0; i < BN; ++i) {
-            sv[i] = ex2_approx(fmaf(sv[i], sl2, -m_run));
-            rsv[i & 7] += sv[i];
-          }
-          rs0 = (rsv[0] + rsv[1]) + (rsv[2] + rsv[3]);
-          rs1 = (rsv[4] + rsv[5]) + (rsv[6] + rsv[7]);
-          {
-            // P as one 64-column store of bf16 pairs (and one of the lo parts)
-            uint32_t pk[64];
-#pragma unroll
-            for (int i = 0; i < 64; ++i) pk[i] = pack_bf16x2(sv[2 * i], sv[2 * i + 1]);
-            tmem_st64u(tS, pk);
-            if (C::kSplit) {
-#pragma unroll
-              for (int i = 0; i < 64; ++i) {
-                const float h0 = __uint_as_float(pk[i] << 16), h1 = __uint_as_float(pk[i] & 0xFFFF0000u);
-                pk[i] = pack_bf16x2(sv[2 * i] - h0, sv[2 * i + 1] - h1);
-              }
-              tmem_st64u(tPlo, pk);
-            }
-          }
-        } else {
-          // pass 1: row max of this tile.  Both passes stay rolled: unrolled
-          // over the four chunks they need more than the 168 registers a
-          // thread of this CTA has, and the spills cost more than the loop.
-          float m0 = -INFINITY, m1 = -INFINITY;
+        }
+        update_max(fmaxf(m0, m1));
+        // pass 2: P = 2^(s*scale*log2e - m); chunk cc lands on columns [16cc, 16cc+16),
+        // all of them already read
 #pragma unroll 1
-          for (int ch = 0; ch < BN / 64; ++ch) {
-            float v[64];
-            tmem_ld64(tS + ch * 64, v);
-            tmem_wait_ld();
+        for (int cc = 0; cc < BN / 32; ++cc) {
+          float v[32];
+          tmem_ld32(tS + cc * 32, v);
+          tmem_wait_ld();
 #pragma unroll
-            for (int i = 0; i < 64; i += 4) {
-              m0 = fmax3(m0, val(v[i], ch * 64 + i), val(v[i + 1], ch * 64 + i + 1));
-              m1 = fmax3(m1, val(v[i + 2], ch * 64 + i + 2), val(v[i + 3], ch * 64 + i + 3));
+          for (int i = 0; i < 32; ++i) {
+            if constexpr (kMask) {
+              v[i] = (cc * 32 + i < nvalid) ? ex2_approx(fmaf(v[i], sl2, -m_run)) : 0.f;
+            } else {
+              v[i] = ex2_approx(fmaf(v[i], sl2, -m_run));
             }
+            if (i & 1) rs1 += v[i]; else rs0 += v[i];
           }
-          update_max(fmaxf(m0, m1));
-          // pass 2: P = 2^(s*scale*log2e - m); chunk cc lands on columns [16cc, 16cc+16),
-          // all of them already read
-#pragma unroll 1
-          for (int cc = 0; cc < BN / 32; ++cc) {
-            float v[32];
-            tmem_ld32(tS + cc * 32, v);
-            tmem_wait_ld();
-#pragma unroll
-            for (int i = 0; i < 32; ++i) {
-              if constexpr (kMask) {
-                v[i] = (cc * 32 + i < nvalid) ? ex2_approx(fmaf(v[i], sl2, -m_run)) : 0.f;
-              } else {
-                v[i] = ex2_approx(fmaf(v[i], sl2, -m_run));
-              }
-              if (i & 1) rs1 += v[i]; else rs0 += v[i];
-            }
-            store_p(v, 16, tS + cc * 16, tPlo + cc * 16);
-          }
+          store_p(v, tS + cc * 16, tPlo + cc * 16);
         }
       };
       if (nvalid >= BN) tile_body(std::false_type{});
@@ -604,7 +506,7 @@ __global__ void __launch_bounds__(AttnCfg<D, MODE>::THREADS, 1) attn_kernel(cons
     const size_t row = (head + (q >= 0 ? q : 0)) * D;
     // the epilogue input of the first chunk is in flight while the last P.V runs
     float4 ein[8];
-    if (kEpiIn && q >= 0) {
+    if (q >= 0) {
       const float4 *src = reinterpret_cast<const float4 *>(ep_in + row);
 #pragma unroll
       for (int u = 0; u < 8; ++u) ein[u] = __ldg(src + u);
@@ -626,7 +528,7 @@ __global__ void __launch_bounds__(AttnCfg<D, MODE>::THREADS, 1) attn_kernel(cons
       for (int cc = 0; cc < D / 32; ++cc) {
         // next chunk's input in flight while this chunk is finished
         float4 enx[8];
-        if (kEpiIn && q >= 0 && cc + 1 < D / 32) {
+        if (q >= 0 && cc + 1 < D / 32) {
           const float4 *src = reinterpret_cast<const float4 *>(ep_in + row + (cc + 1) * 32);
 #pragma unroll
           for (int u = 0; u < 8; ++u) enx[u] = __ldg(src + u);
@@ -653,13 +555,7 @@ __global__ void __launch_bounds__(AttnCfg<D, MODE>::THREADS, 1) attn_kernel(cons
             rp[u] = make_float4(ein[u].x - o[4 * u], ein[u].y - o[4 * u + 1], ein[u].z - o[4 * u + 2],
                                 ein[u].w - o[4 * u + 3]);
         }
-        if (MODE == kModePlanDense) {
-          float4 *op = reinterpret_cast<float4 *>(a.O32 + row + cc * 32);
-#pragma unroll
-          for (int u = 0; u < 8; ++u)
-            op[u] = make_float4(o[4 * u], o[4 * u + 1], o[4 * u + 2], o[4 * u + 3]);
-        }
-        if (MODE == kModeDense || MODE == kModeStep || (MODE == kModePlanDense && a.O != nullptr)) {
+        if (MODE == kModeStep) {
           uint4 *op = reinterpret_cast<uint4 *>(a.O + row + cc * 32);
 #pragma unroll
           for (int u = 0; u < 4; ++u) {
@@ -672,14 +568,10 @@ __global__ void __launch_bounds__(AttnCfg<D, MODE>::THREADS, 1) attn_kernel(cons
           }
         }
         }   // q >= 0
-        if (kEpiIn && cc + 1 < D / 32) {
+        if (cc + 1 < D / 32) {
 #pragma unroll
           for (int u = 0; u < 8; ++u) ein[u] = enx[u];
         }
-      }
-      if (MODE == kModePlanDense && q >= 0) {
-        a.row_m[head + q] = m_run;
-        a.row_l[head + q] = l_run;
       }
     }
     }   // items

@@ -115,31 +115,29 @@ struct QKV {
 
 template <int D, int MODE>
 cudaError_t launch_attn(AttnArgs &a, const QKV &t, int grid_x, int BH, cudaStream_t s) {
-  using C = AttnCfg<D, MODE>;
-  static_assert(C::SMEM <= 232448, "shared memory budget");
-  bool ok;
-  if (C::kSparse) {
-    const size_t rows = static_cast<size_t>(BH) * a.N;
-    ok = map_gather(&a.tmQ, t.Q, D, rows) && map_gather(&a.tmK, t.K, D, rows) && map_gather(&a.tmV, t.V, D, rows);
-  } else {
-    ok = map_tile(&a.tmQ, t.Q, D, a.N, BH) && map_tile(&a.tmK, t.K, D, a.N, BH) && map_tile(&a.tmV, t.V, D, a.N, BH);
-  }
-  if (!ok) return cudaErrorInvalidValue;
   a.BH = BH;
   const long items = static_cast<long>(grid_x) * BH;
-  if (items == 0) return cudaSuccess;
   cudaError_t e;
-  if constexpr (!C::kSparse) {
+  if constexpr (!is_sparse_mode(MODE)) {
     // Dense modes (long items, small epilogues): one CTA per (head, query
     // tile), two softmax warpgroups taking alternate key tiles.
-    using H = DualCfg<D, MODE>;
-    static_assert(H::SMEM <= 232448, "shared memory budget");
-    if ((e = set_smem(attn_dual_kernel<D, MODE>, H::SMEM)) != cudaSuccess) return e;
-    attn_dual_kernel<D, MODE><<<static_cast<unsigned>(items), H::THREADS, H::SMEM, s>>>(a);
+    using C = DualCfg<D, MODE>;
+    static_assert(C::SMEM <= 232448, "shared memory budget");
+    if (!(map_tile(&a.tmQ, t.Q, D, a.N, BH) && map_tile(&a.tmK, t.K, D, a.N, BH) && map_tile(&a.tmV, t.V, D, a.N, BH)))
+      return cudaErrorInvalidValue;
+    if (items == 0) return cudaSuccess;
+    if ((e = set_smem(attn_dual_kernel<D, MODE>, C::SMEM)) != cudaSuccess) return e;
+    attn_dual_kernel<D, MODE><<<static_cast<unsigned>(items), C::THREADS, C::SMEM, s>>>(a);
   } else {
     // Sparse modes run persistent, one CTA per SM (the kernel takes all of an
     // SM's shared memory and TMEM) looping over (head, group) items, so each
     // item's gathers and first Q.K^T overlap the previous item's epilogue.
+    using C = AttnCfg<D, MODE>;
+    static_assert(C::SMEM <= 232448, "shared memory budget");
+    const size_t rows = static_cast<size_t>(BH) * a.N;
+    if (!(map_gather(&a.tmQ, t.Q, D, rows) && map_gather(&a.tmK, t.K, D, rows) && map_gather(&a.tmV, t.V, D, rows)))
+      return cudaErrorInvalidValue;
+    if (items == 0) return cudaSuccess;
     if ((e = set_smem(attn_kernel<D, MODE>, C::SMEM)) != cudaSuccess) return e;
     int sms = 0;
     if ((e = sm_count(&sms)) != cudaSuccess) return e;
