@@ -336,22 +336,28 @@ __global__ void __launch_bounds__(DualCfg<D, MODE>::THREADS, 1) attn_dual_kernel
           }
           if (up) m_run = cm;
         }
-        float rsv[4] = {0.f, 0.f, 0.f, 0.f};
+        // pairs of columns through the packed two-lane fp32 instructions
+        const float2 sc2 = make_float2(sl2, sl2), nm2 = make_float2(-m_run, -m_run);
+        float2 rs2[2] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f)};
 #pragma unroll
-        for (int i = 0; i < 64; ++i) {
-          v[i] = ex2_approx(fmaf(v[i], sl2, -m_run));   // masked columns: 2^-inf = 0
-          rsv[i & 3] += v[i];
+        for (int i = 0; i < 32; ++i) {
+          const float2 x = __ffma2_rn(make_float2(v[2 * i], v[2 * i + 1]), sc2, nm2);
+          v[2 * i] = ex2_approx(x.x);   // masked columns: 2^-inf = 0
+          v[2 * i + 1] = ex2_approx(x.y);
+          rs2[i & 1] = __fadd2_rn(rs2[i & 1], make_float2(v[2 * i], v[2 * i + 1]));
         }
-        rs += (rsv[0] + rsv[1]) + (rsv[2] + rsv[3]);
+        rs += (rs2[0].x + rs2[0].y) + (rs2[1].x + rs2[1].y);
         uint32_t pk[32];
 #pragma unroll
         for (int i = 0; i < 32; ++i) pk[i] = pack_bf16x2(v[2 * i], v[2 * i + 1]);
         tmem_st32u(tS + 64 * c, pk);
         if (C::kSplit) {
+          const float2 neg1 = make_float2(-1.f, -1.f);
 #pragma unroll
           for (int i = 0; i < 32; ++i) {
-            const float h0 = __uint_as_float(pk[i] << 16), h1 = __uint_as_float(pk[i] & 0xFFFF0000u);
-            pk[i] = pack_bf16x2(v[2 * i] - h0, v[2 * i + 1] - h1);
+            const float2 h = make_float2(__uint_as_float(pk[i] << 16), __uint_as_float(pk[i] & 0xFFFF0000u));
+            const float2 lo = __ffma2_rn(h, neg1, make_float2(v[2 * i], v[2 * i + 1]));   // exact v - h
+            pk[i] = pack_bf16x2(lo.x, lo.y);
           }
           tmem_st32u(tS + 64 * c + 32, pk);
         }
