@@ -428,10 +428,12 @@ __global__ void __launch_bounds__(AttnCfg<D, MODE>::THREADS, 1) attn_kernel(cons
 #pragma unroll
         for (int i = 0; i < 16; ++i) pk[i] = pack_bf16x2(pv[2 * i], pv[2 * i + 1]);
         tmem_st16u(dst_hi, pk);
+        const float2 neg1 = make_float2(-1.f, -1.f);
 #pragma unroll
         for (int i = 0; i < 16; ++i) {
-          const float h0 = __uint_as_float(pk[i] << 16), h1 = __uint_as_float(pk[i] & 0xFFFF0000u);
-          pk[i] = pack_bf16x2(pv[2 * i] - h0, pv[2 * i + 1] - h1);
+          const float2 h = make_float2(__uint_as_float(pk[i] << 16), __uint_as_float(pk[i] & 0xFFFF0000u));
+          const float2 lo = __ffma2_rn(h, neg1, make_float2(pv[2 * i], pv[2 * i + 1]));   // exact v - h
+          pk[i] = pack_bf16x2(lo.x, lo.y);
         }
         tmem_st16u(dst_lo, pk);
       };
@@ -464,15 +466,22 @@ __global__ void __launch_bounds__(AttnCfg<D, MODE>::THREADS, 1) attn_kernel(cons
           float v[32];
           tmem_ld32(tS + cc * 32, v);
           tmem_wait_ld();
+          // column pairs through the packed two-lane fp32 instructions
+          const float2 sc2 = make_float2(sl2, sl2), nm2 = make_float2(-m_run, -m_run);
+          float2 rs2 = make_float2(rs0, rs1);
 #pragma unroll
-          for (int i = 0; i < 32; ++i) {
+          for (int i = 0; i < 32; i += 2) {
+            const float2 x = __ffma2_rn(make_float2(v[i], v[i + 1]), sc2, nm2);
+            v[i] = ex2_approx(x.x);
+            v[i + 1] = ex2_approx(x.y);
             if constexpr (kMask) {
-              v[i] = (cc * 32 + i < nvalid) ? ex2_approx(fmaf(v[i], sl2, -m_run)) : 0.f;
-            } else {
-              v[i] = ex2_approx(fmaf(v[i], sl2, -m_run));
+              if (cc * 32 + i >= nvalid) v[i] = 0.f;
+              if (cc * 32 + i + 1 >= nvalid) v[i + 1] = 0.f;
             }
-            if (i & 1) rs1 += v[i]; else rs0 += v[i];
+            rs2 = __fadd2_rn(rs2, make_float2(v[i], v[i + 1]));
           }
+          rs0 = rs2.x;
+          rs1 = rs2.y;
           store_p(v, tS + cc * 16, tPlo + cc * 16);
         }
       };

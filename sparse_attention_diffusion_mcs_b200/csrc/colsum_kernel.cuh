@@ -119,8 +119,9 @@ __global__ void __launch_bounds__(224, 2) colsum_kernel(const __grid_constant__ 
   }
   if (tid < 128) {
     const int q = q_token(tid);
-    // fold the normaliser into the exponent; a padding query contributes 2^-inf = 0
-    stat[tid] = q >= 0 ? a.row_m[head + q] + log2f(a.row_l[head + q]) : INFINITY;
+    // fold the normaliser into the exponent (stored negated, the addend of
+    // the scale-and-shift); a padding query contributes 2^-inf = 0
+    stat[tid] = q >= 0 ? -(a.row_m[head + q] + log2f(a.row_l[head + q])) : -INFINITY;
   }
   if (warp == 4) {
     tmem_alloc(smem_u32(tmem_slot), C::TMEM_COLS);
@@ -213,7 +214,8 @@ __global__ void __launch_bounds__(224, 2) colsum_kernel(const __grid_constant__ 
       const int b = j & 1;
       if (!mbar_wait_warp(b_sfull0 + 8 * b, (j >> 1) & 1, a.wait_ns, abort_flag)) { ok = false; break; }
       tc_fence_after();
-      float acc0 = 0.f, acc1 = 0.f, acc2 = 0.f, acc3 = 0.f;
+      float2 acc01 = make_float2(0.f, 0.f), acc23 = make_float2(0.f, 0.f);
+      const float2 sc2 = make_float2(sl2, sl2);
       float v[2][32];
       tmem_ld32(tbase + lane_addr + b * 128, v[0]);
 #pragma unroll
@@ -225,21 +227,18 @@ __global__ void __launch_bounds__(224, 2) colsum_kernel(const __grid_constant__ 
 #pragma unroll
         for (int i = 0; i < 32; i += 4) {
           const float4 c = c4[i / 4];     // same address in every lane: one broadcast read
-          const float cv[4] = {c.x, c.y, c.z, c.w};
+          // two queries per packed two-lane fp32 instruction
+          const float2 x01 = __ffma2_rn(make_float2(cur[i], cur[i + 1]), sc2, make_float2(c.x, c.y));
+          const float2 x23 = __ffma2_rn(make_float2(cur[i + 2], cur[i + 3]), sc2, make_float2(c.z, c.w));
+          const float x[4] = {x01.x, x01.y, x23.x, x23.y};
           float e[4];
 #pragma unroll
-          for (int u = 0; u < 4; ++u) {
-            const float x = fmaf(cur[i + u], sl2, -cv[u]);
-            e[u] = ((kFmaExpMask >> ((i + u) & 7)) & 1u) ? ex2_fma(x) : ex2_approx(x);
-          }
-          acc0 += e[0];
-          acc1 += e[1];
-          acc2 += e[2];
-          acc3 += e[3];
+          for (int u = 0; u < 4; ++u) e[u] = ((kFmaExpMask >> ((i + u) & 7)) & 1u) ? ex2_fma(x[u]) : ex2_approx(x[u]);
+          acc01 = __fadd2_rn(acc01, make_float2(e[0], e[1]));
+          acc23 = __fadd2_rn(acc23, make_float2(e[2], e[3]));
         }
       }
-      acc0 += acc1;
-      acc2 += acc3;
+      const float acc0 = acc01.x + acc01.y, acc2 = acc23.x + acc23.y;
       tc_fence_before();
       mbar_arrive(b_sfree0 + 8 * b);
       const int key = j * BM + tid;
