@@ -47,6 +47,7 @@ __all__ = [
     "group_rows", "scores", "row_stats", "probabilities", "group_prob_sums",
     "select_kv", "dense_rows", "dense_attention", "sparse_group",
     "sparse_attention", "residual_group", "plan_head", "reused_step_head",
+    "rel_l2", "schedule_head",
 ]
 
 
@@ -273,3 +274,48 @@ def reused_step_head(Q, K, V, scale: float, perm, kv_idx, residual, G: int, grou
         return sparse_attention(Q, K, V, scale, perm, kv_idx, G) + residual
     rows, osp = sparse_attention(Q, K, V, scale, perm, kv_idx, G, groups=groups)
     return rows, osp + residual[rows]
+
+
+# ---------------------------------------------------------------------------
+# A denoising loop: plan on some steps, reuse the metadata on the others
+# ---------------------------------------------------------------------------
+
+def rel_l2(x, ref) -> float:
+    """||x - ref|| / ||ref|| (Frobenius), in fp64."""
+    x = np.asarray(x, dtype=np.float64)
+    ref = np.asarray(ref, dtype=np.float64)
+    den = np.linalg.norm(ref)
+    return float(np.linalg.norm(x - ref) / den) if den > 0 else float(np.linalg.norm(x))
+
+
+def schedule_head(steps, plan_steps, G: int, k: int, scale: float):
+    """One head through a denoising loop.
+
+    ``steps`` lists the (Q, K, V) of denoising steps 1, 2, ...; ``plan_steps``
+    holds the 1-based steps that compute fresh metadata (the first step always
+    does, as nothing is cached before it).  The metadata -- query groups, KV
+    indices and residual -- are computed once and reused on the following
+    steps ([abstract]; [p1-mcs]): a plan step outputs the dense attention of
+    its own inputs, a reused step outputs O_sparse(current Q, K, V; cached
+    groups and indices) + cached R.
+
+    Returns one dict per step: kind ("plan" or "reused"), the output O, the
+    dense attention of that step's inputs, and the fidelity to it with the
+    residual (rel_l2) and without it (rel_l2_no_residual, O - R).
+    """
+    plan_steps = set(int(t) for t in plan_steps)
+    out = []
+    meta = None
+    for t, (Q, K, V) in enumerate(steps, start=1):
+        if meta is None or t in plan_steps:
+            meta = plan_head(Q, K, V, G, k, scale)
+            kind, O = "plan", meta["O_dense"]
+            Od = O
+        else:
+            kind = "reused"
+            O = reused_step_head(Q, K, V, scale, meta["perm"], meta["kv_idx"], meta["residual"], G)
+            Od = dense_attention(Q, K, V, scale)
+        out.append({"step": t, "kind": kind, "O": O, "O_dense": Od,
+                    "rel_l2": rel_l2(O, Od), "rel_l2_no_residual": rel_l2(O - meta["residual"], Od)})
+    return out
+

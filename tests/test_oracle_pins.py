@@ -268,3 +268,64 @@ def test_widen_bf16_exact():
     assert w[0] == 1.0 and w[1] == -1.0 and w[3] == 0.0
     assert w[2] == 3.140625
     assert w[4] == float(np.float32(3.3895313892515355e38))
+
+
+# --- denoising schedule ----------------------------------------------------------
+
+def _drifted(n, d, steps, seed, sigma):
+    """(Q, K, V) per step: a random walk of the step-1 tensors."""
+    rng = np.random.default_rng(seed)
+    cur = [_rand(n, d, seed + 1, 2.0), _rand(n, d, seed + 2, 2.0), _rand(n, d, seed + 3)]
+    out = [tuple(cur)]
+    for _ in range(steps - 1):
+        cur = [x + sigma * rng.standard_normal(x.shape) for x in cur]
+        out.append(tuple(cur))
+    return out
+
+
+def test_rel_l2_closed_forms():
+    ref = np.array([[3.0, 4.0]])
+    assert orc.rel_l2(ref, ref) == 0.0
+    assert orc.rel_l2(2 * ref, ref) == pytest.approx(1.0, abs=1e-15)
+    assert orc.rel_l2(ref + np.array([[0.0, 0.5]]), ref) == pytest.approx(0.1, abs=1e-15)
+
+
+def test_schedule_on_unchanged_inputs_is_dense_at_every_step():
+    st = _drifted(80, 8, 4, 100, 0.0)
+    r = orc.schedule_head(st, [1], G=16, k=8, scale=0.35)
+    assert [x["kind"] for x in r] == ["plan", "reused", "reused", "reused"]
+    dense = orc.dense_attention(*st[0], 0.35)
+    for x in r:
+        assert x["rel_l2"] < 1e-12
+        np.testing.assert_allclose(x["O"], dense, rtol=0, atol=1e-12)
+    # the same cached metadata on the same inputs: the sparse-only error is the same each step
+    assert r[0]["rel_l2_no_residual"] > 1e-3
+    for x in r[1:]:
+        assert x["rel_l2_no_residual"] == pytest.approx(r[0]["rel_l2_no_residual"], rel=1e-12)
+
+
+def test_schedule_with_k_equal_n_is_dense_with_or_without_residual():
+    st = _drifted(64, 8, 3, 200, 0.1)
+    for x in orc.schedule_head(st, [1], G=16, k=64, scale=0.35):
+        assert x["rel_l2"] < 1e-12 and x["rel_l2_no_residual"] < 1e-12
+
+
+def test_schedule_plan_steps_output_dense_of_their_own_inputs():
+    st = _drifted(64, 8, 4, 300, 0.2)
+    r = orc.schedule_head(st, [1, 3], G=16, k=6, scale=0.35)
+    assert [x["kind"] for x in r] == ["plan", "reused", "plan", "reused"]
+    for t in (0, 2):
+        np.testing.assert_allclose(r[t]["O"], orc.dense_attention(*st[t], 0.35), rtol=0, atol=1e-12)
+        assert r[t]["rel_l2"] < 1e-12
+    # drift moves the reused steps away from dense; the residual still helps
+    for t in (1, 3):
+        assert r[t]["rel_l2"] > 1e-6
+        assert r[t]["rel_l2"] < r[t]["rel_l2_no_residual"]
+
+
+def test_schedule_constant_values_exact_under_drift():
+    st = _drifted(48, 6, 3, 400, 0.3)
+    c = np.array([[1.5, -0.25, 2.0, 0.0, -1.0, 3.0]])
+    st = [(q, k, np.tile(c, (48, 1))) for q, k, _ in st]
+    for x in orc.schedule_head(st, [1], G=8, k=4, scale=0.4):
+        assert x["rel_l2"] < 1e-13 and x["rel_l2_no_residual"] < 1e-13
