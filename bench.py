@@ -55,6 +55,9 @@ def parse_args():
                     help="sparsity sweep on the 131K-token layer: one JSON line per (G, k) point "
                          "(plan, reused step and dense times, roofline fraction, speedup)")
     ap.add_argument("--sweep-reps", type=int, default=5, help="timed repetitions per sweep point")
+    ap.add_argument("--schedule", action="store_true",
+                    help="run the workload's whole denoising schedule (re-plans, drift) and report "
+                         "per-step times and fidelity to dense; not the contract line")
     return ap.parse_args()
 
 
@@ -347,10 +350,97 @@ def run_sweep(args):
     return 0
 
 
+def _drift_step_head(args):
+    cfg, k, G, bh, seed_shift, step, q, kk, v = args
+    w = synth.workload(cfg, k=k, G=G).with_(seed=seed_shift)
+    return bh, (synth.drift_head(q, w, step, 0, bh), synth.drift_head(kk, w, step, 1, bh),
+                synth.drift_head(v, w, step, 2, bh))
+
+
+def schedule_inputs(w):
+    """Yields (step, [Q, K, V] uint16 [B,H,N,d]) for steps 1 .. w.steps, each
+    step the previous one plus the workload's drift; heads in worker processes."""
+    import concurrent.futures as cf
+    import multiprocessing as mp
+    cur, _ = make_inputs(w, 0)
+    yield 1, cur
+    nproc = max(1, min(w.BH, len(os.sched_getaffinity(0)), 16))
+    with cf.ProcessPoolExecutor(nproc, mp_context=mp.get_context("spawn")) as ex:
+        for step in range(2, w.steps + 1):
+            flat = [x.reshape(w.BH, w.N, w.d) for x in cur]
+            jobs = [(w.cfg_id, w.k, w.G, bh, w.seed, step, flat[0][bh], flat[1][bh], flat[2][bh])
+                    for bh in range(w.BH)]
+            nxt = [np.empty_like(x) for x in flat]
+            for bh, t in ex.map(_drift_step_head, jobs):
+                for i in range(3):
+                    nxt[i][bh] = t[i]
+            cur = [x.reshape(w.B, w.H, w.N, w.d) for x in nxt]
+            yield step, cur
+
+
+def run_schedule(args):
+    """The workload's denoising loop through mcs.Schedule: plan on its plan
+    steps, reuse the metadata in between, inputs drifting every step.  Per
+    step: CUDA-event time of the MC-Sparse step and of dense attention on the
+    same inputs, and the output's rel-L2 to dense with and without the
+    residual.  One JSON line per step, then a summary line with the measured
+    amortised speedup (sum of dense times / sum of MC-Sparse times).  The
+    first step is run once untimed first (allocation, tensor maps)."""
+    import torch
+    import sparse_attention_diffusion_mcs_b200 as mcs
+    w = synth.workload(args.config, k=args.k, G=args.G)
+    if args.heads:
+        w = w.with_(H=min(args.heads, w.H))
+    dev = torch.device("cuda", 0)
+    up = lambda a: torch.from_numpy(a.view(np.int16)).view(torch.bfloat16).to(dev)
+    stream = torch.cuda.current_stream()
+    sch = mcs.Schedule(w.G, w.k, w.plan_steps)
+    Od = None
+    rows = []
+    for step, host in schedule_inputs(w):
+        Q, K, V = (up(x) for x in host)
+        if Od is None:
+            Od = torch.empty_like(Q)
+            sch.step(1, Q, K, V)
+            mcs.dense(Q, K, V, w.scale, out=Od)
+            sch.reset()              # the timed first step plans again, on the same buffers
+            torch.cuda.synchronize()
+        ev = [torch.cuda.Event(enable_timing=True) for _ in range(4)]
+        ev[0].record(stream)
+        O, kind = sch.step(step, Q, K, V)
+        ev[1].record(stream)
+        ev[2].record(stream)
+        mcs.dense(Q, K, V, w.scale, out=Od)
+        ev[3].record(stream)
+        torch.cuda.synchronize()
+        rel, rel_nr = mcs.fidelity(O, Od, sch.meta.residual)
+        row = {"schedule": w.name, "step": step, "kind": kind, "ms": ev[0].elapsed_time(ev[1]),
+               "dense_ms": ev[2].elapsed_time(ev[3]), "rel_l2_to_dense": rel,
+               "rel_l2_to_dense_without_residual": rel_nr, "device_status": mcs.last_device_status()}
+        rows.append(row)
+        print(json.dumps(row), flush=True)
+        del Q, K, V
+    t_mcs = sum(r["ms"] for r in rows)
+    t_dense = sum(r["dense_ms"] for r in rows)
+    reused = [r for r in rows if r["kind"] == "reused"]
+    print(json.dumps({
+        "schedule": w.name, "workload": workload_config(w, 1)["workload"],
+        "steps": w.steps, "plan_steps": list(w.plan_steps), "drift": w.drift,
+        "mcs_ms_total": t_mcs, "dense_ms_total": t_dense, "amortized_speedup_measured": t_dense / t_mcs,
+        "reused_rel_l2_mean": float(np.mean([r["rel_l2_to_dense"] for r in reused])) if reused else None,
+        "reused_rel_l2_max": max((r["rel_l2_to_dense"] for r in reused), default=None),
+        "reused_rel_l2_without_residual_mean":
+            float(np.mean([r["rel_l2_to_dense_without_residual"] for r in reused])) if reused else None,
+    }), flush=True)
+    return 0
+
+
 def main():
     args = parse_args()
     if args.impl == "reference":
         return run_reference(args)
+    if args.schedule:
+        return run_schedule(args)
     if args.sweep:
         return run_sweep(args)
 

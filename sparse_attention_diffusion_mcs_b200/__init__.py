@@ -23,3 +23,4 @@ from .api import (  # noqa: F401
     validate_meta,
     workspace_size,
 )
+from .denoise import Schedule, fidelity  # noqa: F401,E402
