@@ -32,6 +32,36 @@ def _check_qkv(*ts: torch.Tensor):
         raise ValueError("Q/K/V shapes differ")
 
 
+def _check_tensor(t: torch.Tensor, name: str, shape, dtype, device):
+    """Buffers the library writes or reads by the sizes it is given must be
+    exactly what those sizes describe: a mismatch would be an out-of-bounds
+    access on the device, so it is refused here, before any launch."""
+    if not isinstance(t, torch.Tensor):
+        raise TypeError(f"{name} must be a tensor")
+    if t.device != device or t.dtype != dtype or not t.is_contiguous() or tuple(t.shape) != tuple(shape):
+        raise ValueError(f"{name} must be a contiguous {dtype} tensor of shape {tuple(shape)} on {device}, "
+                         f"got {t.dtype} {tuple(t.shape)} on {t.device}")
+
+
+def _check_meta(meta: "Meta", B: int, H: int, N: int, d: int, device, G: Optional[int] = None,
+                k: Optional[int] = None):
+    """meta's sizes match the layer [B, H, N, d] (and G, k when given) and
+    its buffers are the sizes those describe."""
+    if (meta.B, meta.H, meta.N, meta.d) != (B, H, N, d):
+        raise ValueError(f"metadata is for [B, H, N, d] = {[meta.B, meta.H, meta.N, meta.d]}, "
+                         f"the layer is {[B, H, N, d]}")
+    if G is not None and meta.G != G:
+        raise ValueError(f"metadata group size {meta.G} != {G}")
+    if k is not None and meta.k != min(int(k), N):
+        raise ValueError(f"metadata keeps {meta.k} keys per group, not min(k, N) = {min(int(k), N)}")
+    ng = -(-N // meta.G)
+    if meta.n_groups != ng:
+        raise ValueError(f"metadata n_groups {meta.n_groups} != ceil(N / G) = {ng}")
+    _check_tensor(meta.perm, "meta.perm", (B, H, N), torch.int32, device)
+    _check_tensor(meta.kv_idx, "meta.kv_idx", (B, H, ng, meta.k), torch.int32, device)
+    _check_tensor(meta.residual, "meta.residual", (B, H, N, d), torch.float32, device)
+
+
 def _scale(d: int, scale: Optional[float]) -> float:
     return float(scale) if scale is not None else 1.0 / math.sqrt(d)
 
@@ -97,6 +127,10 @@ def plan(Q, K, V, G: int, k: int, scale: Optional[float] = None,
     B, H, N, d = Q.shape
     if meta is None:
         meta = Meta.empty(B, H, N, d, G, k, Q.device)
+    else:
+        _check_meta(meta, B, H, N, d, Q.device, G, k)
+    if out_dense is not None:
+        _check_tensor(out_dense, "out_dense", Q.shape, torch.bfloat16, Q.device)
     if return_dense and out_dense is None:
         out_dense = torch.empty_like(Q)
     ws = _ws(workspace, B, H, N, d, G, k, Q.device)
@@ -113,6 +147,8 @@ def plan_group(Q, workspace: Optional[torch.Tensor] = None,
     """Step a1 alone: int32 perm [B, H, N]."""
     _check_qkv(Q)
     B, H, N, d = Q.shape
+    if out is not None:
+        _check_tensor(out, "out", (B, H, N), torch.int32, Q.device)
     perm = out if out is not None else torch.empty((B, H, N), dtype=torch.int32, device=Q.device)
     ws = _ws(workspace, B, H, N, d, 128, 1, Q.device)
     check(lib().mcs_plan_group(_ptr(Q), B, H, N, d, _ptr(perm), _ptr(ws), ws.numel(), _stream()),
@@ -128,6 +164,8 @@ def plan_stats(Q, K, V, G: int, k: int, scale: Optional[float] = None,
     _check_qkv(Q, K, V)
     B, H, N, d = Q.shape
     ws = _ws(workspace, B, H, N, d, G, k, Q.device)
+    if out_dense is not None:
+        _check_tensor(out_dense, "out_dense", Q.shape, torch.bfloat16, Q.device)
     od = out_dense if out_dense is not None else (torch.empty_like(Q) if return_dense else None)
     check(lib().mcs_plan_stats(_ptr(Q), _ptr(K), _ptr(V), B, H, N, d, G, k, _scale(d, scale), _ptr(od),
                                _ptr(ws), ws.numel(), _stream()), "mcs_plan_stats")
@@ -140,6 +178,7 @@ def plan_scores(Q, K, perm, G: int, k: int, workspace: torch.Tensor,
     _check_qkv(Q, K)
     B, H, N, d = Q.shape
     perm = perm.to(torch.int32).contiguous()
+    _check_tensor(perm, "perm", (B, H, N), torch.int32, Q.device)
     check(lib().mcs_plan_scores(_ptr(Q), _ptr(K), _ptr(perm), B, H, N, d, G, k, _scale(d, scale),
                                 _ptr(workspace), workspace.numel(), _stream()), "mcs_plan_scores")
 
@@ -150,6 +189,8 @@ def plan_topk(B: int, H: int, N: int, d: int, G: int, k: int, workspace: torch.T
     kk = min(int(k), N)
     if out is None:
         out = torch.empty((B, H, -(-N // G), kk), dtype=torch.int32, device=workspace.device)
+    else:
+        _check_tensor(out, "out", (B, H, -(-N // G), kk), torch.int32, workspace.device)
     check(lib().mcs_plan_topk(B, H, N, d, G, k, _ptr(out), _ptr(workspace), workspace.numel(),
                               _stream()), "mcs_plan_topk")
     return out
@@ -166,6 +207,8 @@ def select_topk(scores: torch.Tensor, k: int, out: Optional[torch.Tensor] = None
     kk = min(int(k), N)
     if out is None:
         out = torch.empty((*scores.shape[:-1], kk), dtype=torch.int32, device=scores.device)
+    else:
+        _check_tensor(out, "out", (*scores.shape[:-1], kk), torch.int32, scores.device)
     if rows == 0:
         return out
     check(lib().mcs_select_topk(_ptr(scores), rows, N, int(k), _ptr(out), _stream()), "mcs_select_topk")
@@ -190,6 +233,10 @@ def plan_residual(Q, K, V, perm, kv_idx, G: int, scale: Optional[float] = None,
     perm = perm.to(torch.int32).contiguous()
     kv_idx = kv_idx.to(torch.int32).contiguous()
     k = kv_idx.shape[-1]
+    _check_tensor(perm, "perm", (B, H, N), torch.int32, Q.device)
+    _check_tensor(kv_idx, "kv_idx", (B, H, -(-N // G), min(k, N)), torch.int32, Q.device)
+    if out is not None:
+        _check_tensor(out, "out", (B, H, N, d), torch.float32, Q.device)
     od = None
     if stats_done:
         if workspace is None:
@@ -210,8 +257,11 @@ def sparse_step(Q, K, V, meta: Meta, scale: Optional[float] = None,
                 out: Optional[torch.Tensor] = None) -> torch.Tensor:
     """Reused denoising step (a6): bf16 O [B, H, N, d]."""
     _check_qkv(Q, K, V)
+    _check_meta(meta, *Q.shape, Q.device)
     if out is None:
         out = torch.empty_like(Q)
+    else:
+        _check_tensor(out, "out", Q.shape, torch.bfloat16, Q.device)
     cm = meta.c_struct()
     check(lib().mcs_sparse_step(_ptr(Q), _ptr(K), _ptr(V), ctypes.byref(cm),
                                 _scale(meta.d, scale), _ptr(out), _stream()), "mcs_sparse_step")
@@ -224,6 +274,8 @@ def dense(Q, K, V, scale: Optional[float] = None, out: Optional[torch.Tensor] = 
     B, H, N, d = Q.shape
     if out is None:
         out = torch.empty_like(Q)
+    else:
+        _check_tensor(out, "out", Q.shape, torch.bfloat16, Q.device)
     check(lib().mcs_dense(_ptr(Q), _ptr(K), _ptr(V), B, H, N, d, _scale(d, scale), _ptr(out),
                           _stream()), "mcs_dense")
     return out
