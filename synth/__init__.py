@@ -6,7 +6,7 @@ It holds none of the sparse-attention method's arithmetic, so that both the
 fp64 oracle and the CUDA path can take their inputs from it without sharing
 any other code.
 """
-from .configs import CONFIGS, Workload, workload, sweep_points
+from .workloads import WORKLOADS, Workload, workload, sweep_points
 from .dit_inputs import (
     bf16_round,
     head_tensors,
@@ -19,7 +19,7 @@ from .dit_inputs import (
 )
 
 __all__ = [
-    "CONFIGS", "Workload", "workload", "sweep_points",
+    "WORKLOADS", "Workload", "workload", "sweep_points",
     "bf16_round", "head_tensors", "layer_tensors", "drift_head", "drift_layer",
     "random_metadata_head", "random_qkv", "rising_qkv",
 ]

@@ -27,7 +27,7 @@ from __future__ import annotations
 
 import numpy as np
 
-from .configs import Workload
+from .workloads import Workload
 
 _PURPOSE_BASE = 0
 _PURPOSE_DRIFT = 1

@@ -69,7 +69,7 @@ def _pct(n: int, pct: int) -> int:
     return (n * pct) // 100
 
 
-def _mk_configs():
+def _mk_workloads():
     c1 = Workload("tiny", 1, 1, 2, (8, 8, 16), 64, 64, 128, 8, "gauss", False,
                   2, 0.05, (1,))
     n2 = 13 * 30 * 40
@@ -87,14 +87,22 @@ def _mk_configs():
     return {1: c1, 2: c2, 3: c3, 4: c4, 5: c5}
 
 
-CONFIGS = _mk_configs()
+WORKLOADS = _mk_workloads()
 
 SWEEP_PCTS = (1, 2, 5, 10, 25)
 SWEEP_GROUPS = (64, 128)
 
 
-def workload(cfg: int, k: Optional[int] = None, G: Optional[int] = None) -> Workload:
-    w = CONFIGS[cfg]
+def workload(which, k: Optional[int] = None, G: Optional[int] = None) -> Workload:
+    """A workload by id (1-5) or by name ("tiny", "video_short", "video_long",
+    "asset3d", "sweep"), optionally with another k or G."""
+    if isinstance(which, str):
+        hits = [w for w in WORKLOADS.values() if w.name == which]
+        if not hits:
+            raise KeyError(which)
+        w = hits[0]
+    else:
+        w = WORKLOADS[which]
     if k is not None:
         w = w.with_(k=k)
     if G is not None:
@@ -104,7 +112,7 @@ def workload(cfg: int, k: Optional[int] = None, G: Optional[int] = None) -> Work
 
 def sweep_points():
     """The sparsity sweep of the 131072-token workload: (G, pct, Workload)."""
-    base = CONFIGS[5]
+    base = WORKLOADS[5]
     out = []
     for G in SWEEP_GROUPS:
         for p in SWEEP_PCTS:

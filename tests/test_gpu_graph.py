@@ -15,7 +15,7 @@ pytestmark = pytest.mark.gpu
 
 
 def test_sparse_step_graph_replay_matches_eager():
-    w = synth.CONFIGS[1].with_(grid=(1, 1, 1000), d=128, G=128, k=300)
+    w = synth.workload("tiny").with_(grid=(1, 1, 1000), d=128, G=128, k=300)
     Q, K, V = synth.random_qkv(1, 2, 1000, 128, seed=8)
     perm = np.stack([synth.random_metadata_head(w, h)[0] for h in range(2)])[None]
     kv = np.stack([synth.random_metadata_head(w, h)[1] for h in range(2)])[None]

@@ -23,7 +23,7 @@ RAISE_LOG2 = 32
 
 
 def _shape_workload(N, d, G, k):
-    return synth.CONFIGS[1].with_(grid=(1, 1, N), d=d, G=G, k=k)
+    return synth.workload("tiny").with_(grid=(1, 1, N), d=d, G=G, k=k)
 
 
 # ----------------------------------------------------------------------------- dense (a7)

@@ -7,7 +7,7 @@ from synth import dit_inputs as di
 
 
 def test_workload_shapes_and_k():
-    c = synth.CONFIGS
+    c = synth.WORKLOADS
     assert (c[1].N, c[1].k, c[1].n_groups) == (1024, 128, 16)
     assert (c[2].N, c[2].k, c[2].n_groups) == (15600, 1560, 122)
     assert (c[3].N, c[3].k, c[3].n_groups) == (32760, 1638, 256)
@@ -30,7 +30,7 @@ def test_bf16_round_matches_torch_rne():
 
 
 def test_heads_deterministic_and_independently_regenerable():
-    w = synth.CONFIGS[1]
+    w = synth.workload("tiny")
     Q, K, V = synth.layer_tensors(w)
     assert Q.shape == (1, 2, 1024, 64) and Q.dtype == np.uint16
     q1, k1, v1 = synth.head_tensors(w, 1)
@@ -41,7 +41,7 @@ def test_heads_deterministic_and_independently_regenerable():
 
 
 def test_q_and_k_share_cluster_structure():
-    w = synth.CONFIGS[1]
+    w = synth.workload("tiny")
     q, k, v = synth.head_tensors(w, 0)
     f = lambda u: (u.astype(np.uint32) << 16).view(np.float32).astype(np.float64)
     q, k, v = f(q), f(k), f(v)
@@ -55,7 +55,7 @@ def test_q_and_k_share_cluster_structure():
 
 
 def test_position_embedding_layout():
-    w = synth.CONFIGS[1]           # d = 64 -> chunks 24 / 20 / 20
+    w = synth.workload("tiny")           # d = 64 -> chunks 24 / 20 / 20
     pe = di.position_embedding(w)
     assert pe.shape == (1024, 64)
     # token 0 is (t,y,x)=(0,0,0): sin terms 0, cos terms 1 in every chunk
@@ -69,7 +69,7 @@ def test_position_embedding_layout():
 
 
 def test_drift_magnitude():
-    w = synth.CONFIGS[1]
+    w = synth.workload("tiny")
     q1, _, _ = synth.head_tensors(w, 0, step=1)
     q2, _, _ = synth.head_tensors(w, 0, step=2)
     f = lambda u: (u.astype(np.uint32) << 16).view(np.float32).astype(np.float64)
@@ -78,9 +78,15 @@ def test_drift_magnitude():
 
 
 def test_random_metadata_valid():
-    w = synth.CONFIGS[1]
+    w = synth.workload("tiny")
     perm, kv, r = synth.random_metadata_head(w, 0)
     assert sorted(perm) == list(range(w.N))
     assert kv.shape == (w.n_groups, w.k)
     assert np.all(np.diff(kv, axis=1) > 0) and kv.min() >= 0 and kv.max() < w.N
     assert r.shape == (w.N, w.d) and r.dtype == np.float32
+
+
+def test_workloads_by_name_and_id_agree():
+    for wid, w in synth.WORKLOADS.items():
+        assert synth.workload(w.name) == w == synth.workload(wid)
+    assert synth.workload("video_long", k=100, G=64).k == 100
