@@ -51,3 +51,12 @@ def test_shape_change_makes_new_buffers_and_plans(monkeypatch):
     sch.step(2, *_qkv(2))
     assert sch.step(3, *_qkv(3))[1] == "plan"
     assert [c[0] for c in rec.calls if c[0] in ("ws", "meta")] == ["ws", "meta", "ws", "meta"]
+
+
+def test_fidelity_closed_forms():
+    D = torch.tensor([[[[3.0, 4.0], [0.0, 0.0]]]])          # ||D|| = 5
+    R = torch.tensor([[[[1.0, 0.0], [0.0, 2.0]]]])
+    O = (D + torch.tensor([[[[0.0, 0.5], [0.0, 0.0]]]])).to(torch.bfloat16)
+    rel, rel_nr = denoise.fidelity(O, D.to(torch.bfloat16), R)
+    assert abs(rel - 0.1) < 1e-12                            # ||(0, .5)|| / 5
+    assert abs(rel_nr - (0.25 + 1 + 4) ** 0.5 / 5) < 1e-12   # O - R - D = (-1, .5, 0, -2)
