@@ -28,7 +28,8 @@ softmax group, one O accumulator, and a CTA that loops over work items
 phases across items; the Q buffer is refilled for the next item once the
 current item's last Q.K^T has executed (a "Q empty" barrier), and the next
 item's first P.V, which overwrites O, must not run before the epilogue has
-read it.
+read it.  The third is the group-score kernel (colsum_kernel.cuh), whose
+reducing warps hand each S buffer back to the MMA thread explicitly.
 """
 import random
 
@@ -452,6 +453,141 @@ def test_sparse_model_catches_planted_defects(defect):
     for seed in range(200):
         try:
             run_sparse(3, 5, 3, 3, seed, defect=defect)
+        except ProtocolError:
+            failures += 1
+    assert failures > 0
+
+
+# ---------------------------------------------------------------------------
+# the group-score kernel: S buffers handed back by the reducing warps
+# ---------------------------------------------------------------------------
+
+class ColsumKernel:
+    def __init__(self, T, NST, defect=None):
+        self.T, self.NST = T, NST
+        self.q = Barrier(1)
+        self.kfull = [Barrier(1) for _ in range(NST)]
+        self.kempty = [Barrier(1) for _ in range(NST)]
+        self.sfull = [Barrier(1), Barrier(1)]
+        sfree = [Barrier(1), Barrier(1)]
+        self.sfree = [sfree[0], sfree[0]] if defect == "one_sfree" else sfree
+        self.sfree_off = 0 if defect == "sfree_parity" else 1
+        self.drain = Barrier(1)
+        self.kslot = [None] * NST
+        self.S = [None, None]            # ("S", j) written, ("read", j) reduced
+        self.qready = False
+        self.pipe, self.done, self.copies = [], set(), []
+
+    def step_pipe(self):
+        op = self.pipe.pop(0)
+        if op[0] == "commit":
+            op[1].arrive()
+            return
+        j = op[1]
+        s = j % self.NST
+        check(self.qready, "Q.K^T before Q landed")
+        check(self.kslot[s] == j, f"Q.K^T({j}) read a K slot holding {self.kslot[s]}")
+        prev = self.S[j & 1]
+        check(prev is None or prev == ("read", j - 2), f"Q.K^T({j}) overwrote S holding {prev}")
+        self.S[j & 1] = ("S", j)
+        self.done.add(("QK", j))
+
+    def step_copy(self, i):
+        kind, slot, tile, bar = self.copies.pop(i)
+        if kind == "K":
+            self.kslot[slot] = tile
+        else:
+            self.qready = True
+        bar.complete_tx(1)
+
+
+def colsum_producer(K):
+    yield from ()
+    K.q.arrive_expect_tx(1)
+    K.copies.append(("Q", 0, 0, K.q))
+    for j in range(K.T):
+        s = j % K.NST
+        if j >= K.NST:
+            t = j - K.NST
+            yield wait(K.kempty[s], ((j // K.NST) & 1) ^ 1, lambda t=t: ("QK", t) in K.done, f"K slot of tile {t} free")
+        K.kslot[s] = None
+        K.kfull[s].arrive_expect_tx(1)
+        K.copies.append(("K", s, j, K.kfull[s]))
+
+
+def colsum_mma(K):
+    yield wait(K.q, 0, lambda: K.qready, "Q landed")
+    for j in range(K.T):
+        s, b = j % K.NST, j & 1
+        if j >= 2:
+            yield wait(K.sfree[b], ((j >> 1) - K.sfree_off) & 1, lambda j=j: K.S[j & 1] == ("read", j - 2),
+                       f"S of tile {j - 2} reduced")
+        yield wait(K.kfull[s], (j // K.NST) & 1, lambda j=j, s=s: K.kslot[s] == j, f"K of tile {j} landed")
+        K.pipe += [("QK", j), ("commit", K.sfull[b]), ("commit", K.kempty[s])]
+    K.pipe.append(("commit", K.drain))
+    yield wait(K.drain, 0, lambda: not any(op[0] != "commit" for op in K.pipe), "pipe drained")
+
+
+def colsum_reducers(K):
+    for j in range(K.T):
+        b = j & 1
+        yield wait(K.sfull[b], (j >> 1) & 1, lambda j=j: K.S[j & 1] == ("S", j), f"S of tile {j}")
+        K.S[b] = ("read", j)
+        K.sfree[b].arrive()
+
+
+def run_colsum(T, NST, seed, defect=None, max_steps=200000):
+    rng = random.Random(seed)
+    K = ColsumKernel(T, NST, defect)
+    actors = {"k": colsum_producer(K), "mma": colsum_mma(K), "red": colsum_reducers(K)}
+    blocked = {name: None for name in actors}
+    finished = set()
+
+    def advance(name):
+        try:
+            blocked[name] = next(actors[name])
+        except StopIteration:
+            finished.add(name)
+            blocked[name] = None
+
+    for name in list(actors):
+        advance(name)
+    for _ in range(max_steps):
+        if len(finished) == len(actors):
+            return K
+        moves = [("actor", n) for n, w in blocked.items()
+                 if n not in finished and w is not None and w[0].parity_done(w[1])]
+        if K.pipe:
+            moves.append(("pipe", None))
+        moves += [("copy", i) for i in range(len(K.copies))]
+        if not moves:
+            raise ProtocolError(f"deadlock: waiting {[(n, w[3]) for n, w in blocked.items() if n not in finished]}")
+        kind, arg = rng.choice(moves)
+        if kind == "pipe":
+            K.step_pipe()
+        elif kind == "copy":
+            K.step_copy(arg)
+        else:
+            w = blocked[arg]
+            check(w[2](), f"{arg}: wait for '{w[3]}' returned before it happened")
+            advance(arg)
+    raise ProtocolError("schedule did not finish")
+
+
+@pytest.mark.parametrize("NST", [2, 4])
+@pytest.mark.parametrize("T", [1, 2, 3, 8, 17])
+def test_colsum_protocol_holds_under_random_schedules(T, NST):
+    for seed in range(60):
+        K = run_colsum(T, NST, seed)
+        assert {("QK", j) for j in range(T)} <= K.done
+
+
+@pytest.mark.parametrize("defect", ["one_sfree", "sfree_parity"])
+def test_colsum_model_catches_planted_defects(defect):
+    failures = 0
+    for seed in range(200):
+        try:
+            run_colsum(9, 2, seed, defect=defect)
         except ProtocolError:
             failures += 1
     assert failures > 0
