@@ -93,6 +93,26 @@ class Meta:
                     torch.empty((B, H, ng, k), dtype=torch.int32, device=device),
                     torch.empty((B, H, N, d), dtype=torch.float32, device=device))
 
+    def save(self, path) -> None:
+        """Write the cached metadata (the state a denoising loop reuses) to
+        `path` with torch.save; `Meta.load` restores it bit for bit."""
+        torch.save({"format": "mcs-meta-1", "sizes": [self.B, self.H, self.N, self.d, self.G, self.k,
+                                                      self.n_groups],
+                    "perm": self.perm.cpu(), "kv_idx": self.kv_idx.cpu(), "residual": self.residual.cpu()},
+                   path)
+
+    @staticmethod
+    def load(path, device="cuda") -> "Meta":
+        """Metadata written by `Meta.save`, on `device`."""
+        blob = torch.load(path, map_location="cpu", weights_only=True)
+        if blob.get("format") != "mcs-meta-1":
+            raise ValueError(f"{path}: not saved metadata")
+        B, H, N, d, G, k, ng = (int(x) for x in blob["sizes"])
+        meta = Meta(B, H, N, d, G, k, ng, blob["perm"].to(device).contiguous(),
+                    blob["kv_idx"].to(device).contiguous(), blob["residual"].to(device).contiguous())
+        _check_meta(meta, B, H, N, d, meta.perm.device)
+        return meta
+
     @staticmethod
     def from_tensors(perm, kv_idx, residual, G: int) -> "Meta":
         B, H, N, d = residual.shape

@@ -63,3 +63,27 @@ def test_output_buffers_are_checked():
             api._check_tensor(bad, "out", (1, 2, 8, 4), torch.bfloat16, CPU)
     with pytest.raises(TypeError):
         api._check_tensor(None, "out", (1,), torch.int32, CPU)
+
+
+def test_metadata_save_load_roundtrip(tmp_path):
+    """The cached metadata is the state a denoising loop resumes from: a save
+    and load gives back the same sizes and the same bits."""
+    m = _meta(N=100, k=10)
+    g = torch.Generator().manual_seed(0)
+    m.perm = torch.randperm(100, generator=g).to(torch.int32).repeat(1, 2, 1).contiguous()
+    m.kv_idx = torch.randint(0, 100, m.kv_idx.shape, generator=g, dtype=torch.int32)
+    m.residual = torch.randn(m.residual.shape, generator=g)
+    path = tmp_path / "meta.pt"
+    m.save(path)
+    r = api.Meta.load(path, device="cpu")
+    assert (r.B, r.H, r.N, r.d, r.G, r.k, r.n_groups) == (m.B, m.H, m.N, m.d, m.G, m.k, m.n_groups)
+    for name in ("perm", "kv_idx", "residual"):
+        a, b = getattr(m, name), getattr(r, name)
+        assert a.dtype == b.dtype and torch.equal(a.view(torch.int32), b.view(torch.int32))
+
+
+def test_metadata_load_refuses_other_files(tmp_path):
+    path = tmp_path / "other.pt"
+    torch.save({"x": torch.zeros(3)}, path)
+    with pytest.raises(ValueError):
+        api.Meta.load(path, device="cpu")

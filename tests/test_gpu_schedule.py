@@ -59,3 +59,17 @@ def test_schedule_reuses_buffers_and_replans_on_shape_change():
     torch.cuda.synchronize()
     assert k3 == "plan" and O3.shape[1] == 1
     assert mcs.last_device_status() == 0
+
+
+def test_saved_metadata_resumes_bit_for_bit(tmp_path):
+    """Checkpoint and resume of the cached state: a reused step on metadata
+    saved and loaded back equals the step on the original, bit for bit."""
+    w = synth.workload("tiny")
+    Q, K, V = (dev_bf16(x) for x in synth.layer_tensors(w))
+    meta = mcs.plan(Q, K, V, w.G, w.k)
+    O1 = mcs.sparse_step(Q, K, V, meta).clone()
+    meta.save(tmp_path / "meta.pt")
+    O2 = mcs.sparse_step(Q, K, V, mcs.Meta.load(tmp_path / "meta.pt"))
+    torch.cuda.synchronize()
+    assert mcs.last_device_status() == 0
+    assert torch.equal(O1.view(torch.int16), O2.view(torch.int16))
