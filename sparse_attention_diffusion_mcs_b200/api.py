@@ -30,6 +30,8 @@ def _check_qkv(*ts: torch.Tensor):
             raise ValueError("Q/K/V must be contiguous CUDA bf16 tensors [B, H, N, d]")
     if any(t.shape != ts[0].shape for t in ts):
         raise ValueError("Q/K/V shapes differ")
+    if any(t.device != ts[0].device for t in ts):
+        raise ValueError("Q/K/V are on different devices")
 
 
 def _check_tensor(t: torch.Tensor, name: str, shape, dtype, device):
