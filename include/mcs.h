@@ -40,7 +40,7 @@
 extern "C" {
 #endif
 
-#define MCS_ABI_VERSION 1
+#define MCS_ABI_VERSION 2
 
 typedef struct CUstream_st *mcs_stream_t; /* same type as cudaStream_t */
 
@@ -56,12 +56,24 @@ typedef enum {
 } mcs_status;
 
 /* Cached metadata of one plan ("query groups, KV indices ... and residuals",
- * aiqbench.com abstract).  All pointers are caller-owned device memory. */
+ * aiqbench.com abstract).  All pointers are caller-owned device memory.
+ *
+ * pair_idx / pair_len (optional, both or neither) are derived from kv_idx:
+ * for each pair p of adjacent groups (2p, 2p+1), the union of their kept
+ * keys, ordered [keys only 2p keeps | keys both keep | keys only 2p+1
+ * keeps], each segment ascending; pair_len[b,h,p] is the union's size u, so
+ * group 2p's keys are positions [0, k) and group 2p+1's are [u - k, u).  When
+ * the head has an odd number of groups the last pair is group 2p alone
+ * (u = k).  Adjacent groups hold similar queries (cctest.ai "Hardware-aware
+ * query organization") and keep mostly the same keys, so the reused step
+ * gathers each shared key once per pair.  n_pairs = ceil(n_groups / 2). */
 typedef struct {
   int32_t B, H, N, d, G, k, n_groups; /* k is stored clamped: k = min(k, N) */
   int32_t *perm;                      /* [B,H,N]                           */
   int32_t *kv_idx;                    /* [B,H,n_groups,k]                  */
   float *residual;                    /* [B,H,N,d]                         */
+  int32_t *pair_idx;                  /* [B,H,n_pairs,2k] or NULL          */
+  int32_t *pair_len;                  /* [B,H,n_pairs]    or NULL          */
 } mcs_meta;
 
 /* Library ABI version (MCS_ABI_VERSION of the build). */
@@ -95,7 +107,9 @@ size_t mcs_plan_workspace_size(int B, int H, int N, int d, int G, int k);
  * three failure modes, one fix"; cctest.ai design choices.
  *
  * meta: scalar fields are set by this call; meta->perm, ->kv_idx and
- *   ->residual must point to caller buffers of the sizes given above.
+ *   ->residual must point to caller buffers of the sizes given above; when
+ *   meta->pair_idx and ->pair_len are set, the pair union lists are built
+ *   into them as well (as mcs_meta_pairs does), else into the workspace.
  * O_dense: optional bf16 [B,H,N,d] output of the dense attention of this step
  *   (what a plan step of the denoising loop produces); may be NULL.
  * workspace: >= mcs_plan_workspace_size(...) bytes of device memory.
@@ -103,6 +117,26 @@ size_t mcs_plan_workspace_size(int B, int H, int N, int d, int G, int k);
 mcs_status mcs_plan(const void *Q, const void *K, const void *V, int B, int H, int N, int d,
                     int G, int k, float scale, mcs_meta *meta, void *O_dense, void *workspace,
                     size_t workspace_bytes, mcs_stream_t stream);
+
+/*
+ * Where mcs_plan_stats and mcs_plan_scores leave their results inside the
+ * workspace, as byte offsets from its start (any pointer argument may be
+ * NULL).  All float32, row-major:
+ *   row_m   [B,H,N]          m_i, a reference near max_j s_ij log2(e) (s_ij =
+ *                            scale Q_i.K_j): the softmax raises it only when
+ *                            a later key exceeds it by more than 32, so
+ *                            max_j s_ij log2(e) - 32 <= m_i <= max_j s_ij log2(e)
+ *   row_l   [B,H,N]          l_i = sum_j 2^(s_ij log2(e) - m_i)
+ *   O32     [B,H,N,d]        the dense output of the statistics pass
+ *   colsum  [B,H,n_groups,N] sum over group g's queries of P_ij
+ * m_i + log2(l_i) is the row's log2 normaliser whatever m_i is, and
+ * P_ij = 2^(s_ij log2(e) - m_i) / l_i are the exact probabilities of
+ * aiqbench.com's abstract; colsum holds the group sums the selection ranks.
+ * For inspection and tests; valid after the stage that writes them.
+ * INVALID_ARG for a shape mcs_plan_workspace_size rejects.
+ */
+mcs_status mcs_plan_workspace_offsets(int B, int H, int N, int d, int G, int k, size_t *row_m,
+                                      size_t *row_l, size_t *O32, size_t *colsum);
 
 /*
  * The plan's steps one by one.  mcs_plan is exactly mcs_plan_group,
@@ -148,11 +182,21 @@ mcs_status mcs_select_topk(const float *scores, int rows, int N, int k, int32_t 
                            mcs_stream_t stream);
 
 /* a5: residual float32 [B,H,N,d] = dense output (from mcs_plan_stats, same
- * Q, K, V) minus the output renormalised over each group's kept keys. */
+ * Q, K, V) minus the output renormalised over each group's kept keys.  Runs
+ * over pairs of groups; their union lists are built in the workspace. */
 mcs_status mcs_plan_residual(const void *Q, const void *K, const void *V, const int32_t *perm,
                              const int32_t *kv_idx, int B, int H, int N, int d, int G, int k,
                              float scale, float *residual, void *workspace,
                              size_t workspace_bytes, mcs_stream_t stream);
+
+/*
+ * mcs_meta_pairs -- build meta->pair_idx and meta->pair_len (layout above)
+ * from meta->kv_idx, e.g. for metadata made or loaded outside mcs_plan.
+ * kv_idx must hold ascending unique lists (as mcs_plan writes them); other
+ * input gives wrong lists but no out-of-bounds access.  Asynchronous.
+ * INVALID_ARG for a null pointer or inconsistent sizes.
+ */
+mcs_status mcs_meta_pairs(const mcs_meta *meta, mcs_stream_t stream);
 
 /*
  * mcs_sparse_step -- step a6, the reused denoising step: for every group g,
@@ -160,7 +204,12 @@ mcs_status mcs_plan_residual(const void *Q, const void *K, const void *V, const 
  * on the current step's Q, K, V with the cached groups, indices and residual
  * (aiqbench.com abstract: metadata "reused across subsequent denoising
  * steps"; cnshai.top section "MC-Sparse: three failure modes, one fix").
- * O: bf16 [B,H,N,d], original token order.  Needs no workspace.
+ * O: bf16 [B,H,N,d], original token order.  Needs no workspace.  With
+ * meta->pair_idx / ->pair_len set it runs over pairs of groups sharing one
+ * gathered key list (the same result up to fp32 summation order); without
+ * them, one group at a time.  A pair_len outside [k, 2k] or an index outside
+ * [0, N) is never read past or gathered: it records MCS_ERR_BAD_META in the
+ * device status word.
  */
 mcs_status mcs_sparse_step(const void *Q, const void *K, const void *V, const mcs_meta *meta,
                            float scale, void *O, mcs_stream_t stream);
@@ -179,9 +228,11 @@ size_t mcs_validate_workspace_size(int B, int H, int N);
 /*
  * Check cached metadata on the device: perm is a permutation per head,
  * kv_idx entries are in [0, N) and strictly ascending per group, the
- * residual is finite.  Synchronous: waits for `stream`.  Returns MCS_OK or
- * MCS_ERR_BAD_META; *first_bad (may be NULL) receives a code of the first
- * failed check: 1 perm, 2 kv_idx range, 3 kv_idx order, 4 residual.
+ * residual is finite, and (when present) every pair_len lies in [k, 2k]
+ * (exactly k for a lone last group) with its list's entries in [0, N).
+ * Synchronous: waits for `stream`.  Returns MCS_OK or MCS_ERR_BAD_META;
+ * *first_bad (may be NULL) receives a code of the first failed check:
+ * 1 perm, 2 kv_idx range, 3 kv_idx order, 4 residual, 5 pair lists.
  * Never traps.
  */
 mcs_status mcs_validate_meta(const mcs_meta *meta, void *workspace, size_t workspace_bytes,
@@ -191,10 +242,10 @@ mcs_status mcs_validate_meta(const mcs_meta *meta, void *workspace, size_t works
  * mcs_validate_meta_noalloc -- the same checks as mcs_validate_meta, for
  * callers that cannot hand over a device workspace.  The pages describe no
  * such call; it exists for users of this library whose code may not call
- * cudaMalloc at the point of the check: code recorded into a CUDA graph
- * capture (allocation is not a capturable operation), runtimes that forbid
- * allocation after start-up, and plugins that only receive raw pointers from
- * a host framework that owns all device memory.
+ * cudaMalloc at the point of the check: runtimes that forbid device
+ * allocation after start-up (a serving process that reserves all memory at
+ * launch), and plugins that only receive raw pointers from a host framework
+ * that owns all device memory and its allocator.
  *
  * Scratch: a fixed array compiled into the library, one per device that
  * loads it, held until the process exits: 256 bytes + one bit per token,

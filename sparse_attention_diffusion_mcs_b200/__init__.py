@@ -22,5 +22,6 @@ from .api import (  # noqa: F401
     sparse_step,
     validate_meta,
     workspace_size,
+    workspace_views,
 )
 from .denoise import Schedule, fidelity  # noqa: F401,E402

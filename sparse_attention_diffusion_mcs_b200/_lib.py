@@ -27,7 +27,8 @@ class McsMeta(ctypes.Structure):
     _fields_ = [("B", ctypes.c_int32), ("H", ctypes.c_int32), ("N", ctypes.c_int32),
                 ("d", ctypes.c_int32), ("G", ctypes.c_int32), ("k", ctypes.c_int32),
                 ("n_groups", ctypes.c_int32),
-                ("perm", c_vp), ("kv_idx", c_vp), ("residual", c_vp)]
+                ("perm", c_vp), ("kv_idx", c_vp), ("residual", c_vp),
+                ("pair_idx", c_vp), ("pair_len", c_vp)]
 
 
 PMETA = ctypes.POINTER(McsMeta)
@@ -39,6 +40,9 @@ PROTOTYPES = {
     "mcs_plan_workspace_size": (c_size_t, [c_int, c_int, c_int, c_int, c_int, c_int]),
     "mcs_plan": (c_int, [c_vp, c_vp, c_vp, c_int, c_int, c_int, c_int, c_int, c_int, c_float,
                          PMETA, c_vp, c_vp, c_size_t, c_vp]),
+    "mcs_plan_workspace_offsets": (c_int, [c_int, c_int, c_int, c_int, c_int, c_int,
+                                           ctypes.POINTER(c_size_t), ctypes.POINTER(c_size_t),
+                                           ctypes.POINTER(c_size_t), ctypes.POINTER(c_size_t)]),
     "mcs_plan_group": (c_int, [c_vp, c_int, c_int, c_int, c_int, c_vp, c_vp, c_size_t, c_vp]),
     "mcs_plan_stats": (c_int, [c_vp, c_vp, c_vp, c_int, c_int, c_int, c_int, c_int, c_int, c_float,
                                c_vp, c_vp, c_size_t, c_vp]),
@@ -48,6 +52,7 @@ PROTOTYPES = {
     "mcs_select_topk": (c_int, [c_vp, c_int, c_int, c_int, c_vp, c_vp]),
     "mcs_plan_residual": (c_int, [c_vp, c_vp, c_vp, c_vp, c_vp, c_int, c_int, c_int, c_int, c_int,
                                   c_int, c_float, c_vp, c_vp, c_size_t, c_vp]),
+    "mcs_meta_pairs": (c_int, [PMETA, c_vp]),
     "mcs_sparse_step": (c_int, [c_vp, c_vp, c_vp, PMETA, c_float, c_vp, c_vp]),
     "mcs_dense": (c_int, [c_vp, c_vp, c_vp, c_int, c_int, c_int, c_int, c_float, c_vp, c_vp]),
     "mcs_validate_workspace_size": (c_size_t, [c_int, c_int, c_int]),

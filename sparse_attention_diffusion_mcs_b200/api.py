@@ -2,7 +2,8 @@
 
 Argument marshalling only: every step of the hot path runs in the CUDA
 library.  Tensors must be CUDA, contiguous; Q/K/V/O are bf16 [B, H, N, d].
-Calls are asynchronous on torch's current stream.
+Each call makes the inputs' device current for its duration and runs
+asynchronously on torch's current stream of that device.
 """
 from __future__ import annotations
 
@@ -20,8 +21,14 @@ def _ptr(t: Optional[torch.Tensor]):
     return ctypes.c_void_p(t.data_ptr()) if t is not None else ctypes.c_void_p(0)
 
 
-def _stream():
-    return ctypes.c_void_p(torch.cuda.current_stream().cuda_stream)
+def _stream(device=None):
+    return ctypes.c_void_p(torch.cuda.current_stream(device).cuda_stream)
+
+
+def _on(device):
+    """The library resolves its status word, tensor maps and launches on the
+    CURRENT device, so every call runs with its tensors' device current."""
+    return torch.cuda.device(device)
 
 
 def _check_qkv(*ts: torch.Tensor):
@@ -62,6 +69,12 @@ def _check_meta(meta: "Meta", B: int, H: int, N: int, d: int, device, G: Optiona
     _check_tensor(meta.perm, "meta.perm", (B, H, N), torch.int32, device)
     _check_tensor(meta.kv_idx, "meta.kv_idx", (B, H, ng, meta.k), torch.int32, device)
     _check_tensor(meta.residual, "meta.residual", (B, H, N, d), torch.float32, device)
+    if (meta.pair_idx is None) != (meta.pair_len is None):
+        raise ValueError("meta.pair_idx and meta.pair_len come together")
+    if meta.pair_idx is not None:
+        npairs = (ng + 1) // 2
+        _check_tensor(meta.pair_idx, "meta.pair_idx", (B, H, npairs, 2 * meta.k), torch.int32, device)
+        _check_tensor(meta.pair_len, "meta.pair_len", (B, H, npairs), torch.int32, device)
 
 
 def _scale(d: int, scale: Optional[float]) -> float:
@@ -81,19 +94,50 @@ class Meta:
     perm: torch.Tensor       # int32 [B, H, N]
     kv_idx: torch.Tensor     # int32 [B, H, n_groups, k]
     residual: torch.Tensor   # float32 [B, H, N, d]
+    # union lists of adjacent group pairs, derived from kv_idx (include/mcs.h);
+    # None: the reused step runs one group at a time
+    pair_idx: Optional[torch.Tensor] = None   # int32 [B, H, n_pairs, 2k]
+    pair_len: Optional[torch.Tensor] = None   # int32 [B, H, n_pairs]
+
+    @property
+    def n_pairs(self) -> int:
+        return (self.n_groups + 1) // 2
 
     def c_struct(self) -> McsMeta:
         return McsMeta(self.B, self.H, self.N, self.d, self.G, self.k, self.n_groups,
-                       self.perm.data_ptr(), self.kv_idx.data_ptr(), self.residual.data_ptr())
+                       self.perm.data_ptr(), self.kv_idx.data_ptr(), self.residual.data_ptr(),
+                       self.pair_idx.data_ptr() if self.pair_idx is not None else 0,
+                       self.pair_len.data_ptr() if self.pair_len is not None else 0)
 
     @staticmethod
-    def empty(B: int, H: int, N: int, d: int, G: int, k: int, device="cuda") -> "Meta":
+    def empty(B: int, H: int, N: int, d: int, G: int, k: int, device="cuda", pairs: bool = True) -> "Meta":
         k = min(int(k), N)
         ng = -(-N // G)
+        np_ = (ng + 1) // 2
         return Meta(B, H, N, d, G, k, ng,
                     torch.empty((B, H, N), dtype=torch.int32, device=device),
                     torch.empty((B, H, ng, k), dtype=torch.int32, device=device),
-                    torch.empty((B, H, N, d), dtype=torch.float32, device=device))
+                    torch.empty((B, H, N, d), dtype=torch.float32, device=device),
+                    torch.empty((B, H, np_, 2 * k), dtype=torch.int32, device=device) if pairs else None,
+                    torch.empty((B, H, np_), dtype=torch.int32, device=device) if pairs else None)
+
+    def build_pairs(self) -> "Meta":
+        """(Re)build pair_idx / pair_len from kv_idx on the device (allocating
+        them when absent); returns self."""
+        dev = self.kv_idx.device
+        if self.pair_idx is None or self.pair_len is None:
+            self.pair_idx = torch.empty((self.B, self.H, self.n_pairs, 2 * self.k), dtype=torch.int32,
+                                        device=dev)
+            self.pair_len = torch.empty((self.B, self.H, self.n_pairs), dtype=torch.int32, device=dev)
+        _check_meta(self, self.B, self.H, self.N, self.d, dev)
+        cm = self.c_struct()
+        with _on(dev):
+            check(lib().mcs_meta_pairs(ctypes.byref(cm), _stream(dev)), "mcs_meta_pairs")
+        return self
+
+    def without_pairs(self) -> "Meta":
+        """The same metadata with no pair lists (one group at a time)."""
+        return dataclasses.replace(self, pair_idx=None, pair_len=None)
 
     def save(self, path) -> None:
         """Write the cached metadata (the state a denoising loop reuses) to
@@ -104,8 +148,9 @@ class Meta:
                    path)
 
     @staticmethod
-    def load(path, device="cuda") -> "Meta":
-        """Metadata written by `Meta.save`, on `device`."""
+    def load(path, device="cuda", pairs: bool = True) -> "Meta":
+        """Metadata written by `Meta.save`, on `device`; the pair lists (derived
+        data, not saved) are rebuilt from kv_idx on a CUDA device."""
         blob = torch.load(path, map_location="cpu", weights_only=True)
         if blob.get("format") != "mcs-meta-1":
             raise ValueError(f"{path}: not saved metadata")
@@ -113,14 +158,20 @@ class Meta:
         meta = Meta(B, H, N, d, G, k, ng, blob["perm"].to(device).contiguous(),
                     blob["kv_idx"].to(device).contiguous(), blob["residual"].to(device).contiguous())
         _check_meta(meta, B, H, N, d, meta.perm.device)
+        if pairs and meta.kv_idx.is_cuda:
+            meta.build_pairs()
         return meta
 
     @staticmethod
-    def from_tensors(perm, kv_idx, residual, G: int) -> "Meta":
+    def from_tensors(perm, kv_idx, residual, G: int, pairs: bool = True) -> "Meta":
+        """Metadata from caller tensors; with `pairs` (CUDA tensors) the pair
+        lists are built from kv_idx."""
         B, H, N, d = residual.shape
         ng, k = kv_idx.shape[2], kv_idx.shape[3]
-        return Meta(B, H, N, d, G, k, ng, perm.contiguous(), kv_idx.contiguous(),
-                    residual.contiguous())
+        meta = Meta(B, H, N, d, G, k, ng, perm.contiguous(), kv_idx.contiguous(), residual.contiguous())
+        if pairs and meta.kv_idx.is_cuda:
+            meta.build_pairs()
+        return meta
 
 
 def workspace_size(B: int, H: int, N: int, d: int, G: int, k: int) -> int:
@@ -133,6 +184,27 @@ def workspace_size(B: int, H: int, N: int, d: int, G: int, k: int) -> int:
 def alloc_workspace(B: int, H: int, N: int, d: int, G: int, k: int, device="cuda") -> torch.Tensor:
     # torch's caching allocator returns 512-byte aligned blocks
     return torch.empty(workspace_size(B, H, N, d, G, k), dtype=torch.uint8, device=device)
+
+
+def workspace_views(workspace: torch.Tensor, B: int, H: int, N: int, d: int, G: int, k: int):
+    """Views of the plan workspace's statistics and group scores (no copies):
+    {"row_m": [B,H,N] (log2 units), "row_l": [B,H,N], "O32": [B,H,N,d],
+    "colsum": [B,H,n_groups,N]}, all float32 (layout in include/mcs.h)."""
+    offs = [ctypes.c_size_t(0) for _ in range(4)]
+    check(lib().mcs_plan_workspace_offsets(B, H, N, d, G, k, *[ctypes.byref(o) for o in offs]),
+          "mcs_plan_workspace_offsets")
+    ng = -(-N // G)
+    shapes = {"row_m": (B, H, N), "row_l": (B, H, N), "O32": (B, H, N, d), "colsum": (B, H, ng, N)}
+    out = {}
+    for (name, shape), off in zip(shapes.items(), offs):
+        n = 1
+        for x in shape:
+            n *= x
+        start = int(off.value)
+        if start + 4 * n > workspace.numel():
+            raise ValueError("workspace smaller than the layout needs")
+        out[name] = workspace[start:start + 4 * n].view(torch.float32).view(shape)
+    return out
 
 
 def _ws(ws: Optional[torch.Tensor], B, H, N, d, G, k, device):
@@ -157,9 +229,10 @@ def plan(Q, K, V, G: int, k: int, scale: Optional[float] = None,
         out_dense = torch.empty_like(Q)
     ws = _ws(workspace, B, H, N, d, G, k, Q.device)
     cm = meta.c_struct()
-    check(lib().mcs_plan(_ptr(Q), _ptr(K), _ptr(V), B, H, N, d, G, k, _scale(d, scale),
-                         ctypes.byref(cm), _ptr(out_dense), _ptr(ws), ws.numel(), _stream()),
-          "mcs_plan")
+    with _on(Q.device):
+        check(lib().mcs_plan(_ptr(Q), _ptr(K), _ptr(V), B, H, N, d, G, k, _scale(d, scale),
+                             ctypes.byref(cm), _ptr(out_dense), _ptr(ws), ws.numel(), _stream(Q.device)),
+              "mcs_plan")
     meta.k, meta.n_groups = cm.k, cm.n_groups
     return (meta, out_dense) if (return_dense or out_dense is not None) else meta
 
@@ -173,8 +246,9 @@ def plan_group(Q, workspace: Optional[torch.Tensor] = None,
         _check_tensor(out, "out", (B, H, N), torch.int32, Q.device)
     perm = out if out is not None else torch.empty((B, H, N), dtype=torch.int32, device=Q.device)
     ws = _ws(workspace, B, H, N, d, 128, 1, Q.device)
-    check(lib().mcs_plan_group(_ptr(Q), B, H, N, d, _ptr(perm), _ptr(ws), ws.numel(), _stream()),
-          "mcs_plan_group")
+    with _on(Q.device):
+        check(lib().mcs_plan_group(_ptr(Q), B, H, N, d, _ptr(perm), _ptr(ws), ws.numel(), _stream(Q.device)),
+              "mcs_plan_group")
     return perm
 
 
@@ -189,8 +263,9 @@ def plan_stats(Q, K, V, G: int, k: int, scale: Optional[float] = None,
     if out_dense is not None:
         _check_tensor(out_dense, "out_dense", Q.shape, torch.bfloat16, Q.device)
     od = out_dense if out_dense is not None else (torch.empty_like(Q) if return_dense else None)
-    check(lib().mcs_plan_stats(_ptr(Q), _ptr(K), _ptr(V), B, H, N, d, G, k, _scale(d, scale), _ptr(od),
-                               _ptr(ws), ws.numel(), _stream()), "mcs_plan_stats")
+    with _on(Q.device):
+        check(lib().mcs_plan_stats(_ptr(Q), _ptr(K), _ptr(V), B, H, N, d, G, k, _scale(d, scale), _ptr(od),
+                                   _ptr(ws), ws.numel(), _stream(Q.device)), "mcs_plan_stats")
     return (ws, od) if (return_dense or out_dense is not None) else ws
 
 
@@ -201,8 +276,10 @@ def plan_scores(Q, K, perm, G: int, k: int, workspace: torch.Tensor,
     B, H, N, d = Q.shape
     perm = perm.to(torch.int32).contiguous()
     _check_tensor(perm, "perm", (B, H, N), torch.int32, Q.device)
-    check(lib().mcs_plan_scores(_ptr(Q), _ptr(K), _ptr(perm), B, H, N, d, G, k, _scale(d, scale),
-                                _ptr(workspace), workspace.numel(), _stream()), "mcs_plan_scores")
+    _check_tensor(workspace, "workspace", (workspace.numel(),), torch.uint8, Q.device)
+    with _on(Q.device):
+        check(lib().mcs_plan_scores(_ptr(Q), _ptr(K), _ptr(perm), B, H, N, d, G, k, _scale(d, scale),
+                                    _ptr(workspace), workspace.numel(), _stream(Q.device)), "mcs_plan_scores")
 
 
 def plan_topk(B: int, H: int, N: int, d: int, G: int, k: int, workspace: torch.Tensor,
@@ -213,8 +290,9 @@ def plan_topk(B: int, H: int, N: int, d: int, G: int, k: int, workspace: torch.T
         out = torch.empty((B, H, -(-N // G), kk), dtype=torch.int32, device=workspace.device)
     else:
         _check_tensor(out, "out", (B, H, -(-N // G), kk), torch.int32, workspace.device)
-    check(lib().mcs_plan_topk(B, H, N, d, G, k, _ptr(out), _ptr(workspace), workspace.numel(),
-                              _stream()), "mcs_plan_topk")
+    with _on(workspace.device):
+        check(lib().mcs_plan_topk(B, H, N, d, G, k, _ptr(out), _ptr(workspace), workspace.numel(),
+                                  _stream(workspace.device)), "mcs_plan_topk")
     return out
 
 
@@ -233,15 +311,18 @@ def select_topk(scores: torch.Tensor, k: int, out: Optional[torch.Tensor] = None
         _check_tensor(out, "out", (*scores.shape[:-1], kk), torch.int32, scores.device)
     if rows == 0:
         return out
-    check(lib().mcs_select_topk(_ptr(scores), rows, N, int(k), _ptr(out), _stream()), "mcs_select_topk")
+    with _on(scores.device):
+        check(lib().mcs_select_topk(_ptr(scores), rows, N, int(k), _ptr(out), _stream(scores.device)),
+              "mcs_select_topk")
     return out
 
 
-def plan_select(Q, K, perm, G: int, k: int, scale: Optional[float] = None,
+def plan_select(Q, K, V, perm, G: int, k: int, scale: Optional[float] = None,
                 workspace: Optional[torch.Tensor] = None) -> torch.Tensor:
-    """Steps a2-a4 for a given grouping: int32 kv_idx [B, H, n_groups, min(k, N)]."""
+    """Steps a2-a4 for a given grouping: int32 kv_idx [B, H, n_groups, min(k, N)].
+    (a2 also leaves the dense output of Q, K, V in the workspace.)"""
     B, H, N, d = Q.shape
-    ws = plan_stats(Q, K, K, G, k, scale, workspace)
+    ws = plan_stats(Q, K, V, G, k, scale, workspace)
     plan_scores(Q, K, perm, G, k, ws, scale)
     return plan_topk(B, H, N, d, G, k, ws)
 
@@ -269,9 +350,11 @@ def plan_residual(Q, K, V, perm, kv_idx, G: int, scale: Optional[float] = None,
     else:
         ws = plan_stats(Q, K, V, G, k, scale, workspace)
     res = out if out is not None else torch.empty((B, H, N, d), dtype=torch.float32, device=Q.device)
-    check(lib().mcs_plan_residual(_ptr(Q), _ptr(K), _ptr(V), _ptr(perm), _ptr(kv_idx), B, H, N, d,
-                                  G, k, _scale(d, scale), _ptr(res), _ptr(ws), ws.numel(), _stream()),
-          "mcs_plan_residual")
+    with _on(Q.device):
+        check(lib().mcs_plan_residual(_ptr(Q), _ptr(K), _ptr(V), _ptr(perm), _ptr(kv_idx), B, H, N, d,
+                                      G, k, _scale(d, scale), _ptr(res), _ptr(ws), ws.numel(),
+                                      _stream(Q.device)),
+              "mcs_plan_residual")
     return (res, od) if return_dense else res
 
 
@@ -285,8 +368,9 @@ def sparse_step(Q, K, V, meta: Meta, scale: Optional[float] = None,
     else:
         _check_tensor(out, "out", Q.shape, torch.bfloat16, Q.device)
     cm = meta.c_struct()
-    check(lib().mcs_sparse_step(_ptr(Q), _ptr(K), _ptr(V), ctypes.byref(cm),
-                                _scale(meta.d, scale), _ptr(out), _stream()), "mcs_sparse_step")
+    with _on(Q.device):
+        check(lib().mcs_sparse_step(_ptr(Q), _ptr(K), _ptr(V), ctypes.byref(cm),
+                                    _scale(meta.d, scale), _ptr(out), _stream(Q.device)), "mcs_sparse_step")
     return out
 
 
@@ -298,26 +382,33 @@ def dense(Q, K, V, scale: Optional[float] = None, out: Optional[torch.Tensor] = 
         out = torch.empty_like(Q)
     else:
         _check_tensor(out, "out", Q.shape, torch.bfloat16, Q.device)
-    check(lib().mcs_dense(_ptr(Q), _ptr(K), _ptr(V), B, H, N, d, _scale(d, scale), _ptr(out),
-                          _stream()), "mcs_dense")
+    with _on(Q.device):
+        check(lib().mcs_dense(_ptr(Q), _ptr(K), _ptr(V), B, H, N, d, _scale(d, scale), _ptr(out),
+                              _stream(Q.device)), "mcs_dense")
     return out
 
 
 def validate_meta(meta: Meta) -> Tuple[bool, int]:
     """(valid, first failing check code); synchronous."""
+    dev = meta.perm.device
+    _check_meta(meta, meta.B, meta.H, meta.N, meta.d, dev)
     n = lib().mcs_validate_workspace_size(meta.B, meta.H, meta.N)
-    ws = torch.empty(int(n), dtype=torch.uint8, device=meta.perm.device)
+    ws = torch.empty(int(n), dtype=torch.uint8, device=dev)
     code = ctypes.c_int(0)
     cm = meta.c_struct()
-    st = lib().mcs_validate_meta(ctypes.byref(cm), _ptr(ws), ws.numel(), ctypes.byref(code), _stream())
+    with _on(dev):
+        st = lib().mcs_validate_meta(ctypes.byref(cm), _ptr(ws), ws.numel(), ctypes.byref(code), _stream(dev))
     if st == 6:
         return False, code.value
     check(st, "mcs_validate_meta")
     return True, 0
 
 
-def last_device_status() -> int:
-    return int(lib().mcs_last_device_status(_stream()))
+def last_device_status(device=None) -> int:
+    """Read and clear the status word of `device` (default: the current one)."""
+    dev = torch.device("cuda", torch.cuda.current_device()) if device is None else torch.device(device)
+    with _on(dev):
+        return int(lib().mcs_last_device_status(_stream(dev)))
 
 
 def set_wait_limit_ns(ns: int) -> None:
@@ -325,4 +416,4 @@ def set_wait_limit_ns(ns: int) -> None:
 
 
 def selftest_wait_timeout(limit_ns: int) -> None:
-    check(lib().mcs_selftest_wait_timeout(int(limit_ns), _stream()), "mcs_selftest_wait_timeout")
+    check(lib().mcs_selftest_wait_timeout(int(limit_ns), _stream(None)), "mcs_selftest_wait_timeout")

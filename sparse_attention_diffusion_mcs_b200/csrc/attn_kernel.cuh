@@ -64,6 +64,9 @@ struct alignas(64) AttnArgs {
   unsigned *status;        // device status word
   uint64_t wait_ns;        // bound on any single wait
   int BH;                  // heads; work items are (head, query tile or group) pairs
+  const int32_t *pair_idx; // [BH, n_pairs, 2k]     pair kernel: union list of groups 2p, 2p+1
+  const int32_t *pair_len; // [BH, n_pairs]         pair kernel: union sizes
+  int n_pairs;             // ceil(n_groups / 2)
 };
 
 template <int D, int MODE>

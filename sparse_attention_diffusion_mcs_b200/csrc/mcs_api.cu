@@ -12,6 +12,7 @@
 #include "attn_kernel.cuh"
 #include "colsum_kernel.cuh"
 #include "group_kernels.cuh"
+#include "pair_kernel.cuh"
 #include "topk_kernel.cuh"
 #include "validate_kernels.cuh"
 
@@ -152,6 +153,42 @@ cudaError_t launch_attn_d(int d, AttnArgs &a, const QKV &t, int grid_x, int BH, 
   return d == 64 ? launch_attn<64, MODE>(a, t, grid_x, BH, s) : launch_attn<128, MODE>(a, t, grid_x, BH, s);
 }
 
+// The sparse modes over pairs of groups sharing one union list of keys
+// (pair_kernel.cuh): persistent, one CTA per SM, items (head, pair).
+template <int D, int MODE>
+cudaError_t launch_pair(AttnArgs &a, const QKV &t, int BH, cudaStream_t s) {
+  using C = PairCfg<D>;
+  a.BH = BH;
+  const size_t rows = static_cast<size_t>(BH) * a.N;
+  if (!(map_gather(&a.tmQ, t.Q, D, rows) && map_gather(&a.tmK, t.K, D, rows) && map_gather(&a.tmV, t.V, D, rows)))
+    return cudaErrorInvalidValue;
+  const long items = static_cast<long>(BH) * a.n_pairs;
+  if (items == 0) return cudaSuccess;
+  cudaError_t e;
+  if ((e = set_smem(pair_kernel<D, MODE>, C::SMEM)) != cudaSuccess) return e;
+  int sms = 0;
+  if ((e = sm_count(&sms)) != cudaSuccess) return e;
+  const long grid = items < sms ? items : sms;
+  pair_kernel<D, MODE><<<static_cast<unsigned>(grid), C::THREADS, C::SMEM, s>>>(a);
+  return cudaGetLastError();
+}
+
+template <int MODE>
+cudaError_t launch_pair_d(int d, AttnArgs &a, const QKV &t, int BH, cudaStream_t s) {
+  return d == 64 ? launch_pair<64, MODE>(a, t, BH, s) : launch_pair<128, MODE>(a, t, BH, s);
+}
+
+inline int pairs_of(int n_groups) { return (n_groups + 1) / 2; }
+
+// union lists of group pairs (2p, 2p+1) from the groups' ascending kv lists
+cudaError_t run_pairs(const int32_t *kv_idx, int BH, int n_groups, int kk, int32_t *pair_idx,
+                      int32_t *pair_len, cudaStream_t s) {
+  const int np = pairs_of(n_groups);
+  if (np == 0 || BH == 0) return cudaSuccess;
+  pair_build_kernel<<<dim3(np, BH), kPairThreads, 0, s>>>(kv_idx, n_groups, kk, np, pair_idx, pair_len);
+  return cudaGetLastError();
+}
+
 AttnArgs base_args(int N, float scale) {
   AttnArgs a;
   std::memset(&a, 0, sizeof(a));
@@ -165,10 +202,10 @@ AttnArgs base_args(int N, float scale) {
 // ---------------------------------------------------------------- plan workspace
 struct PlanWs {
   size_t mean_part, mean, cov_part, cov64, vdir, lambda, keys0, vals0, keys1, vals1;
-  size_t row_m, row_l, O32, colsum, total;
+  size_t row_m, row_l, O32, colsum, pair_idx, pair_len, total;
 };
 
-PlanWs plan_ws(int B, int H, int N, int d, int G) {
+PlanWs plan_ws(int B, int H, int N, int d, int G, int k) {
   const size_t BH = static_cast<size_t>(B) * H;
   const size_t nch = (N + kGroupChunk - 1) / kGroupChunk;
   const size_t ng = (N + G - 1) / G;
@@ -193,6 +230,9 @@ PlanWs plan_ws(int B, int H, int N, int d, int G) {
   w.row_l = take(BH * N * 4);
   w.O32 = take(BH * N * static_cast<size_t>(d) * 4);
   w.colsum = take(BH * ng * static_cast<size_t>(N) * 4);
+  const size_t np = (ng + 1) / 2, kk = static_cast<size_t>(k < N ? k : N);
+  w.pair_idx = take(BH * np * 2 * kk * 4);   // union lists for the residual pass (stage entry)
+  w.pair_len = take(BH * np * 4);
   w.total = o;
   return w;
 }
@@ -293,18 +333,31 @@ cudaError_t run_topk(int BH, int N, int G, int k, int32_t *kv_idx, void *ws, con
   return launch_topk(at<float>(ws, w.colsum), BH * ng, N, k, kv_idx, s);
 }
 
+// a5 over pairs of groups: the union lists go to (pair_idx, pair_len), which
+// are the metadata's own lists or the workspace's scratch
 cudaError_t run_residual(const void *Q, const void *K, const void *V, const int32_t *perm,
                          const int32_t *kv_idx, int BH, int N, int d, int G, int k, float scale,
-                         float *residual, void *ws, const PlanWs &w, cudaStream_t s) {
+                         float *residual, void *ws, const PlanWs &w, int32_t *pair_idx, int32_t *pair_len,
+                         cudaStream_t s) {
+  const int ng = (N + G - 1) / G;
+  if (!pair_idx || !pair_len) {
+    pair_idx = at<int32_t>(ws, w.pair_idx);
+    pair_len = at<int32_t>(ws, w.pair_len);
+  }
+  cudaError_t e = run_pairs(kv_idx, BH, ng, k, pair_idx, pair_len, s);
+  if (e != cudaSuccess) return e;
   AttnArgs a = base_args(N, scale);
   a.G = G;
   a.k = k;
-  a.n_groups = (N + G - 1) / G;
+  a.n_groups = ng;
+  a.n_pairs = pairs_of(ng);
   a.perm = perm;
   a.kv_idx = kv_idx;
+  a.pair_idx = pair_idx;
+  a.pair_len = pair_len;
   a.O32_in = at<float>(ws, w.O32);
   a.R_out = residual;
-  return launch_attn_d<kModePlanResid>(d, a, QKV{Q, K, V}, a.n_groups, BH, s);
+  return launch_pair_d<kModePlanResid>(d, a, QKV{Q, K, V}, BH, s);
 }
 
 mcs_status check_common(const void *Q, const void *K, const void *V, int B, int H, int N, int d,
@@ -341,6 +394,16 @@ unsigned char *noalloc_scratch() {
     g_noalloc_ptr[dev] = static_cast<unsigned char *>(p);
   }
   return g_noalloc_ptr[dev];
+}
+
+// pair-list check of mcs_validate_meta(_noalloc), when the metadata has them
+void launch_pair_check(const mcs_meta *meta, int *bad, cudaStream_t s) {
+  if (!meta->pair_idx || !meta->pair_len) return;
+  const int np = pairs_of(meta->n_groups);
+  const size_t items = static_cast<size_t>(meta->B) * meta->H * np;
+  const unsigned grid = static_cast<unsigned>(items < 148 * 8 ? items : 148 * 8);
+  pair_check_kernel<<<grid, 256, 0, s>>>(meta->pair_idx, meta->pair_len, meta->N, meta->k, meta->n_groups, np,
+                                          items, bad);
 }
 
 }  // namespace
@@ -381,7 +444,18 @@ mcs_status mcs_meta_init(mcs_meta *meta, int B, int H, int N, int d, int G, int 
 
 size_t mcs_plan_workspace_size(int B, int H, int N, int d, int G, int k) {
   if (!shape_ok(B, H, N, d) || !d_ok(d) || !g_ok(G) || k < 1) return 0;
-  return plan_ws(B, H, N, d, G).total;
+  return plan_ws(B, H, N, d, G, k).total;
+}
+
+mcs_status mcs_plan_workspace_offsets(int B, int H, int N, int d, int G, int k, size_t *row_m, size_t *row_l,
+                                      size_t *O32, size_t *colsum) {
+  if (!shape_ok(B, H, N, d) || !d_ok(d) || !g_ok(G) || k < 1) return MCS_ERR_INVALID_ARG;
+  const PlanWs w = plan_ws(B, H, N, d, G, k);
+  if (row_m) *row_m = w.row_m;
+  if (row_l) *row_l = w.row_l;
+  if (O32) *O32 = w.O32;
+  if (colsum) *colsum = w.colsum;
+  return MCS_OK;
 }
 
 mcs_status mcs_plan_group(const void *Q, int B, int H, int N, int d, int32_t *perm, void *workspace,
@@ -389,7 +463,7 @@ mcs_status mcs_plan_group(const void *Q, int B, int H, int N, int d, int32_t *pe
   mcs_status st = check_common(Q, Q, Q, B, H, N, d, 1.f);
   if (st != MCS_OK) return st;
   if (!perm) return MCS_ERR_INVALID_ARG;
-  const PlanWs w = plan_ws(B, H, N, d, 128);
+  const PlanWs w = plan_ws(B, H, N, d, 128, 1);
   // grouping needs only the part of the workspace before the statistics
   if ((st = check_ws(workspace, workspace_bytes, w.row_m)) != MCS_OK) return st;
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
@@ -405,7 +479,7 @@ mcs_status mcs_plan_stats(const void *Q, const void *K, const void *V, int B, in
   if (st != MCS_OK) return st;
   if (k < 1 || (O_dense && !aligned16(O_dense))) return MCS_ERR_INVALID_ARG;
   if (!g_ok(G)) return MCS_ERR_UNSUPPORTED;
-  const PlanWs w = plan_ws(B, H, N, d, G);
+  const PlanWs w = plan_ws(B, H, N, d, G, k);
   if ((st = check_ws(workspace, workspace_bytes, w.total)) != MCS_OK) return st;
   return cuda_status(run_plan_dense(Q, K, V, B * H, N, d, scale, O_dense, workspace, w,
                                     reinterpret_cast<cudaStream_t>(stream)));
@@ -418,7 +492,7 @@ mcs_status mcs_plan_scores(const void *Q, const void *K, const int32_t *perm, in
   if (st != MCS_OK) return st;
   if (!perm || k < 1) return MCS_ERR_INVALID_ARG;
   if (!g_ok(G)) return MCS_ERR_UNSUPPORTED;
-  const PlanWs w = plan_ws(B, H, N, d, G);
+  const PlanWs w = plan_ws(B, H, N, d, G, k);
   if ((st = check_ws(workspace, workspace_bytes, w.total)) != MCS_OK) return st;
   return cuda_status(run_scores(Q, K, perm, B * H, N, d, G, scale, workspace, w,
                                 reinterpret_cast<cudaStream_t>(stream)));
@@ -428,7 +502,7 @@ mcs_status mcs_plan_topk(int B, int H, int N, int d, int G, int k, int32_t *kv_i
                          size_t workspace_bytes, mcs_stream_t stream) {
   if (!shape_ok(B, H, N, d) || !kv_idx || k < 1) return MCS_ERR_INVALID_ARG;
   if (!d_ok(d) || !g_ok(G)) return MCS_ERR_UNSUPPORTED;
-  const PlanWs w = plan_ws(B, H, N, d, G);
+  const PlanWs w = plan_ws(B, H, N, d, G, k);
   mcs_status st = check_ws(workspace, workspace_bytes, w.total);
   if (st != MCS_OK) return st;
   return cuda_status(run_topk(B * H, N, G, k < N ? k : N, kv_idx, workspace, w,
@@ -449,10 +523,10 @@ mcs_status mcs_plan_residual(const void *Q, const void *K, const void *V, const 
   if (st != MCS_OK) return st;
   if (!perm || !kv_idx || !residual || k < 1 || !aligned16(residual)) return MCS_ERR_INVALID_ARG;
   if (!g_ok(G)) return MCS_ERR_UNSUPPORTED;
-  const PlanWs w = plan_ws(B, H, N, d, G);
+  const PlanWs w = plan_ws(B, H, N, d, G, k);
   if ((st = check_ws(workspace, workspace_bytes, w.total)) != MCS_OK) return st;
   return cuda_status(run_residual(Q, K, V, perm, kv_idx, B * H, N, d, G, k < N ? k : N, scale, residual,
-                                  workspace, w, reinterpret_cast<cudaStream_t>(stream)));
+                                  workspace, w, nullptr, nullptr, reinterpret_cast<cudaStream_t>(stream)));
 }
 
 mcs_status mcs_plan(const void *Q, const void *K, const void *V, int B, int H, int N, int d, int G, int k,
@@ -463,7 +537,7 @@ mcs_status mcs_plan(const void *Q, const void *K, const void *V, int B, int H, i
   if (!meta || !meta->perm || !meta->kv_idx || !meta->residual) return MCS_ERR_INVALID_ARG;
   if (!aligned16(meta->residual) || (O_dense && !aligned16(O_dense))) return MCS_ERR_INVALID_ARG;
   if ((st = mcs_meta_init(meta, B, H, N, d, G, k)) != MCS_OK) return st;
-  const PlanWs w = plan_ws(B, H, N, d, G);
+  const PlanWs w = plan_ws(B, H, N, d, G, k);
   if ((st = check_ws(workspace, workspace_bytes, w.total)) != MCS_OK) return st;
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
   const int BH = B * H;
@@ -474,8 +548,18 @@ mcs_status mcs_plan(const void *Q, const void *K, const void *V, int B, int H, i
   if (e == cudaSuccess) e = run_topk(BH, N, G, meta->k, meta->kv_idx, workspace, w, s);
   if (e == cudaSuccess)
     e = run_residual(Q, K, V, meta->perm, meta->kv_idx, BH, N, d, G, meta->k, scale, meta->residual,
-                     workspace, w, s);
+                     workspace, w, meta->pair_idx, meta->pair_len, s);
   return cuda_status(e);
+}
+
+mcs_status mcs_meta_pairs(const mcs_meta *meta, mcs_stream_t stream) {
+  if (!meta || !meta->kv_idx || !meta->pair_idx || !meta->pair_len) return MCS_ERR_INVALID_ARG;
+  if (!shape_ok(meta->B, meta->H, meta->N, meta->d) || !d_ok(meta->d) || !g_ok(meta->G))
+    return MCS_ERR_INVALID_ARG;
+  if (meta->k < 1 || meta->k > meta->N || meta->n_groups != (meta->N + meta->G - 1) / meta->G)
+    return MCS_ERR_INVALID_ARG;
+  return cuda_status(run_pairs(meta->kv_idx, meta->B * meta->H, meta->n_groups, meta->k, meta->pair_idx,
+                               meta->pair_len, reinterpret_cast<cudaStream_t>(stream)));
 }
 
 mcs_status mcs_sparse_step(const void *Q, const void *K, const void *V, const mcs_meta *meta, float scale,
@@ -497,6 +581,12 @@ mcs_status mcs_sparse_step(const void *Q, const void *K, const void *V, const mc
   a.residual = meta->residual;
   a.O = static_cast<bf16 *>(O);
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  if (meta->pair_idx && meta->pair_len) {
+    a.n_pairs = pairs_of(meta->n_groups);
+    a.pair_idx = meta->pair_idx;
+    a.pair_len = meta->pair_len;
+    return cuda_status(launch_pair_d<kModeStep>(meta->d, a, QKV{Q, K, V}, meta->B * meta->H, s));
+  }
   return cuda_status(launch_attn_d<kModeStep>(meta->d, a, QKV{Q, K, V}, meta->n_groups, meta->B * meta->H, s));
 }
 
@@ -542,6 +632,7 @@ mcs_status mcs_validate_meta(const mcs_meta *meta, void *workspace, size_t works
                                        static_cast<size_t>(BH) * meta->n_groups, bad);
   residual_check_kernel<<<grid, 256, 0, s>>>(meta->residual,
                                              static_cast<size_t>(BH) * meta->N * meta->d, bad);
+  launch_pair_check(meta, bad, s);
   if (cudaGetLastError() != cudaSuccess) return MCS_ERR_CUDA;
   int h = INT_MAX;
   e = cudaMemcpyAsync(&h, bad, sizeof(int), cudaMemcpyDeviceToHost, s);
@@ -578,6 +669,7 @@ mcs_status mcs_validate_meta_noalloc(const mcs_meta *meta, int *first_bad, mcs_s
   kv_check_kernel<<<grid, 256, 0, s>>>(meta->kv_idx, meta->N, meta->k,
                                        static_cast<size_t>(BH) * meta->n_groups, bad);
   residual_check_kernel<<<grid, 256, 0, s>>>(meta->residual, tokens * meta->d, bad);
+  launch_pair_check(meta, bad, s);
   if (cudaGetLastError() != cudaSuccess) return MCS_ERR_CUDA;
   int h = INT_MAX;
   e = cudaMemcpyAsync(&h, bad, sizeof(int), cudaMemcpyDeviceToHost, s);

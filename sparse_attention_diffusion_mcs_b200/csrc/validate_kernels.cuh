@@ -45,6 +45,26 @@ __global__ void residual_check_kernel(const float *__restrict__ r, size_t n, int
   }
 }
 
+// Pair union lists (pair_kernel.cuh): every length in [k, 2k] (exactly k for
+// a lone last group) and every listed entry in [0, N); else code 5.
+__global__ void pair_check_kernel(const int32_t *__restrict__ pair_idx, const int32_t *__restrict__ pair_len,
+                                  int N, int kk, int n_groups, int n_pairs, size_t items, int *__restrict__ bad) {
+  for (size_t it = blockIdx.x; it < items; it += gridDim.x) {
+    const int p = static_cast<int>(it % n_pairs);
+    const int umax = 2 * p + 1 < n_groups ? 2 * kk : kk;
+    const int u = pair_len[it];
+    if (u < kk || u > umax) {
+      if (threadIdx.x == 0) atomicMin(bad, 5);
+      continue;
+    }
+    const int32_t *L = pair_idx + it * 2 * static_cast<size_t>(kk);
+    for (int i = threadIdx.x; i < u; i += blockDim.x) {
+      const int v = L[i];
+      if (v < 0 || v >= N) atomicMin(bad, 5);
+    }
+  }
+}
+
 // Waits on an mbarrier that nothing ever arrives on.  The bounded wait gives
 // up after limit_ns and records the timeout in the status word; the kernel
 // then returns normally.

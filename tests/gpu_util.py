@@ -8,6 +8,18 @@ OUT_MAX_ABS = 2e-2
 OUT_REL_L2 = 1e-2
 RES_REL_L2 = 1e-3
 KV_THRESHOLD_REL = 1e-4
+# Plan statistics (a2) and group scores (a3), read from the plan workspace.
+# s_ij comes out of fp32 tensor-core accumulation of exact bf16 products, and
+# l_i is an fp32 sum of N terms; rounding in both behaves like sqrt(N) * 2^-24
+# (about 1e-5 for N up to 131072), so the row's log normaliser m + log l
+# (natural units) is held to 2e-4 absolute.  Each group score is a sum of G
+# probabilities each carrying that relative error plus ex2.approx's 2^-22, so
+# it is held to 1e-4 relative -- the same margin the KV-set rule grants at
+# the k-th score -- plus an absolute floor for terms below fp32's smallest
+# normal value, which the kernels flush to zero (at most G * 2^-126 per score).
+LSE_ABS = 2e-4
+COLSUM_REL = 1e-4
+COLSUM_ABS = 128 * 2.0 ** -126
 
 
 def dev_bf16(u16: np.ndarray) -> torch.Tensor:

@@ -38,8 +38,26 @@ def test_every_declared_symbol_is_exported_and_bound(L):
     assert set(_lib.PROTOTYPES) == set(names)
 
 
+def test_micro_library_exports_its_header():
+    """libmcs_micro.so (include/mcs_micro.h) loads without a GPU, exports what
+    its header declares, and refuses bad arguments before any launch."""
+    from sparse_attention_diffusion_mcs_b200 import micro
+    _build.build()
+    text = re.sub(r"/\*.*?\*/", "", open(os.path.join(ROOT, "include", "mcs_micro.h")).read(), flags=re.S)
+    names = sorted(set(re.findall(r"\b(mcs_[a-z_0-9]+)\s*\(", text)))
+    M = micro.lib()
+    assert set(names) == set(micro.PROTOTYPES)
+    for n in names:
+        assert hasattr(M, n), n
+    assert M.mcs_micro_gather(None, 1024, FAKE, 1, 1, 0, 1, None) == INVALID
+    assert M.mcs_micro_gather(FAKE, 64, FAKE, 1, 1, 0, 1, None) == INVALID        # fewer rows than a tile
+    assert M.mcs_micro_gather(FAKE, 1024, FAKE, 1, 1, 0, 9, None) == INVALID      # more than 8 warps
+    assert M.mcs_micro_gather(FAKE, 1024, FAKE, 1, 1, 3, 1, None) == INVALID      # no such mode
+    assert M.mcs_micro_gather(FAKE + 8, 1024, FAKE, 1, 1, 0, 1, None) == INVALID  # misaligned source
+
+
 def test_version_and_status_strings(L):
-    assert L.mcs_abi_version() == 1
+    assert L.mcs_abi_version() == 2
     for code, name in _lib.STATUS_NAMES.items():
         assert L.mcs_status_string(code).decode() == name
 

@@ -12,8 +12,8 @@ import torch
 import sparse_attention_diffusion_mcs_b200 as mcs
 import synth
 from oracle import mcs_oracle as orc
-from tests.gpu_util import (assert_out_close, assert_residual_close, dev_bf16, host,
-                            kv_sets_agree)
+from tests.gpu_util import (COLSUM_ABS, COLSUM_REL, LSE_ABS, assert_out_close, assert_residual_close,
+                            dev_bf16, host, kv_sets_agree)
 
 pytestmark = pytest.mark.gpu
 
@@ -157,9 +157,10 @@ def test_plan_group_matches_oracle_order(cfg_or_shape):
 @pytest.mark.parametrize("cfg,G,k", [(1, 64, 128), (1, 128, 300), (1, 64, 1), (1, 128, 1024)])
 def test_plan_select_on_oracle_grouping(cfg, G, k):
     w = synth.workload(cfg, G=G, k=k)
-    Q, K, _ = synth.layer_tensors(w)
+    Q, K, V = synth.layer_tensors(w)
     perms = np.stack([orc.group_queries(Q[0, h]) for h in range(w.H)]).astype(np.int32)[None]
-    kv = mcs.plan_select(dev_bf16(Q), dev_bf16(K), torch.from_numpy(perms).cuda(), G, k).cpu().numpy()
+    kv = mcs.plan_select(dev_bf16(Q), dev_bf16(K), dev_bf16(V), torch.from_numpy(perms).cuda(), G,
+                         k).cpu().numpy()
     torch.cuda.synchronize()
     assert mcs.last_device_status() == 0
     assert kv.shape == (1, w.H, w.n_groups, min(k, w.N))
@@ -216,33 +217,98 @@ def test_plan_residual_on_oracle_metadata(cfg, G, k):
 
 @pytest.mark.parametrize("cfg,G,k", [(1, 64, 128), (1, 128, 77)])
 def test_plan_end_to_end(cfg, G, k):
+    """The whole plan, then the comparison protocol: perm equal to the
+    oracle's; every group's KV set within the 1e-4 band of the oracle's
+    scores; then the residual of EVERY group recomputed by the oracle on the
+    GPU's own selection; the dense output; and a reused step on the plan's
+    own inputs, which must reproduce dense attention."""
     w = synth.workload(cfg, G=G, k=k)
     Q, K, V = synth.layer_tensors(w)
     q, kd, v = dev_bf16(Q), dev_bf16(K), dev_bf16(V)
-    meta, od = mcs.plan(q, kd, v, G, k, return_dense=True)
+    ws = mcs.alloc_workspace(w.B, w.H, w.N, w.d, G, k, q.device)
+    meta, od = mcs.plan(q, kd, v, G, k, workspace=ws, return_dense=True)
     o_step = host(mcs.sparse_step(q, kd, v, meta))
     torch.cuda.synchronize()
     assert mcs.last_device_status() == 0
     ok, code = mcs.validate_meta(meta)
     assert ok, code
+    views = mcs.workspace_views(ws, w.B, w.H, w.N, w.d, G, k)
     perm = meta.perm.cpu().numpy()
     kv = meta.kv_idx.cpu().numpy()
     res = meta.residual.cpu().numpy().astype(np.float64)
+    cs = views["colsum"].cpu().numpy().astype(np.float64)
     od = host(od)
+    n_groups = 0
     for h in range(w.H):
         ref = orc.plan_head(Q[0, h], K[0, h], V[0, h], G, k, w.scale)
         assert np.array_equal(perm[0, h], ref["perm"])
         c = orc.group_prob_sums(Q[0, h], K[0, h], w.scale, ref["perm"], G)
-        same = []
+        assert np.all(np.abs(cs[0, h] - c) <= COLSUM_REL * c + COLSUM_ABS)
         for g in range(w.n_groups):
             kv_sets_agree(kv[0, h, g], c[g], k)
-            same.append(np.array_equal(kv[0, h, g], ref["kv_idx"][g]))
-        rows = np.concatenate([orc.group_rows(ref["perm"], G, g) for g in range(w.n_groups) if same[g]])
-        assert len(rows) > 0
-        assert_residual_close(res[0, h][rows], ref["residual"][rows], f"plan residual h{h}")
+            rows = orc.group_rows(ref["perm"], G, g)
+            R, _, _ = orc.residual_group(Q[0, h][rows], K[0, h], V[0, h], w.scale, kv[0, h, g])
+            assert_residual_close(res[0, h][rows], R, f"plan residual h{h} g{g}")
+            n_groups += 1
         assert_out_close(od[0, h], ref["O_dense"], f"plan O_dense h{h}")
         # a reused step on the plan's own inputs reproduces dense attention
         assert_out_close(o_step[0, h], ref["O_dense"], f"step on unchanged inputs h{h}")
+    assert n_groups == w.H * w.n_groups
+
+
+@pytest.mark.parametrize("N,d,G", [(1000, 128, 128), (777, 64, 64)])
+def test_plan_statistics_elementwise(N, d, G):
+    """a2 and a3 read back from the workspace: every row's log normaliser
+    m + log2 l against the oracle's row statistics (m inside its documented
+    band), and every group score against the oracle's sums of exact
+    probabilities."""
+    Q, K, V = synth.random_qkv(1, 1, N, d, seed=15, q_std=2.0)
+    q, kd, v = dev_bf16(Q), dev_bf16(K), dev_bf16(V)
+    k = 100
+    perm = orc.group_queries(Q[0, 0]).astype(np.int32)
+    ws = mcs.alloc_workspace(1, 1, N, d, G, k, q.device)
+    mcs.plan_stats(q, kd, v, G, k, workspace=ws)
+    mcs.plan_scores(q, kd, torch.from_numpy(perm[None, None].copy()).cuda(), G, k, ws)
+    torch.cuda.synchronize()
+    assert mcs.last_device_status() == 0
+    views = mcs.workspace_views(ws, 1, 1, N, d, G, k)
+    m_gpu = views["row_m"][0, 0].cpu().numpy().astype(np.float64)
+    l_gpu = views["row_l"][0, 0].cpu().numpy().astype(np.float64)
+    m_ref, l_ref = orc.row_stats(Q[0, 0], K[0, 0], 1 / np.sqrt(d))
+    lse_gpu = (m_gpu + np.log2(l_gpu)) * np.log(2.0)
+    assert np.abs(lse_gpu - (m_ref + np.log(l_ref))).max() <= LSE_ABS
+    mx = m_ref * np.log2(np.e)
+    assert np.all(m_gpu <= mx + 1e-3) and np.all(m_gpu >= mx - 32 - 1e-3)
+    c = orc.group_prob_sums(Q[0, 0], K[0, 0], 1 / np.sqrt(d), perm, G)
+    cs = views["colsum"][0, 0].cpu().numpy().astype(np.float64)
+    assert cs.shape == c.shape
+    assert np.all(np.abs(cs - c) <= COLSUM_REL * c + COLSUM_ABS)
+    # O32, the plan's fp32 dense output, against the oracle's dense attention
+    o32 = views["O32"][0, 0].cpu().numpy().astype(np.float64)
+    ref = orc.dense_attention(Q[0, 0], K[0, 0], V[0, 0], 1 / np.sqrt(d))
+    assert_residual_close(o32, ref, "plan fp32 dense output")
+
+
+@pytest.mark.parametrize("N,d,G", [(1000, 128, 128), (700, 64, 64)])
+def test_plan_with_k_equal_n(N, d, G):
+    """k = N keeps every key: the residual vanishes (up to the fp32 rounding
+    of two equal sums) and a reused step, on these or on drifted inputs,
+    equals dense attention of its own inputs."""
+    Q, K, V = synth.random_qkv(1, 1, N, d, seed=16, q_std=2.0)
+    q, kd, v = dev_bf16(Q), dev_bf16(K), dev_bf16(V)
+    meta, od = mcs.plan(q, kd, v, G, N, return_dense=True)
+    torch.cuda.synchronize()
+    assert meta.k == N
+    res = meta.residual.cpu().numpy().astype(np.float64)
+    ref = orc.dense_attention(Q[0, 0], K[0, 0], V[0, 0], 1 / np.sqrt(d))
+    assert np.linalg.norm(res[0, 0]) <= 1e-3 * np.linalg.norm(ref)
+    assert_out_close(host(mcs.sparse_step(q, kd, v, meta))[0, 0], ref, "k = N step, plan inputs")
+    Q2, K2, V2 = synth.random_qkv(1, 1, N, d, seed=17, q_std=2.0)
+    o2 = host(mcs.sparse_step(dev_bf16(Q2), dev_bf16(K2), dev_bf16(V2), meta))
+    torch.cuda.synchronize()
+    assert mcs.last_device_status() == 0
+    ref2 = orc.dense_attention(Q2[0, 0], K2[0, 0], V2[0, 0], 1 / np.sqrt(d))
+    assert_out_close(o2[0, 0], ref2, "k = N step, other inputs")
 
 
 # ----------------------------------------------------------------------------- failure handling

@@ -1,9 +1,10 @@
 """The allocation-free validation entry point (mcs_validate_meta_noalloc).
 
 Some callers of this library cannot allocate device memory when they want to
-check cached metadata, for instance code recorded into a CUDA graph capture,
-where cudaMalloc is not allowed, or a plugin whose host framework owns all
-device memory.  For them the library keeps a fixed scratch array of its own.
+check cached metadata: a serving runtime that reserves all device memory at
+start-up and forbids allocation afterwards, or a plugin whose host framework
+owns all device memory and its allocator.  For them the library keeps a fixed
+scratch array of its own (a call is synchronous, like mcs_validate_meta).
 These tests call it through the C ABI and check that it reports exactly what
 the workspace-based mcs_validate_meta reports, call after call, so leftovers
 in the shared array never leak into a later answer.
