@@ -91,7 +91,7 @@ __device__ __forceinline__ void mbar_arrive(uint32_t bar) {
 }
 
 // Non-blocking test of a phase: cheap when the phase has already completed
-// (on B200 about 40 cycles of the issuing thread).
+// (on B200 about 40 cycles of the issuing thread), so every wait starts with it.
 __device__ __forceinline__ bool mbar_test_wait(uint32_t bar, uint32_t parity) {
   uint32_t ok;
   asm volatile(
@@ -104,19 +104,18 @@ __device__ __forceinline__ bool mbar_test_wait(uint32_t bar, uint32_t parity) {
   return ok != 0;
 }
 
-// One bounded, suspending test of a phase.  The suspend-time hint lets the
-// hardware park the thread (up to 0.2 ms) until the phase completes instead
-// of returning at once, so waiting warps stop taking issue slots from the
-// working ones.  It costs about 200 cycles even when the phase is complete,
-// so mbar_wait tries mbar_test_wait first.
+// One bounded test of a phase that may suspend the thread for a short,
+// hardware-chosen time.  (A suspend-time hint of 1-200 us was measured to
+// slow the pair kernel by 6-14 %: a hinted wait costs about 200 cycles even
+// when the phase has completed, and wake-up after completion is slower.)
 __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
   uint32_t ok;
   asm volatile(
       "{\n\t.reg .pred p;\n\t"
-      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
+      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
       "selp.u32 %0, 1, 0, p;\n\t}\n"
       : "=r"(ok)
-      : "r"(bar), "r"(parity), "r"(200000u)
+      : "r"(bar), "r"(parity)
       : "memory");
   return ok != 0;
 }
