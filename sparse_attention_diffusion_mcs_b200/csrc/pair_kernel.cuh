@@ -409,14 +409,18 @@ __global__ void __launch_bounds__(PairCfg<D>::THREADS, 1) pair_kernel(const __gr
           if (last) umma_commit_elect(b_vempty(s));
           return true;
         };
-        // the first two tiles' Q.K^T of each group, in tile order
+        // the first two tiles' Q.K^T of each group, in tile order (the group
+        // loops are unrolled so each group's counters stay in registers)
         ok = true;
-        for (int j = 0; j < 2 && ok; ++j)
-          for (int X = 0; X < 2 && ok; ++X)
-            if (act(X, j)) ok = issue_qk(j, X);
+#pragma unroll
+        for (int j = 0; j < 2; ++j)
+#pragma unroll
+          for (int X = 0; X < 2; ++X)
+            if (ok && act(X, j)) ok = issue_qk(j, X);
         for (int j = 0; j < T && ok; ++j) {
-          for (int X = 0; X < 2 && ok; ++X) {
-            if (act(X, j)) ok = issue_pv(j, X);
+#pragma unroll
+          for (int X = 0; X < 2; ++X) {
+            if (ok && act(X, j)) ok = issue_pv(j, X);
             if (ok && j + 2 < T && act(X, j + 2)) ok = issue_qk(j + 2, X);
           }
         }

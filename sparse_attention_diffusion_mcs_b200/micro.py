@@ -72,4 +72,4 @@ def gather_rate(mode: str, warps: int, rows: int = 65536, tiles: int = 256, reps
     t = sorted(times)[len(times) // 2]
     nbytes = sms * tiles * 128 * 256
     return {"mode": mode, "warps": warps, "bytes": nbytes, "seconds": t, "gbs": nbytes / t / 1e9,
-            "ops_per_sm_cycle_at_1965mhz": (nbytes / 512) / sms / (t * 1.965e9)}
+            "gbs_per_sm": nbytes / t / 1e9 / sms}
