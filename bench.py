@@ -10,8 +10,10 @@ events on the launching stream.
 
 The headline metric is the reused step's effective TFLOP/s (4*B*H*N*k*d per
 step); ms per reused step, per plan and per dense call, and the speedup over
-dense, are reported beside it.  Multi-GPU runs are weak-scaled: every rank
-runs its own layer (heads are independent; no collective on the data path).
+dense, are reported beside it.  Multi-GPU runs shard one layer by head blocks
+(shard.py): rank r holds heads [r*BH, (r+1)*BH) of a layer of W*BH heads, so
+the per-GPU work stays fixed (weak scaling) and nothing crosses GPUs on the
+data path (heads are independent).
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl reference]
 """
@@ -71,10 +73,16 @@ def parse_args():
 
 # ----------------------------------------------------------------------------- ranks
 
-def rank_workload(w, rank: int):
-    """Weak scaling: every rank runs its own layer of the same shape, seeded
-    apart (heads are independent; nothing is exchanged on the data path)."""
-    return w.with_(seed=w.seed + rank)
+def rank_heads(w, rank: int):
+    """Multi-GPU runs shard ONE layer by head blocks (heads are independent;
+    nothing is exchanged on the data path): with W ranks the layer has
+    W * B*H flattened heads and rank r holds [r*BH, (r+1)*BH) -- every rank
+    the workload's own per-GPU size (weak scaling).  Inputs are seeded per
+    global head, so rank r regenerates exactly its block."""
+    from sparse_attention_diffusion_mcs_b200.shard import head_range
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    start, count = head_range(w.BH * world, world, rank)
+    return list(range(start, start + count))
 
 
 def max_over_ranks(t):
@@ -89,30 +97,31 @@ def max_over_ranks(t):
 # ----------------------------------------------------------------------------- inputs
 
 def _gen_head(args):
-    cfg, k, G, bh, seed_shift = args
-    w = synth.workload(cfg, k=k, G=G).with_(seed=seed_shift)
+    cfg, k, G, slot, bh, seed = args
+    w = synth.workload(cfg, k=k, G=G).with_(seed=seed)
     q1, k1, v1 = synth.head_tensors(w, bh, step=1)
     q2 = synth.drift_head(q1, w, 2, 0, bh)
     k2 = synth.drift_head(k1, w, 2, 1, bh)
     v2 = synth.drift_head(v1, w, 2, 2, bh)
-    return bh, (q1, k1, v1), (q2, k2, v2)
+    return slot, (q1, k1, v1), (q2, k2, v2)
 
 
 def make_inputs(w, rank: int):
-    """Step-1 (plan) and step-2 (reused) tensors of one layer, uint16 [B,H,N,d]."""
+    """Step-1 (plan) and step-2 (reused) tensors of this rank's block of
+    heads (the whole layer on one GPU), uint16 [B,H,N,d]."""
     import concurrent.futures as cf
     import multiprocessing as mp
     shape = (w.BH, w.N, w.d)
     s1 = [np.empty(shape, np.uint16) for _ in range(3)]
     s2 = [np.empty(shape, np.uint16) for _ in range(3)]
-    wr = rank_workload(w, rank)
-    jobs = [(w.cfg_id, w.k, w.G, bh, wr.seed) for bh in range(w.BH)]
+    heads = rank_heads(w, rank)
+    jobs = [(w.cfg_id, w.k, w.G, slot, bh, w.seed) for slot, bh in enumerate(heads)]
     nproc = max(1, min(len(jobs), len(os.sched_getaffinity(0)), 16))
     with cf.ProcessPoolExecutor(nproc, mp_context=mp.get_context("spawn")) as ex:
-        for bh, a, b in ex.map(_gen_head, jobs):
+        for slot, a, b in ex.map(_gen_head, jobs):
             for i in range(3):
-                s1[i][bh] = a[i]
-                s2[i][bh] = b[i]
+                s1[i][slot] = a[i]
+                s2[i][slot] = b[i]
     rs = lambda x: x.reshape(w.B, w.H, w.N, w.d)
     return [rs(x) for x in s1], [rs(x) for x in s2]
 
@@ -295,7 +304,8 @@ def workload_config(w, n):
             "global_batch": w.B * n, "seq_len": w.N,
             "l2": "inputs larger than L2 (each of Q, K, V is "
                   f"{w.BH * w.N * w.d * 2 / 1e6:.0f} MB per step; no explicit flush)",
-            "parallelism": f"weak scaling, {n} independent layer(s), one per GPU"}
+            "parallelism": (f"one layer of {n}x{w.BH} heads sharded by head blocks, {w.BH} per GPU "
+                            "(weak scaling; no data-path collective)") if n > 1 else "1 GPU"}
 
 
 # ----------------------------------------------------------------------------- main arm
