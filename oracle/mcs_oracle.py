@@ -48,6 +48,7 @@ __all__ = [
     "select_kv", "dense_rows", "dense_attention", "sparse_group",
     "sparse_attention", "residual_group", "plan_head", "reused_step_head",
     "rel_l2", "schedule_head",
+    "select_blocks", "pooled_scores", "ungrouped_rows", "retained_mass",
 ]
 
 
@@ -319,3 +320,60 @@ def schedule_head(steps, plan_steps, G: int, k: int, scale: float):
                     "rel_l2": rel_l2(O, Od), "rel_l2_no_residual": rel_l2(O - meta["residual"], Od)})
     return out
 
+
+
+# ---------------------------------------------------------------------------
+# Synthetic ablations of the three failure modes the method addresses
+#   ([abstract] "controlled oracle comparisons": the dense-sparse gap comes
+#    from constraints imposed by token grouping, from inaccurate interaction
+#    selection, and from the attention contributions lost; [p1-mcs] the three
+#    failure modes and the one fix).  Each function below is the counterpart
+#    of one MC-Sparse choice with that choice taken away.
+# ---------------------------------------------------------------------------
+
+def select_blocks(c: np.ndarray, k_blocks: int, block: int) -> np.ndarray:
+    """Block-granular selection instead of individual tokens: the keys are cut
+    into aligned blocks of `block` keys (a ragged last block is not a
+    candidate), a block's score is the sum of its keys' scores, the
+    k_blocks' = min(k_blocks, full blocks) highest blocks are kept (ties to the
+    lower block index), and their keys are returned ascending."""
+    c = np.asarray(c, dtype=np.float64)
+    nb = c.shape[0] // block
+    bs = c[:nb * block].reshape(nb, block).sum(axis=1)
+    kb = min(int(k_blocks), nb)
+    blocks = np.sort(np.lexsort((np.arange(nb), -bs))[:kb])
+    return (blocks[:, None] * block + np.arange(block)[None, :]).reshape(-1)
+
+
+def pooled_scores(Q, K, scale: float, perm, G: int, groups=None) -> np.ndarray:
+    """A pooled, heuristic group score instead of exact summed probabilities:
+    the group's queries are averaged into one query q_g and key j scores
+    softmax_j(scale q_g . K_j), the probability the pooled query gives it.
+    [len(groups), N]"""
+    Q = _as_f64(Q)
+    n = Q.shape[0]
+    ng = -(-n // G)
+    groups = range(ng) if groups is None else groups
+    out = np.empty((len(groups), _as_f64(K).shape[0]))
+    for r, g in enumerate(groups):
+        qbar = Q[group_rows(perm, G, g)].mean(axis=0, keepdims=True)
+        out[r] = probabilities(qbar, K, scale)[0]
+    return out
+
+
+def ungrouped_rows(Qrows, K, V, scale: float, k: int) -> np.ndarray:
+    """No grouping constraint: every query keeps its own k' = min(k, N) largest
+    exact probabilities (ties to the lower key index) and attends to them
+    alone, renormalised.  [rows, d]"""
+    Qrows = _as_f64(Qrows)
+    P = probabilities(Qrows, K, scale)
+    out = np.empty((Qrows.shape[0], _as_f64(V).shape[1]))
+    for r in range(Qrows.shape[0]):
+        out[r] = sparse_group(Qrows[r:r + 1], K, V, scale, select_kv(P[r], k))[0]
+    return out
+
+
+def retained_mass(c_row: np.ndarray, idx, size: int) -> float:
+    """alpha_g: the share of group g's dense attention mass its kept keys hold,
+    sum_{j in S_g} c_gj / |g| (c the group's summed exact probabilities)."""
+    return float(np.asarray(c_row, dtype=np.float64)[np.asarray(idx)].sum() / size)

@@ -329,3 +329,68 @@ def test_schedule_constant_values_exact_under_drift():
     st = [(q, k, np.tile(c, (48, 1))) for q, k, _ in st]
     for x in orc.schedule_head(st, [1], G=8, k=4, scale=0.4):
         assert x["rel_l2"] < 1e-13 and x["rel_l2_no_residual"] < 1e-13
+
+
+# --- ablations of the three failure modes -------------------------------------
+
+def test_select_blocks_of_one_key_is_token_selection():
+    c = np.random.default_rng(40).random(37)
+    for k in (1, 5, 37):
+        assert np.array_equal(orc.select_blocks(c, k, 1), orc.select_kv(c, k))
+
+
+def test_select_blocks_brute_force_and_ragged_tail():
+    rng = np.random.default_rng(41)
+    block, n = 4, 22                       # 5 full blocks, a ragged tail of 2 keys
+    for trial in range(20):
+        c = rng.integers(0, 3, size=n).astype(np.float64)    # many exact ties
+        c[20:] = 100.0                                       # the tail is never a candidate
+        for kb in (1, 2, 3, 5, 9):
+            got = orc.select_blocks(c, kb, block)
+            kk = min(kb, n // block)
+            sums = [c[b * block:(b + 1) * block].sum() for b in range(n // block)]
+            best = max(sum(sums[b] for b in comb) for comb in itertools.combinations(range(n // block), kk))
+            chosen = sorted(set((got // block).tolist()))
+            assert len(got) == kk * block and np.all(np.diff(got) > 0)
+            assert sum(sums[b] for b in chosen) == best
+            # among subsets of equal total the lowest block indices win
+            first = min(itertools.combinations(range(n // block), kk),
+                        key=lambda comb: (-sum(sums[b] for b in comb), comb))
+            assert chosen == list(first)
+            assert np.all(got < 20)
+
+
+def test_pooled_score_of_single_query_groups_is_its_probability_row():
+    Q, K = _rand(9, 4, 42), _rand(13, 4, 43)
+    perm = np.arange(9)
+    got = orc.pooled_scores(Q, K, 0.5, perm, 1)
+    assert np.allclose(got, orc.probabilities(Q, K, 0.5), rtol=0, atol=1e-15)
+    assert np.allclose(got.sum(axis=1), 1.0)
+
+
+def test_pooled_score_uses_the_mean_query():
+    Q, K = _rand(8, 5, 44), _rand(11, 5, 45)
+    perm = np.array([3, 1, 7, 0, 2, 6, 5, 4])
+    got = orc.pooled_scores(Q, K, 0.3, perm, 4)
+    for g in range(2):
+        qbar = Q[perm[4 * g:4 * g + 4]].sum(axis=0) / 4
+        s = [0.3 * float(qbar @ K[j]) for j in range(11)]
+        e = np.exp(np.array(s) - max(s))
+        assert np.allclose(got[g], e / e.sum(), rtol=1e-13)
+
+
+def test_ungrouped_rows_closed_forms():
+    Q, K, V = _rand(6, 4, 46, 2.0), _rand(10, 4, 47), _rand(10, 3, 48)
+    assert np.allclose(orc.ungrouped_rows(Q, K, V, 0.5, 10), orc.dense_rows(Q, K, V, 0.5), atol=1e-14)
+    top1 = orc.ungrouped_rows(Q, K, V, 0.5, 1)
+    P = orc.probabilities(Q, K, 0.5)
+    assert np.allclose(top1, V[np.argmax(P, axis=1)], atol=0)
+
+
+def test_retained_mass_closed_forms():
+    Q, K = _rand(5, 4, 49), _rand(12, 4, 50)
+    c = orc.probabilities(Q, K, 0.7).sum(axis=0)
+    assert abs(orc.retained_mass(c, np.arange(12), 5) - 1.0) < 1e-14
+    idx = orc.select_kv(c, 4)
+    other = np.setdiff1d(np.arange(12), idx)
+    assert abs(orc.retained_mass(c, idx, 5) + orc.retained_mass(c, other, 5) - 1.0) < 1e-14
