@@ -59,6 +59,11 @@ def parse_args():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-micro", action="store_true", help="skip the gather-ceiling measurement")
+    ap.add_argument("--ablate", action="store_true",
+                    help="controlled comparisons of the three failure modes on the workload's schedule "
+                         "(token vs block vs pooled selection, with and without the residual, and the "
+                         "ungrouped per-query oracle on sampled queries); not the contract line")
+    ap.add_argument("--ablate-rows", type=int, default=64, help="sampled queries per head for the ungrouped oracle")
     ap.add_argument("--micro", choices=["gather"], default=None,
                     help="run the gather microbenchmark alone: one JSON line per (mode, warps)")
     ap.add_argument("--sweep", action="store_true",
@@ -370,6 +375,82 @@ def run_sweep(args):
     return 0
 
 
+def _ungrouped_head(args):
+    """fp64 oracle, one head: the ungrouped per-query selection planned on
+    step 1 and reused on step t, for sampled queries (rows); returns the
+    rel-L2 numerator and denominator of the with- and without-residual
+    outputs against dense attention of step t."""
+    from oracle import mcs_oracle as orc
+    cfg, k, G, bh, seed, rows, step = args
+    w = synth.workload(cfg, k=k, G=G).with_(seed=seed)
+    q1, k1, v1 = synth.head_tensors(w, bh, step=1)
+    qt, kt, vt = synth.head_tensors(w, bh, step=step)
+    P1 = orc.probabilities(q1[rows], k1, w.scale)
+    num = num_nr = den = 0.0
+    O1 = P1 @ orc.widen_bf16(v1)
+    for r_i, r in enumerate(rows):
+        idx = orc.select_kv(P1[r_i], w.k)
+        R = O1[r_i] - orc.sparse_group(q1[r:r + 1], k1, v1, w.scale, idx)[0]
+        o = orc.sparse_group(qt[r:r + 1], kt, vt, w.scale, idx)[0]
+        dref = orc.dense_rows(qt[r:r + 1], kt, vt, w.scale)[0]
+        num += float(((o + R - dref) ** 2).sum())
+        num_nr += float(((o - dref) ** 2).sum())
+        den += float((dref ** 2).sum())
+    return num, num_nr, den
+
+
+def run_ablate(args):
+    """The workload's denoising steps with one plan at step 1 (so every later
+    step measures how well each selection's metadata carries over) and every
+    variant of sparse_attention_diffusion_mcs_b200.ablate reused on steps
+    2..S: one JSON line per step with each variant's rel-L2 to dense, with
+    and without its residual, and the groups' mean retained mass; then the
+    ungrouped per-query oracle on sampled queries of two heads."""
+    import concurrent.futures as cf
+    import multiprocessing as mp
+    w = synth.workload(args.config, k=args.k, G=args.G)
+    if args.heads:
+        w = w.with_(H=min(args.heads, w.H))
+    steps = list(schedule_inputs(w))            # host tensors of every step (process pool first)
+    rng = np.random.default_rng(7)
+    heads = sorted({0, w.BH - 1})
+    rows = np.sort(rng.choice(w.N, size=min(args.ablate_rows, w.N), replace=False))
+    jobs = [(w.cfg_id, w.k, w.G, bh, w.seed, rows, t) for t in range(2, w.steps + 1) for bh in heads]
+    with cf.ProcessPoolExecutor(max(1, min(len(jobs), 16)), mp_context=mp.get_context("spawn")) as ex:
+        ungrouped = list(ex.map(_ungrouped_head, jobs))
+    import torch
+    from sparse_attention_diffusion_mcs_b200 import ablate
+    import sparse_attention_diffusion_mcs_b200 as mcs
+    dev = torch.device("cuda", 0)
+    up = lambda a: torch.from_numpy(a.view(np.int16)).view(torch.bfloat16).to(dev)
+    abl = None
+    summary = {}
+    for t, host in steps:
+        Q, K, V = (up(x) for x in host)
+        if abl is None:
+            abl = ablate.Ablation(Q, K, V, w.G, w.k, scale=w.scale)
+            print(json.dumps({"ablate": w.name, "step": t, "kind": "plan",
+                              "alpha_mean": abl.alpha}), flush=True)
+            continue
+        Od = mcs.dense(Q, K, V, w.scale)
+        res = abl.step(Q, K, V, Od)
+        i0 = (t - 2) * len(heads)
+        num, num_nr, den = (sum(x[i] for x in ungrouped[i0:i0 + len(heads)]) for i in range(3))
+        res["ungrouped (oracle, sampled)"] = {"rel_l2": (num / den) ** 0.5,
+                                              "rel_l2_without_residual": (num_nr / den) ** 0.5,
+                                              "keys": min(w.k, w.N), "queries": int(len(rows) * len(heads))}
+        for name, r in res.items():
+            summary.setdefault(name, []).append(r)
+        print(json.dumps({"ablate": w.name, "step": t, "kind": "reused", "variants": res}), flush=True)
+        del Q, K, V, Od
+    print(json.dumps({"ablate": w.name, "workload": workload_config(w, 1)["workload"],
+                      "plan_steps": [1], "steps": w.steps, "drift": w.drift,
+                      "mean_rel_l2": {n: float(np.mean([x["rel_l2"] for x in v])) for n, v in summary.items()},
+                      "mean_rel_l2_without_residual": {n: float(np.mean([x["rel_l2_without_residual"] for x in v]))
+                                                       for n, v in summary.items()}}), flush=True)
+    return 0
+
+
 def run_micro(args):
     """--micro gather: the rate at which one CTA per SM brings index-listed
     256-byte rows (bf16, d = 128) into shared memory, by TMA tile::gather4
@@ -482,6 +563,8 @@ def main():
         return run_sweep(args)
     if args.micro:
         return run_micro(args)
+    if args.ablate:
+        return run_ablate(args)
 
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))

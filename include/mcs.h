@@ -262,6 +262,37 @@ mcs_status mcs_validate_meta(const mcs_meta *meta, void *workspace, size_t works
 #define MCS_NOALLOC_MAX_TOKENS (1u << 23)
 mcs_status mcs_validate_meta_noalloc(const mcs_meta *meta, int *first_bad, mcs_stream_t stream);
 
+/*
+ * Ablation tools -- the selection rules MC-Sparse replaces, for controlled
+ * comparisons of its three failure modes (aiqbench.com abstract:
+ * "constraints imposed by token grouping, inaccurate interaction selection,
+ * and the attention contributions lost"; cnshai.top post, section "MC-Sparse:
+ * three failure modes, one fix").  Their key lists feed mcs_plan_residual and
+ * mcs_sparse_step like any other selection.  Not on the hot path.
+ */
+
+/* Bytes of workspace mcs_select_blocks needs; 0 for invalid sizes. */
+size_t mcs_select_blocks_workspace_size(int rows, int N, int block, int k_blocks);
+
+/* Block-granular selection: per row of `scores` (float32 [rows, N], >= 0,
+ * e.g. the group probability sums), the keys are cut into aligned blocks of
+ * `block` keys (a ragged last block is not a candidate), a block scores the
+ * sum of its keys' scores, the k_blocks highest blocks are kept (ties to the
+ * lower block index) and their keys written ascending to kv_idx (int32
+ * [rows, k_blocks * block]).  1 <= k_blocks <= N / block, else INVALID_ARG.
+ * workspace: >= mcs_select_blocks_workspace_size(...) bytes, 256-byte
+ * aligned.  Asynchronous. */
+mcs_status mcs_select_blocks(const float *scores, int rows, int N, int block, int k_blocks, int32_t *kv_idx,
+                             void *workspace, size_t workspace_bytes, mcs_stream_t stream);
+
+/* Pooled-query scores: for each group g of the grouping `perm` (int32
+ * [B,H,N]), its queries averaged into one query qbar_g, and scores[b,h,g,j] =
+ * softmax_j(scale qbar_g . K_j) (float32 [B,H,ceil(N/G),N]): a heuristic in
+ * place of the exact summed probabilities; select with mcs_select_topk.  Same
+ * Q/K conventions as mcs_plan; G in {64, 128}.  Asynchronous. */
+mcs_status mcs_pooled_scores(const void *Q, const void *K, const int32_t *perm, int B, int H, int N, int d, int G,
+                             float scale, float *scores, mcs_stream_t stream);
+
 /* Synchronise `stream`, then read and clear this device's status word.
  * Returns MCS_OK, or MCS_ERR_TIMEOUT if a kernel's bounded wait ran out
  * since the last read. */

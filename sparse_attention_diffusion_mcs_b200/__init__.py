@@ -16,6 +16,8 @@ from .api import (  # noqa: F401
     plan_select,
     plan_stats,
     plan_topk,
+    pooled_scores,
+    select_blocks,
     select_topk,
     selftest_wait_timeout,
     set_wait_limit_ns,

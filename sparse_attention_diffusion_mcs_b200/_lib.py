@@ -58,6 +58,9 @@ PROTOTYPES = {
     "mcs_validate_workspace_size": (c_size_t, [c_int, c_int, c_int]),
     "mcs_validate_meta": (c_int, [PMETA, c_vp, c_size_t, ctypes.POINTER(c_int), c_vp]),
     "mcs_validate_meta_noalloc": (c_int, [PMETA, ctypes.POINTER(c_int), c_vp]),
+    "mcs_select_blocks_workspace_size": (c_size_t, [c_int, c_int, c_int, c_int]),
+    "mcs_select_blocks": (c_int, [c_vp, c_int, c_int, c_int, c_int, c_vp, c_vp, c_size_t, c_vp]),
+    "mcs_pooled_scores": (c_int, [c_vp, c_vp, c_vp, c_int, c_int, c_int, c_int, c_int, c_float, c_vp, c_vp]),
     "mcs_last_device_status": (c_int, [c_vp]),
     "mcs_selftest_wait_timeout": (c_int, [c_u64, c_vp]),
     "mcs_set_wait_limit_ns": (None, [c_u64]),

@@ -317,6 +317,49 @@ def select_topk(scores: torch.Tensor, k: int, out: Optional[torch.Tensor] = None
     return out
 
 
+def select_blocks(scores: torch.Tensor, k_blocks: int, block: int, out: Optional[torch.Tensor] = None) -> torch.Tensor:
+    """Block-granular selection on a float32 score matrix [..., N] (an
+    ablation of token-level selection): per row the k_blocks aligned blocks
+    of `block` keys with the highest summed score (full blocks only), as
+    their keys ascending: int32 [..., k_blocks * block]."""
+    if scores.dtype != torch.float32 or not scores.is_cuda:
+        raise TypeError("scores must be a float32 CUDA tensor")
+    scores = scores.contiguous()
+    N = scores.shape[-1]
+    rows = scores.numel() // N if N else 0
+    if not 1 <= k_blocks <= N // block:
+        raise ValueError(f"k_blocks must be in [1, N // block] = [1, {N // block}]")
+    if out is None:
+        out = torch.empty((*scores.shape[:-1], k_blocks * block), dtype=torch.int32, device=scores.device)
+    else:
+        _check_tensor(out, "out", (*scores.shape[:-1], k_blocks * block), torch.int32, scores.device)
+    n = lib().mcs_select_blocks_workspace_size(rows, N, block, k_blocks)
+    ws = torch.empty(max(int(n), 1), dtype=torch.uint8, device=scores.device)
+    with _on(scores.device):
+        check(lib().mcs_select_blocks(_ptr(scores), rows, N, block, k_blocks, _ptr(out), _ptr(ws), ws.numel(),
+                                      _stream(scores.device)), "mcs_select_blocks")
+    return out
+
+
+def pooled_scores(Q, K, perm, G: int, scale: Optional[float] = None,
+                  out: Optional[torch.Tensor] = None) -> torch.Tensor:
+    """Pooled-query scores (an ablation of exact summed probabilities):
+    float32 [B, H, n_groups, N], softmax_j(scale mean_{i in g}(Q_i) . K_j)."""
+    _check_qkv(Q, K)
+    B, H, N, d = Q.shape
+    perm = perm.to(torch.int32).contiguous()
+    _check_tensor(perm, "perm", (B, H, N), torch.int32, Q.device)
+    ng = -(-N // G)
+    if out is None:
+        out = torch.empty((B, H, ng, N), dtype=torch.float32, device=Q.device)
+    else:
+        _check_tensor(out, "out", (B, H, ng, N), torch.float32, Q.device)
+    with _on(Q.device):
+        check(lib().mcs_pooled_scores(_ptr(Q), _ptr(K), _ptr(perm), B, H, N, d, G, _scale(d, scale), _ptr(out),
+                                      _stream(Q.device)), "mcs_pooled_scores")
+    return out
+
+
 def plan_select(Q, K, V, perm, G: int, k: int, scale: Optional[float] = None,
                 workspace: Optional[torch.Tensor] = None) -> torch.Tensor:
     """Steps a2-a4 for a given grouping: int32 kv_idx [B, H, n_groups, min(k, N)].

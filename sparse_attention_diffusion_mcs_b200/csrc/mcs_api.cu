@@ -8,6 +8,7 @@
 #include <mutex>
 
 #include "../../include/mcs.h"
+#include "ablation_kernels.cuh"
 #include "attn_dual_kernel.cuh"
 #include "attn_kernel.cuh"
 #include "colsum_kernel.cuh"
@@ -678,6 +679,54 @@ mcs_status mcs_validate_meta_noalloc(const mcs_meta *meta, int *first_bad, mcs_s
   if (h == INT_MAX) return MCS_OK;
   if (first_bad) *first_bad = h;
   return MCS_ERR_BAD_META;
+}
+
+size_t mcs_select_blocks_workspace_size(int rows, int N, int block, int k_blocks) {
+  if (rows < 0 || N < 1 || block < 1 || k_blocks < 1 || N / block < k_blocks) return 0;
+  const size_t nb = N / block;
+  return align256(static_cast<size_t>(rows) * nb * 4) + align256(static_cast<size_t>(rows) * k_blocks * 4);
+}
+
+mcs_status mcs_select_blocks(const float *scores, int rows, int N, int block, int k_blocks, int32_t *kv_idx,
+                             void *workspace, size_t workspace_bytes, mcs_stream_t stream) {
+  if (!scores || !kv_idx || rows < 0 || N < 1 || block < 1 || k_blocks < 1 || N / block < k_blocks)
+    return MCS_ERR_INVALID_ARG;
+  const size_t need = mcs_select_blocks_workspace_size(rows, N, block, k_blocks);
+  if (rows == 0) return MCS_OK;
+  mcs_status st = check_ws(workspace, workspace_bytes, need);
+  if (st != MCS_OK) return st;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  const int nb = N / block;
+  float *bs = static_cast<float *>(workspace);
+  int32_t *blk = reinterpret_cast<int32_t *>(static_cast<uint8_t *>(workspace) +
+                                             align256(static_cast<size_t>(rows) * nb * 4));
+  block_sum_kernel<<<148 * 8, 256, 0, s>>>(scores, rows, N, block, bs);
+  cudaError_t e = cudaGetLastError();
+  if (e == cudaSuccess) e = launch_topk(bs, rows, nb, k_blocks, blk, s);
+  if (e == cudaSuccess) {
+    expand_blocks_kernel<<<148 * 8, 256, 0, s>>>(blk, rows, k_blocks, block, kv_idx);
+    e = cudaGetLastError();
+  }
+  return cuda_status(e);
+}
+
+mcs_status mcs_pooled_scores(const void *Q, const void *K, const int32_t *perm, int B, int H, int N, int d, int G,
+                             float scale, float *scores, mcs_stream_t stream) {
+  mcs_status st = check_common(Q, K, K, B, H, N, d, scale);
+  if (st != MCS_OK) return st;
+  if (!perm || !scores) return MCS_ERR_INVALID_ARG;
+  if (!g_ok(G)) return MCS_ERR_UNSUPPORTED;
+  const int ng = (N + G - 1) / G;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  const float sl2 = scale * 1.4426950408889634f;
+  const dim3 grid(ng, B * H);
+  if (d == 64)
+    pooled_scores_kernel<64><<<grid, kPooledThreads, 0, s>>>(static_cast<const bf16 *>(Q), static_cast<const bf16 *>(K),
+                                                             perm, N, G, ng, sl2, scores, status_ptr());
+  else
+    pooled_scores_kernel<128><<<grid, kPooledThreads, 0, s>>>(static_cast<const bf16 *>(Q), static_cast<const bf16 *>(K),
+                                                              perm, N, G, ng, sl2, scores, status_ptr());
+  return cuda_status(cudaGetLastError());
 }
 
 mcs_status mcs_last_device_status(mcs_stream_t stream) {

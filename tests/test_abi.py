@@ -155,3 +155,16 @@ def test_binding_refuses_to_run_without_library(monkeypatch, tmp_path):
     monkeypatch.setattr(_lib, "_lib", None)
     with pytest.raises(ImportError):
         _lib.lib()
+
+
+def test_ablation_tool_argument_errors(L):
+    s = None
+    assert L.mcs_select_blocks_workspace_size(4, 1000, 64, 15) > 0
+    assert L.mcs_select_blocks_workspace_size(4, 1000, 64, 16) == 0          # only 15 full blocks
+    assert L.mcs_select_blocks(None, 4, 1000, 64, 2, FAKE, FAKE, 1 << 20, s) == INVALID
+    assert L.mcs_select_blocks(FAKE, 4, 1000, 64, 0, FAKE, FAKE, 1 << 20, s) == INVALID
+    assert L.mcs_select_blocks(FAKE, 4, 1000, 64, 16, FAKE, FAKE, 1 << 20, s) == INVALID
+    assert L.mcs_select_blocks(FAKE, 4, 1000, 64, 2, FAKE, FAKE, 8, s) == WORKSPACE
+    assert L.mcs_pooled_scores(FAKE, FAKE, None, 1, 1, 128, 64, 64, 0.125, FAKE, s) == INVALID
+    assert L.mcs_pooled_scores(FAKE, FAKE, FAKE, 1, 1, 128, 64, 32, 0.125, FAKE, s) == UNSUPPORTED
+    assert L.mcs_pooled_scores(FAKE, FAKE, FAKE, 1, 1, 128, 96, 64, 0.125, FAKE, s) == UNSUPPORTED
