@@ -64,6 +64,8 @@ def parse_args():
                          "(token vs block vs pooled selection, with and without the residual, and the "
                          "ungrouped per-query oracle on sampled queries); not the contract line")
     ap.add_argument("--ablate-rows", type=int, default=64, help="sampled queries per head for the ungrouped oracle")
+    ap.add_argument("--blocks", action="store_true",
+                    help="block-granular vs token selection: reused-step time and fidelity (not the contract line)")
     ap.add_argument("--micro", choices=["gather"], default=None,
                     help="run the gather microbenchmark alone: one JSON line per (mode, warps)")
     ap.add_argument("--sweep", action="store_true",
@@ -451,6 +453,86 @@ def run_ablate(args):
     return 0
 
 
+def run_blocks(args):
+    """--blocks: block-granular against token-granular selection on one layer
+    of the workload, planned on step 1 and reused on step 2.  For blocks of 64
+    and 128 keys at kb = k // block blocks per group, and for token selection
+    at the same key budget kb * block, time the reused step (block step: one
+    TMA tile load per 64 keys; token step: row gathers) and report its rel-L2
+    to dense attention of step 2 with the residual of its own selection.
+    The token step over the blocks' expanded keys (same keys, gathered) is
+    timed too, so the difference between the two steps is the cost of the
+    gather alone.  One JSON line per variant; not the contract line."""
+    import torch
+    import sparse_attention_diffusion_mcs_b200 as mcs
+    from sparse_attention_diffusion_mcs_b200.denoise import fidelity
+    w = synth.workload(args.config, k=args.k, G=args.G)
+    if args.heads:
+        w = w.with_(H=min(args.heads, w.H))
+    s1, s2 = make_inputs(w, 0)
+    dev = torch.device("cuda", 0)
+    up = lambda a: torch.from_numpy(a.view(np.int16)).view(torch.bfloat16).to(dev)
+    Q1, K1, V1 = (up(x) for x in s1)
+    Q2, K2, V2 = (up(x) for x in s2)
+    del s1, s2
+    B, H, N, d, G, k = w.B, w.H, w.N, w.d, w.G, w.k
+    stream = torch.cuda.current_stream()
+    tc = measured_peaks()["bf16_tflops_sustained"]
+
+    def timed(fn, reps):
+        for _ in range(3):
+            fn()
+        torch.cuda.synchronize()
+        ms = []
+        for _ in range(reps):
+            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            a.record(stream)
+            fn()
+            b.record(stream)
+            torch.cuda.synchronize()
+            ms.append(a.elapsed_time(b))
+        return float(np.median(ms))
+
+    ws = mcs.alloc_workspace(B, H, N, d, G, k, dev)
+    meta = mcs.plan(Q1, K1, V1, G, k, w.scale, workspace=ws)
+    colsum = mcs.workspace_views(ws, B, H, N, d, G, k)["colsum"]
+    Od = mcs.dense(Q2, K2, V2, w.scale)
+    O = torch.empty_like(Q2)
+    reps = max(3, args.steps)
+
+    def report(name, keys, fn, residual):
+        ms = timed(lambda: fn(O), reps)
+        fn(O)
+        rel, rel_nr = fidelity(O, Od, residual)
+        flops = 4 * B * H * N * keys * d
+        print(json.dumps({"blocks": w.name, "variant": name, "keys_per_group": keys, "step_ms": ms,
+                          "tflops": flops / (ms * 1e-3) / 1e12,
+                          "frac_of_sustained_bf16": flops / (ms * 1e-3) / 1e12 / tc,
+                          "rel_l2": rel, "rel_l2_without_residual": rel_nr,
+                          "device_status": mcs.last_device_status()}), flush=True)
+
+    report("token", min(k, N), lambda out: mcs.sparse_step(Q2, K2, V2, meta, w.scale, out=out), meta.residual)
+    for block in (64, 128):
+        kb = k // block
+        if kb < 1 or N // block < kb:
+            continue
+        blk = mcs.select_block_indices(colsum, kb, block)
+        keys = mcs.select_blocks(colsum, kb, block)
+        res = mcs.plan_residual(Q1, K1, V1, meta.perm, keys, G, w.scale, workspace=ws, stats_done=True)
+        bm = mcs.BlockMeta.build(meta.perm, blk, G, block, res)
+        report(f"block{block}", kb * block, lambda out: mcs.sparse_step_blocks(Q2, K2, V2, bm, w.scale, out=out), res)
+        m_keys = mcs.Meta.from_tensors(meta.perm, keys, res, G)
+        report(f"block{block} keys gathered", kb * block,
+               lambda out: mcs.sparse_step(Q2, K2, V2, m_keys, w.scale, out=out), res)
+        tok = mcs.select_topk(colsum, kb * block)
+        res_t = mcs.plan_residual(Q1, K1, V1, meta.perm, tok, G, w.scale, workspace=ws, stats_done=True)
+        m_tok = mcs.Meta.from_tensors(meta.perm, tok, res_t, G)
+        report(f"token@k{kb * block}", kb * block,
+               lambda out: mcs.sparse_step(Q2, K2, V2, m_tok, w.scale, out=out), res_t)
+        del bm, m_keys, m_tok, res, res_t
+    return 0
+
+
 def run_micro(args):
     """--micro gather: the rate at which one CTA per SM brings index-listed
     256-byte rows (bf16, d = 128) into shared memory, by TMA tile::gather4
@@ -565,6 +647,8 @@ def main():
         return run_micro(args)
     if args.ablate:
         return run_ablate(args)
+    if args.blocks:
+        return run_blocks(args)
 
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))

@@ -293,6 +293,50 @@ mcs_status mcs_select_blocks(const float *scores, int rows, int N, int block, in
 mcs_status mcs_pooled_scores(const void *Q, const void *K, const int32_t *perm, int B, int H, int N, int d, int G,
                              float scale, float *scores, mcs_stream_t stream);
 
+/* Block-granular selection as block indices: as mcs_select_blocks, but the
+ * kept blocks' indices b (keys [b*block, (b+1)*block)) are written ascending
+ * to blk_idx (int32 [rows, k_blocks]) instead of their keys.  Same workspace
+ * (mcs_select_blocks_workspace_size) and errors.  Asynchronous. */
+mcs_status mcs_select_block_indices(const float *scores, int rows, int N, int block, int k_blocks,
+                                    int32_t *blk_idx, void *workspace, size_t workspace_bytes,
+                                    mcs_stream_t stream);
+
+/* Union lists of group pairs (the pair_idx / pair_len layout above) from any
+ * ascending unique per-group lists `lists` (int32 [B,H,n_groups,k]): keys as
+ * kv_idx, or block indices for mcs_sparse_step_blocks.  pair_idx int32
+ * [B,H,ceil(n_groups/2),2k], pair_len int32 [B,H,ceil(n_groups/2)].
+ * Unsorted input gives wrong lists but no out-of-bounds access.
+ * INVALID_ARG for a null pointer or k < 1; UNSUPPORTED for B*H > 65535.
+ * Asynchronous. */
+mcs_status mcs_union_pairs(const int32_t *lists, int B, int H, int n_groups, int k, int32_t *pair_idx,
+                           int32_t *pair_len, mcs_stream_t stream);
+
+/*
+ * mcs_sparse_step_blocks -- the reused step over a block-granular selection,
+ * the coarse-block pattern that MC-Sparse's individual KV selection replaces
+ * (cctest.ai article, "Individual KV selection"; cnshai.top post, section
+ * "MC-Sparse: three failure modes, one fix": dropping whole blocks evicts
+ * wanted tokens).  For every group g with kept blocks S_g:
+ *   O_i = sum_{j in keys of S_g} softmax_j(scale Q_i.K_j) V_j (+ R_i)   (i in g)
+ * Each 64-key tile is one contiguous TMA box per 64 columns instead of a row
+ * gather; everything else is the pair kernel of mcs_sparse_step.
+ * perm: int32 [B,H,N] grouping (as mcs_plan writes it).
+ * pair_idx / pair_len: union lists of the groups' ascending block indices
+ *   (mcs_union_pairs over int32 [B,H,n_groups,k_blocks]).
+ * residual: float32 [B,H,N,d] added in the epilogue, or NULL for none.
+ * block in {64, 128} (UNSUPPORTED otherwise), 1 <= k_blocks <= N / block
+ * (INVALID_ARG otherwise).  O: bf16 [B,H,N,d].  A block index outside
+ * [0, N / block) or a pair_len outside [k_blocks, 2 k_blocks] is never read
+ * past: it records MCS_ERR_BAD_META in the device status word.
+ * Given the expanded keys of the same blocks as kv_idx, mcs_sparse_step
+ * (with pair lists) visits the same tiles in the same order and writes the
+ * same bits.  Asynchronous; needs no workspace.
+ */
+mcs_status mcs_sparse_step_blocks(const void *Q, const void *K, const void *V, int B, int H, int N, int d, int G,
+                                  int block, int k_blocks, const int32_t *perm, const int32_t *pair_idx,
+                                  const int32_t *pair_len, const float *residual, float scale, void *O,
+                                  mcs_stream_t stream);
+
 /* Synchronise `stream`, then read and clear this device's status word.
  * Returns MCS_OK, or MCS_ERR_TIMEOUT if a kernel's bounded wait ran out
  * since the last read. */

@@ -5,6 +5,7 @@ package is its Python binding.  Import is cheap: the library is loaded on the
 first call.
 """
 from .api import (  # noqa: F401
+    BlockMeta,
     Meta,
     alloc_workspace,
     dense,
@@ -17,11 +18,14 @@ from .api import (  # noqa: F401
     plan_stats,
     plan_topk,
     pooled_scores,
+    select_block_indices,
     select_blocks,
     select_topk,
     selftest_wait_timeout,
     set_wait_limit_ns,
     sparse_step,
+    sparse_step_blocks,
+    union_pairs,
     validate_meta,
     workspace_size,
     workspace_views,

@@ -61,6 +61,10 @@ PROTOTYPES = {
     "mcs_select_blocks_workspace_size": (c_size_t, [c_int, c_int, c_int, c_int]),
     "mcs_select_blocks": (c_int, [c_vp, c_int, c_int, c_int, c_int, c_vp, c_vp, c_size_t, c_vp]),
     "mcs_pooled_scores": (c_int, [c_vp, c_vp, c_vp, c_int, c_int, c_int, c_int, c_int, c_float, c_vp, c_vp]),
+    "mcs_select_block_indices": (c_int, [c_vp, c_int, c_int, c_int, c_int, c_vp, c_vp, c_size_t, c_vp]),
+    "mcs_union_pairs": (c_int, [c_vp, c_int, c_int, c_int, c_int, c_vp, c_vp, c_vp]),
+    "mcs_sparse_step_blocks": (c_int, [c_vp, c_vp, c_vp, c_int, c_int, c_int, c_int, c_int, c_int, c_int,
+                                       c_vp, c_vp, c_vp, c_vp, c_float, c_vp, c_vp]),
     "mcs_last_device_status": (c_int, [c_vp]),
     "mcs_selftest_wait_timeout": (c_int, [c_u64, c_vp]),
     "mcs_set_wait_limit_ns": (None, [c_u64]),

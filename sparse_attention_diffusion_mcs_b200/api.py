@@ -341,6 +341,95 @@ def select_blocks(scores: torch.Tensor, k_blocks: int, block: int, out: Optional
     return out
 
 
+def select_block_indices(scores: torch.Tensor, k_blocks: int, block: int,
+                         out: Optional[torch.Tensor] = None) -> torch.Tensor:
+    """As `select_blocks`, but the kept blocks' indices ascending: int32
+    [..., k_blocks] (block b holds keys [b*block, (b+1)*block))."""
+    if scores.dtype != torch.float32 or not scores.is_cuda:
+        raise TypeError("scores must be a float32 CUDA tensor")
+    scores = scores.contiguous()
+    N = scores.shape[-1]
+    rows = scores.numel() // N if N else 0
+    if not 1 <= k_blocks <= N // block:
+        raise ValueError(f"k_blocks must be in [1, N // block] = [1, {N // block}]")
+    if out is None:
+        out = torch.empty((*scores.shape[:-1], k_blocks), dtype=torch.int32, device=scores.device)
+    else:
+        _check_tensor(out, "out", (*scores.shape[:-1], k_blocks), torch.int32, scores.device)
+    n = lib().mcs_select_blocks_workspace_size(rows, N, block, k_blocks)
+    ws = torch.empty(max(int(n), 1), dtype=torch.uint8, device=scores.device)
+    with _on(scores.device):
+        check(lib().mcs_select_block_indices(_ptr(scores), rows, N, block, k_blocks, _ptr(out), _ptr(ws),
+                                             ws.numel(), _stream(scores.device)), "mcs_select_block_indices")
+    return out
+
+
+def union_pairs(lists: torch.Tensor) -> Tuple[torch.Tensor, torch.Tensor]:
+    """Union lists of adjacent group pairs of ascending per-group lists
+    (int32 [B, H, n_groups, k], keys or block indices): (pair_idx int32
+    [B, H, n_pairs, 2k], pair_len int32 [B, H, n_pairs])."""
+    if lists.dtype != torch.int32 or not lists.is_cuda or lists.dim() != 4:
+        raise TypeError("lists must be an int32 CUDA tensor [B, H, n_groups, k]")
+    lists = lists.contiguous()
+    B, H, ng, k = lists.shape
+    np_ = (ng + 1) // 2
+    pair_idx = torch.empty((B, H, np_, 2 * k), dtype=torch.int32, device=lists.device)
+    pair_len = torch.empty((B, H, np_), dtype=torch.int32, device=lists.device)
+    with _on(lists.device):
+        check(lib().mcs_union_pairs(_ptr(lists), B, H, ng, k, _ptr(pair_idx), _ptr(pair_len),
+                                    _stream(lists.device)), "mcs_union_pairs")
+    return pair_idx, pair_len
+
+
+@dataclasses.dataclass
+class BlockMeta:
+    """A block-granular selection for `sparse_step_blocks`: the grouping, each
+    group's kept block indices, their pair union lists, an optional residual."""
+    G: int
+    block: int
+    perm: torch.Tensor                       # int32 [B, H, N]
+    blk_idx: torch.Tensor                    # int32 [B, H, n_groups, k_blocks], ascending
+    pair_idx: torch.Tensor                   # int32 [B, H, n_pairs, 2 k_blocks]
+    pair_len: torch.Tensor                   # int32 [B, H, n_pairs]
+    residual: Optional[torch.Tensor] = None  # float32 [B, H, N, d]
+
+    @property
+    def k_blocks(self) -> int:
+        return self.blk_idx.shape[3]
+
+    @staticmethod
+    def build(perm, blk_idx, G: int, block: int, residual: Optional[torch.Tensor] = None) -> "BlockMeta":
+        pair_idx, pair_len = union_pairs(blk_idx)
+        return BlockMeta(G, block, perm.contiguous(), blk_idx.contiguous(), pair_idx, pair_len,
+                         None if residual is None else residual.contiguous())
+
+
+def sparse_step_blocks(Q, K, V, bm: BlockMeta, scale: Optional[float] = None,
+                       out: Optional[torch.Tensor] = None) -> torch.Tensor:
+    """The reused step over a block-granular selection (blocks of 64 or 128
+    keys), with bm's residual added when it has one: bf16 O [B, H, N, d]."""
+    _check_qkv(Q, K, V)
+    B, H, N, d = Q.shape
+    ng = -(-N // bm.G)
+    np_ = (ng + 1) // 2
+    _check_tensor(bm.perm, "perm", (B, H, N), torch.int32, Q.device)
+    _check_tensor(bm.blk_idx, "blk_idx", (B, H, ng, bm.k_blocks), torch.int32, Q.device)
+    _check_tensor(bm.pair_idx, "pair_idx", (B, H, np_, 2 * bm.k_blocks), torch.int32, Q.device)
+    _check_tensor(bm.pair_len, "pair_len", (B, H, np_), torch.int32, Q.device)
+    if bm.residual is not None:
+        _check_tensor(bm.residual, "residual", (B, H, N, d), torch.float32, Q.device)
+    if out is None:
+        out = torch.empty_like(Q)
+    else:
+        _check_tensor(out, "out", Q.shape, torch.bfloat16, Q.device)
+    with _on(Q.device):
+        check(lib().mcs_sparse_step_blocks(_ptr(Q), _ptr(K), _ptr(V), B, H, N, d, bm.G, bm.block, bm.k_blocks,
+                                           _ptr(bm.perm), _ptr(bm.pair_idx), _ptr(bm.pair_len),
+                                           _ptr(bm.residual), _scale(d, scale), _ptr(out), _stream(Q.device)),
+              "mcs_sparse_step_blocks")
+    return out
+
+
 def pooled_scores(Q, K, perm, G: int, scale: Optional[float] = None,
                   out: Optional[torch.Tensor] = None) -> torch.Tensor:
     """Pooled-query scores (an ablation of exact summed probabilities):

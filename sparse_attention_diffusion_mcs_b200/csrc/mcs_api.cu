@@ -70,18 +70,21 @@ PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
   return fn;
 }
 
-// rows x D bf16 rows, box of one 64-column row (128 bytes): tile::gather4 source
-bool map_gather(CUtensorMap *m, const void *base, int D, size_t rows) {
+// rows x D bf16 rows, box of 64 columns (128 bytes) x box_rows rows; one
+// row: the tile::gather4 source, 64 rows: contiguous key tiles
+bool map_rows(CUtensorMap *m, const void *base, int D, size_t rows, unsigned box_rows) {
   auto fn = encode_fn();
   if (!fn) return false;
   const cuuint64_t dims[2] = {static_cast<cuuint64_t>(D), static_cast<cuuint64_t>(rows)};
   const cuuint64_t strides[1] = {static_cast<cuuint64_t>(D) * 2};
-  const cuuint32_t box[2] = {64, 1};
+  const cuuint32_t box[2] = {64, box_rows};
   const cuuint32_t es[2] = {1, 1};
   return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void *>(base), dims, strides, box, es,
             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
+
+bool map_gather(CUtensorMap *m, const void *base, int D, size_t rows) { return map_rows(m, base, D, rows, 1); }
 
 // [BH, N, D] bf16, box of 128 rows x 64 columns of one head: rows past N read as zero
 bool map_tile(CUtensorMap *m, const void *base, int D, int N, int BH) {
@@ -155,22 +158,25 @@ cudaError_t launch_attn_d(int d, AttnArgs &a, const QKV &t, int grid_x, int BH, 
 }
 
 // The sparse modes over pairs of groups sharing one union list of keys
-// (pair_kernel.cuh): persistent, one CTA per SM, items (head, pair).
-template <int D, int MODE>
+// (pair_kernel.cuh): persistent, one CTA per SM, items (head, pair).  With
+// BLOCK the lists hold block indices and K/V tiles are contiguous 64-row boxes.
+template <int D, int MODE, int BLOCK = 0>
 cudaError_t launch_pair(AttnArgs &a, const QKV &t, int BH, cudaStream_t s) {
   using C = PairCfg<D>;
   a.BH = BH;
   const size_t rows = static_cast<size_t>(BH) * a.N;
-  if (!(map_gather(&a.tmQ, t.Q, D, rows) && map_gather(&a.tmK, t.K, D, rows) && map_gather(&a.tmV, t.V, D, rows)))
+  const unsigned kv_box = BLOCK ? C::BN : 1;
+  if (!(map_gather(&a.tmQ, t.Q, D, rows) && map_rows(&a.tmK, t.K, D, rows, kv_box) &&
+        map_rows(&a.tmV, t.V, D, rows, kv_box)))
     return cudaErrorInvalidValue;
   const long items = static_cast<long>(BH) * a.n_pairs;
   if (items == 0) return cudaSuccess;
   cudaError_t e;
-  if ((e = set_smem(pair_kernel<D, MODE>, C::SMEM)) != cudaSuccess) return e;
+  if ((e = set_smem(pair_kernel<D, MODE, BLOCK>, C::SMEM)) != cudaSuccess) return e;
   int sms = 0;
   if ((e = sm_count(&sms)) != cudaSuccess) return e;
   const long grid = items < sms ? items : sms;
-  pair_kernel<D, MODE><<<static_cast<unsigned>(grid), C::THREADS, C::SMEM, s>>>(a);
+  pair_kernel<D, MODE, BLOCK><<<static_cast<unsigned>(grid), C::THREADS, C::SMEM, s>>>(a);
   return cudaGetLastError();
 }
 
@@ -707,6 +713,61 @@ mcs_status mcs_select_blocks(const float *scores, int rows, int N, int block, in
     expand_blocks_kernel<<<148 * 8, 256, 0, s>>>(blk, rows, k_blocks, block, kv_idx);
     e = cudaGetLastError();
   }
+  return cuda_status(e);
+}
+
+mcs_status mcs_select_block_indices(const float *scores, int rows, int N, int block, int k_blocks,
+                                    int32_t *blk_idx, void *workspace, size_t workspace_bytes,
+                                    mcs_stream_t stream) {
+  if (!scores || !blk_idx || rows < 0 || N < 1 || block < 1 || k_blocks < 1 || N / block < k_blocks)
+    return MCS_ERR_INVALID_ARG;
+  const size_t need = mcs_select_blocks_workspace_size(rows, N, block, k_blocks);
+  if (rows == 0) return MCS_OK;
+  mcs_status st = check_ws(workspace, workspace_bytes, need);
+  if (st != MCS_OK) return st;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  float *bs = static_cast<float *>(workspace);
+  block_sum_kernel<<<148 * 8, 256, 0, s>>>(scores, rows, N, block, bs);
+  cudaError_t e = cudaGetLastError();
+  if (e == cudaSuccess) e = launch_topk(bs, rows, N / block, k_blocks, blk_idx, s);
+  return cuda_status(e);
+}
+
+mcs_status mcs_union_pairs(const int32_t *lists, int B, int H, int n_groups, int k, int32_t *pair_idx,
+                           int32_t *pair_len, mcs_stream_t stream) {
+  if (!lists || !pair_idx || !pair_len || B < 0 || H < 0 || n_groups < 0 || k < 1) return MCS_ERR_INVALID_ARG;
+  if (static_cast<long long>(B) * H > 65535) return MCS_ERR_UNSUPPORTED;
+  return cuda_status(run_pairs(lists, B * H, n_groups, k, pair_idx, pair_len, reinterpret_cast<cudaStream_t>(stream)));
+}
+
+mcs_status mcs_sparse_step_blocks(const void *Q, const void *K, const void *V, int B, int H, int N, int d, int G,
+                                  int block, int k_blocks, const int32_t *perm, const int32_t *pair_idx,
+                                  const int32_t *pair_len, const float *residual, float scale, void *O,
+                                  mcs_stream_t stream) {
+  mcs_status st = check_common(Q, K, V, B, H, N, d, scale);
+  if (st != MCS_OK) return st;
+  if (!O || !aligned16(O) || !perm || !pair_idx || !pair_len) return MCS_ERR_INVALID_ARG;
+  if (residual && !aligned16(residual)) return MCS_ERR_INVALID_ARG;
+  if (!g_ok(G) || (block != 64 && block != 128)) return MCS_ERR_UNSUPPORTED;
+  if (k_blocks < 1 || k_blocks > N / block) return MCS_ERR_INVALID_ARG;
+  AttnArgs a = base_args(N, scale);
+  a.G = G;
+  a.k = k_blocks;
+  a.n_groups = (N + G - 1) / G;
+  a.perm = perm;
+  a.residual = residual;
+  a.O = static_cast<bf16 *>(O);
+  a.n_pairs = pairs_of(a.n_groups);
+  a.pair_idx = pair_idx;
+  a.pair_len = pair_len;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  const QKV t{Q, K, V};
+  const int BH = B * H;
+  cudaError_t e;
+  if (d == 64)
+    e = block == 64 ? launch_pair<64, kModeStep, 64>(a, t, BH, s) : launch_pair<64, kModeStep, 128>(a, t, BH, s);
+  else
+    e = block == 64 ? launch_pair<128, kModeStep, 64>(a, t, BH, s) : launch_pair<128, kModeStep, 128>(a, t, BH, s);
   return cuda_status(e);
 }
 

@@ -166,6 +166,15 @@ __device__ __forceinline__ void tma_gather4(uint32_t dst, const void *tmap, int 
       : "memory");
 }
 
+// One box of a 2D map at (column, row).
+__device__ __forceinline__ void tma_load_2d(uint32_t dst, const void *tmap, int c0, int c1, uint32_t bar) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
+      " [%0], [%1, {%2, %3}], [%4];" ::"r"(dst),
+      "l"(reinterpret_cast<uint64_t>(tmap)), "r"(c0), "r"(c1), "r"(bar)
+      : "memory");
+}
+
 // One box of a 3D map (box {64, 128, 1}): coordinates (column, row, head).
 __device__ __forceinline__ void tma_load_3d(uint32_t dst, const void *tmap, int c0, int c1, int c2, uint32_t bar) {
   asm volatile(

@@ -84,9 +84,16 @@ struct PairCfg {
 static_assert(PairCfg<128>::SMEM <= 232448 && PairCfg<64>::SMEM <= 232448, "shared memory budget");
 static_assert(PairCfg<128>::REG_SOFTMAX * 256 + PairCfg<128>::REG_OTHER * 256 <= 65536, "register split");
 
-template <int D, int MODE>
+// BLOCK = 0: the union lists hold individual keys, gathered row by row.
+// BLOCK = 64 or 128: they hold indices of aligned blocks of BLOCK keys (a
+// block-sparse selection, the comparison point of block-granular methods);
+// each 64-key tile is then one contiguous TMA tile load per column block, by
+// one lane, and no tile is partial.  Everything past the producers works in
+// key positions, so the rest of the kernel is the same.
+template <int D, int MODE, int BLOCK = 0>
 __global__ void __launch_bounds__(PairCfg<D>::THREADS, 1) pair_kernel(const __grid_constant__ AttnArgs a) {
   static_assert(MODE == kModeStep || MODE == kModePlanResid, "sparse modes only");
+  static_assert(BLOCK == 0 || BLOCK == 64 || BLOCK == 128, "blocks of 64 or 128 keys");
   using C = PairCfg<D>;
   constexpr int BM = C::BM, BN = C::BN, NK = C::NK, NV = C::NV;
   constexpr int NDB = D / 64;                       // 64-column (128-byte) blocks per row
@@ -121,7 +128,8 @@ __global__ void __launch_bounds__(PairCfg<D>::THREADS, 1) pair_kernel(const __gr
   const int warp = tid >> 5;
   const int lane = tid & 31;
   const int N = a.N;
-  const int kk = a.k;                 // keys per group, <= N
+  const int k_units = a.k;            // list entries per group: keys, or blocks
+  const int kk = BLOCK ? k_units * BLOCK : k_units;   // keys per group, <= N
   const int n_pairs = a.n_pairs;
   const int n_items = a.BH * n_pairs;
   const int a_tiles = (kk + BN - 1) / BN;   // group A's tiles: [0, a_tiles)
@@ -140,17 +148,17 @@ __global__ void __launch_bounds__(PairCfg<D>::THREADS, 1) pair_kernel(const __gr
     w.p = item % n_pairs;
     w.bh = item / n_pairs;
     w.head = static_cast<size_t>(w.bh) * N;
-    w.list = a.pair_idx + (static_cast<size_t>(w.bh) * n_pairs + w.p) * (2 * static_cast<size_t>(kk));
+    w.list = a.pair_idx + (static_cast<size_t>(w.bh) * n_pairs + w.p) * (2 * static_cast<size_t>(k_units));
     w.hasB = 2 * w.p + 1 < a.n_groups;
-    int u = a.pair_len[static_cast<size_t>(w.bh) * n_pairs + w.p];
-    const int umax = w.hasB ? 2 * kk : kk;
-    if (u < kk || u > umax) {   // corrupt metadata: never read past the list
+    int u = a.pair_len[static_cast<size_t>(w.bh) * n_pairs + w.p];   // list entries
+    const int umax = w.hasB ? 2 * k_units : k_units;
+    if (u < k_units || u > umax) {   // corrupt metadata: never read past the list
       record_status(a.status, kStatusBadMeta);
-      u = u < kk ? kk : umax;
+      u = u < k_units ? k_units : umax;
     }
-    w.u = u;
-    w.T = (u + BN - 1) / BN;
-    w.b0 = w.hasB ? (u - kk) / BN : w.T;
+    w.u = BLOCK ? u * BLOCK : u;     // union positions, in keys
+    w.T = (w.u + BN - 1) / BN;
+    w.b0 = w.hasB ? (w.u - kk) / BN : w.T;
     return w;
   };
   // query row r of block X (0: group 2p, 1: group 2p+1) -> token, or -1 for padding
@@ -252,7 +260,7 @@ __global__ void __launch_bounds__(PairCfg<D>::THREADS, 1) pair_kernel(const __gr
       int pre[R][4];
 #pragma unroll
       for (int s = 0; s < R; ++s)
-        if (active && s < w.T) tile_rows(s, pre[s]);
+        if (BLOCK == 0 && active && s < w.T) tile_rows(s, pre[s]);
       if (!is_k) {
         // each group's query block, once that group's last Q.K^T of its
         // previous item has read the buffer; the rows are looked up first
@@ -297,6 +305,34 @@ __global__ void __launch_bounds__(PairCfg<D>::THREADS, 1) pair_kernel(const __gr
         }
         if (!ok) break;
       }
+      if constexpr (BLOCK != 0) {
+        // contiguous blocks: one lane of the ring's first warp loads each
+        // 64-key tile as NDB tile boxes of 64 rows
+        for (int j = 0; j < w.T && ok && h == 0; ++j) {
+          const int slot = issued % NS;
+          int got = 1;
+          if (lane == 0)
+            got = mbar_wait(is_k ? b_kempty(slot) : b_vempty(slot), ((issued / NS) & 1) ^ 1, a.wait_ns,
+                            abort_flag);
+          got = __shfl_sync(0xffffffffu, got, 0);
+          if (!got) { ok = false; break; }
+          if (lane == 0) {
+            const uint32_t full = is_k ? b_kfull(slot) : b_vfull(slot);
+            const uint32_t dst = ring + slot * C::KV_BYTES;
+            int blk = w.list[(j * BN) / BLOCK];
+            if (static_cast<unsigned>(blk) >= static_cast<unsigned>(N / BLOCK)) {   // corrupt metadata
+              record_status(a.status, kStatusBadMeta);
+              blk = 0;
+            }
+            const int row = static_cast<int>(w.head) + blk * BLOCK + (j * BN) % BLOCK;
+            mbar_arrive_expect_tx(full, TILE_TX);
+#pragma unroll
+            for (int db = 0; db < NDB; ++db) tma_load_2d(dst + db * (BN * 128), tm, db * 64, row, full);
+          }
+          __syncwarp();
+          ++issued;
+        }
+      } else {
       for (int jb = 0; jb < w.T && ok; jb += R) {
 #pragma unroll
         for (int s = 0; s < R; ++s) {
@@ -321,6 +357,7 @@ __global__ void __launch_bounds__(PairCfg<D>::THREADS, 1) pair_kernel(const __gr
           }
           ++issued;
         }
+      }
       }
       w = wn;
     }
@@ -449,6 +486,7 @@ __global__ void __launch_bounds__(PairCfg<D>::THREADS, 1) pair_kernel(const __gr
     const float sl2 = a.scale_log2;
     // the epilogue's second input (residual, or the dense output), per row
     const float *ep_in = MODE == kModeStep ? a.residual : a.O32_in;
+    const bool has_res = ep_in != nullptr;   // a reused step may add no residual (a block-sparse comparison)
     bool ok = true;
     int c = 0;       // this group's tiles so far (S buffer, barrier phases)
     for (int item = blockIdx.x; item < n_items && ok; item += gridDim.x) {
@@ -456,7 +494,7 @@ __global__ void __launch_bounds__(PairCfg<D>::THREADS, 1) pair_kernel(const __gr
       if (X == 1 && !w.hasB) continue;
       const int q = q_check(q_raw(w, X, r));
       const size_t row = (w.head + (q >= 0 ? q : 0)) * D;
-      if (q >= 0) {   // pull the epilogue row into L2 well before it is read
+      if (q >= 0 && has_res) {   // pull the epilogue row into L2 well before it is read
 #pragma unroll
         for (int cc = 0; cc < D / 32; ++cc) asm volatile("prefetch.global.L2 [%0];" ::"l"(ep_in + row + cc * 32));
       }
@@ -540,7 +578,7 @@ __global__ void __launch_bounds__(PairCfg<D>::THREADS, 1) pair_kernel(const __gr
       // the epilogue input of the first chunk is in flight while the last P.V runs
       constexpr int EC = 16;   // epilogue chunk (columns)
       float4 ein[EC / 4];
-      if (q >= 0) {
+      if (q >= 0 && has_res) {
         const float4 *src = reinterpret_cast<const float4 *>(ep_in + row);
 #pragma unroll
         for (int u = 0; u < EC / 4; ++u) ein[u] = __ldg(src + u);
@@ -556,7 +594,7 @@ __global__ void __launch_bounds__(PairCfg<D>::THREADS, 1) pair_kernel(const __gr
 #pragma unroll 1
       for (int cc = 0; cc < D / EC; ++cc) {
         float4 enx[EC / 4];   // next chunk's input in flight while this chunk is finished
-        if (q >= 0 && cc + 1 < D / EC) {
+        if (q >= 0 && has_res && cc + 1 < D / EC) {
           const float4 *src = reinterpret_cast<const float4 *>(ep_in + row + (cc + 1) * EC);
 #pragma unroll
           for (int u = 0; u < EC / 4; ++u) enx[u] = __ldg(src + u);
@@ -569,7 +607,7 @@ __global__ void __launch_bounds__(PairCfg<D>::THREADS, 1) pair_kernel(const __gr
           for (int i = 0; i < EC; ++i) o[i] *= inv_l;
           if (MODE == kModeStep) {
 #pragma unroll
-            for (int u = 0; u < EC / 4; ++u) {
+            for (int u = 0; u < EC / 4 && has_res; ++u) {
               o[4 * u + 0] += ein[u].x;
               o[4 * u + 1] += ein[u].y;
               o[4 * u + 2] += ein[u].z;

@@ -13,6 +13,7 @@ from .dit_inputs import (
     layer_tensors,
     drift_head,
     drift_layer,
+    random_blocks_head,
     random_metadata_head,
     random_qkv,
     rising_qkv,
@@ -21,5 +22,5 @@ from .dit_inputs import (
 __all__ = [
     "WORKLOADS", "Workload", "workload", "sweep_points",
     "bf16_round", "head_tensors", "layer_tensors", "drift_head", "drift_layer",
-    "random_metadata_head", "random_qkv", "rising_qkv",
+    "random_blocks_head", "random_metadata_head", "random_qkv", "rising_qkv",
 ]

@@ -32,6 +32,7 @@ from .workloads import Workload
 _PURPOSE_BASE = 0
 _PURPOSE_DRIFT = 1
 _PURPOSE_META = 2
+_PURPOSE_BLOCKS = 3
 
 
 def _rng(w: Workload, *key: int) -> np.random.Generator:
@@ -176,6 +177,18 @@ def random_metadata_head(w: Workload, bh: int, r_scale: float = 0.1):
         kv[g] = np.sort(rng.choice(N, size=k, replace=False)).astype(np.int32)
     res = (r_scale * rng.standard_normal((N, w.d))).astype(np.float32)
     return perm, kv, res
+
+
+def random_blocks_head(w: Workload, bh: int, block: int, k_blocks: int):
+    """Arbitrary valid block selections for one head: for each query group
+    k_blocks sorted unique block indices in [0, N // block) (block b holds
+    keys [b*block, (b+1)*block)).  Returns int32 [n_groups, k_blocks]."""
+    rng = _rng(w, _PURPOSE_BLOCKS, block, k_blocks, bh)
+    nb = w.N // block
+    out = np.empty((w.n_groups, k_blocks), np.int32)
+    for g in range(w.n_groups):
+        out[g] = np.sort(rng.choice(nb, size=k_blocks, replace=False)).astype(np.int32)
+    return out
 
 
 def random_qkv(B: int, H: int, N: int, d: int, seed: int = 0, q_std: float = 1.0):

@@ -168,3 +168,26 @@ def test_ablation_tool_argument_errors(L):
     assert L.mcs_pooled_scores(FAKE, FAKE, None, 1, 1, 128, 64, 64, 0.125, FAKE, s) == INVALID
     assert L.mcs_pooled_scores(FAKE, FAKE, FAKE, 1, 1, 128, 64, 32, 0.125, FAKE, s) == UNSUPPORTED
     assert L.mcs_pooled_scores(FAKE, FAKE, FAKE, 1, 1, 128, 96, 64, 0.125, FAKE, s) == UNSUPPORTED
+
+
+def test_block_step_argument_errors(L):
+    s = None
+    assert L.mcs_select_block_indices(None, 4, 1000, 64, 2, FAKE, FAKE, 1 << 20, s) == INVALID
+    assert L.mcs_select_block_indices(FAKE, 4, 1000, 64, 16, FAKE, FAKE, 1 << 20, s) == INVALID
+    assert L.mcs_select_block_indices(FAKE, 4, 1000, 64, 2, FAKE, FAKE, 8, s) == WORKSPACE
+    assert L.mcs_union_pairs(None, 1, 1, 4, 8, FAKE, FAKE, s) == INVALID
+    assert L.mcs_union_pairs(FAKE, 1, 1, 4, 0, FAKE, FAKE, s) == INVALID
+    assert L.mcs_union_pairs(FAKE, 256, 257, 4, 8, FAKE, FAKE, s) == UNSUPPORTED
+    args = lambda **kw: dict(dict(B=1, H=2, N=1024, d=128, G=128, block=64, kb=4, perm=FAKE, pidx=FAKE,
+                                  plen=FAKE, res=None, scale=0.125, O=FAKE), **kw)
+    step = lambda a: L.mcs_sparse_step_blocks(FAKE, FAKE, FAKE, a["B"], a["H"], a["N"], a["d"], a["G"], a["block"],
+                                             a["kb"], a["perm"], a["pidx"], a["plen"], a["res"], a["scale"], a["O"], s)
+    assert step(args(block=32)) == UNSUPPORTED
+    assert step(args(G=96)) == UNSUPPORTED
+    assert step(args(kb=0)) == INVALID
+    assert step(args(kb=17)) == INVALID                   # only 16 blocks of 64 in 1024 keys
+    assert step(args(block=128, kb=9)) == INVALID
+    assert step(args(perm=None)) == INVALID
+    assert step(args(pidx=None)) == INVALID
+    assert step(args(res=FAKE + 4)) == INVALID   # a residual must be 16-byte aligned
+    assert step(args(scale=0.0)) == INVALID
