@@ -455,7 +455,8 @@ def run_ablate(args):
 
 def run_blocks(args):
     """--blocks: block-granular against token-granular selection on one layer
-    of the workload, planned on step 1 and reused on step 2.  For blocks of 64
+    of the workload, planned on step 1 and reused on step 2 (and the token
+    step with its residual stored as bf16).  For blocks of 64
     and 128 keys at kb = k // block blocks per group, and for token selection
     at the same key budget kb * block, time the reused step (block step: one
     TMA tile load per 64 keys; token step: row gathers) and report its rel-L2
@@ -512,6 +513,10 @@ def run_blocks(args):
                           "device_status": mcs.last_device_status()}), flush=True)
 
     report("token", min(k, N), lambda out: mcs.sparse_step(Q2, K2, V2, meta, w.scale, out=out), meta.residual)
+    r16 = mcs.compact_residual(meta.residual)
+    report("token, bf16 residual", min(k, N),
+           lambda out: mcs.sparse_step_compact(Q2, K2, V2, meta, r16, w.scale, out=out), r16.float())
+    del r16
     for block in (64, 128):
         kb = k // block
         if kb < 1 or N // block < kb:

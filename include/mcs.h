@@ -215,6 +215,27 @@ mcs_status mcs_sparse_step(const void *Q, const void *K, const void *V, const mc
                            float scale, void *O, mcs_stream_t stream);
 
 /*
+ * mcs_residual_compact -- the cached residual stored compactly: bf16 copy
+ * residual_bf16[i] = round-to-nearest-even(residual[i]) of n float32 values
+ * (e.g. n = B*H*N*d for meta->residual).  Both pointers 16-byte aligned
+ * device memory (INVALID_ARG otherwise); n = 0 is a no-op.  Asynchronous.
+ * The bf16 copy holds each value to 2^-9 relative; it halves what the reused
+ * step reads per row and what a cached plan keeps per token.
+ */
+mcs_status mcs_residual_compact(const float *residual, size_t n, void *residual_bf16, mcs_stream_t stream);
+
+/*
+ * mcs_sparse_step_compact -- mcs_sparse_step with the residual read from a
+ * bf16 copy (mcs_residual_compact, bf16 [B,H,N,d]) instead of
+ * meta->residual, which is not read and may be NULL.  Needs the pair lists
+ * (meta->pair_idx / ->pair_len; INVALID_ARG without them).  The result equals
+ * mcs_sparse_step's on a residual whose values are the bf16 copy's.
+ * Asynchronous; needs no workspace.
+ */
+mcs_status mcs_sparse_step_compact(const void *Q, const void *K, const void *V, const mcs_meta *meta,
+                                   const void *residual_bf16, float scale, void *O, mcs_stream_t stream);
+
+/*
  * mcs_dense -- step a7, dense attention O = softmax(scale Q K^T) V, the
  * comparison baseline the pages measure against ("relative to dense
  * attention", aiqbench.com abstract).  O: bf16 [B,H,N,d].

@@ -49,6 +49,7 @@ __all__ = [
     "sparse_attention", "residual_group", "plan_head", "reused_step_head",
     "rel_l2", "schedule_head",
     "select_blocks", "pooled_scores", "ungrouped_rows", "retained_mass",
+    "round_bf16",
 ]
 
 
@@ -56,6 +57,39 @@ def widen_bf16(u16: np.ndarray) -> np.ndarray:
     """bf16 bit patterns (uint16) -> float64, exactly."""
     u = np.asarray(u16, dtype=np.uint16)
     return (u.astype(np.uint32) << np.uint32(16)).view(np.float32).astype(np.float64)
+
+
+def round_bf16(x) -> np.ndarray:
+    """float32 values -> bf16 bit patterns (uint16), IEEE round to nearest,
+    ties to even: of the two bf16 values bracketing x (x's float32 bits with
+    the low 16 bits cleared, and the next bf16 away from zero) take the nearer;
+    on a tie the one whose last mantissa bit is 0.  Magnitudes that round past
+    the largest finite bf16 become infinity (the bracket above it counts as
+    2^128, as in an unbounded exponent range).  NaN -> a quiet NaN.  (The
+    storage format of the compact cached residual, a reading of this library,
+    not of the pages.)"""
+    with np.errstate(invalid="ignore"):
+        return _round_bf16(np.ascontiguousarray(np.asarray(x, dtype=np.float32)))
+
+
+def _round_bf16(x32: np.ndarray) -> np.ndarray:
+    bits = x32.view(np.uint32)
+    lo = (bits >> np.uint32(16)).astype(np.uint32)      # toward zero
+    hi = lo + np.uint32(1)                               # away from zero
+    mag = np.abs(x32.astype(np.float64))
+    lo_v = np.abs(widen_bf16(lo.astype(np.uint16)))
+    hi_exp_all_ones = (hi & np.uint32(0x7F80)) == np.uint32(0x7F80)
+    hi_v = np.where(hi_exp_all_ones, 2.0 ** 128,
+                    np.abs(widen_bf16((hi & np.uint32(0xFFFF)).astype(np.uint16))))
+    d_lo, d_hi = mag - lo_v, hi_v - mag
+    take_hi = (d_hi < d_lo) | ((d_hi == d_lo) & ((lo & np.uint32(1)) == np.uint32(1)))
+    exact = d_lo == 0.0
+    out = np.where(take_hi & ~exact, hi, lo).astype(np.uint32)
+    inf_or_nan = (bits & np.uint32(0x7F800000)) == np.uint32(0x7F800000)
+    out = np.where(inf_or_nan, lo, out)                  # infinities are exact
+    nan = np.isnan(x32)
+    out = np.where(nan, np.uint32(0x7FC0), out)
+    return (out & np.uint32(0xFFFF)).astype(np.uint16)
 
 
 def _as_f64(x) -> np.ndarray:

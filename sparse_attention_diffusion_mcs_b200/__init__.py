@@ -8,6 +8,7 @@ from .api import (  # noqa: F401
     BlockMeta,
     Meta,
     alloc_workspace,
+    compact_residual,
     dense,
     last_device_status,
     plan,
@@ -25,6 +26,7 @@ from .api import (  # noqa: F401
     set_wait_limit_ns,
     sparse_step,
     sparse_step_blocks,
+    sparse_step_compact,
     union_pairs,
     validate_meta,
     workspace_size,

@@ -55,6 +55,8 @@ PROTOTYPES = {
     "mcs_meta_pairs": (c_int, [PMETA, c_vp]),
     "mcs_sparse_step": (c_int, [c_vp, c_vp, c_vp, PMETA, c_float, c_vp, c_vp]),
     "mcs_dense": (c_int, [c_vp, c_vp, c_vp, c_int, c_int, c_int, c_int, c_float, c_vp, c_vp]),
+    "mcs_residual_compact": (c_int, [c_vp, c_size_t, c_vp, c_vp]),
+    "mcs_sparse_step_compact": (c_int, [c_vp, c_vp, c_vp, PMETA, c_vp, c_float, c_vp, c_vp]),
     "mcs_validate_workspace_size": (c_size_t, [c_int, c_int, c_int]),
     "mcs_validate_meta": (c_int, [PMETA, c_vp, c_size_t, ctypes.POINTER(c_int), c_vp]),
     "mcs_validate_meta_noalloc": (c_int, [PMETA, ctypes.POINTER(c_int), c_vp]),

@@ -506,6 +506,44 @@ def sparse_step(Q, K, V, meta: Meta, scale: Optional[float] = None,
     return out
 
 
+def compact_residual(residual: torch.Tensor, out: Optional[torch.Tensor] = None) -> torch.Tensor:
+    """The cached residual as bf16 (round to nearest even), same shape: half
+    the bytes the reused step reads and a cached plan keeps."""
+    if residual.dtype != torch.float32 or not residual.is_cuda:
+        raise TypeError("residual must be a float32 CUDA tensor")
+    residual = residual.contiguous()
+    if out is None:
+        out = torch.empty(residual.shape, dtype=torch.bfloat16, device=residual.device)
+    else:
+        _check_tensor(out, "out", residual.shape, torch.bfloat16, residual.device)
+    with _on(residual.device):
+        check(lib().mcs_residual_compact(_ptr(residual), residual.numel(), _ptr(out), _stream(residual.device)),
+              "mcs_residual_compact")
+    return out
+
+
+def sparse_step_compact(Q, K, V, meta: Meta, residual16: torch.Tensor, scale: Optional[float] = None,
+                        out: Optional[torch.Tensor] = None) -> torch.Tensor:
+    """The reused step with the residual read from its bf16 copy
+    (`compact_residual`) instead of meta.residual: bf16 O [B, H, N, d].
+    Needs meta's pair lists."""
+    _check_qkv(Q, K, V)
+    _check_meta(meta, *Q.shape, Q.device)
+    if meta.pair_idx is None:
+        raise ValueError("the compact-residual step needs the metadata's pair lists (Meta.build_pairs)")
+    _check_tensor(residual16, "residual16", Q.shape, torch.bfloat16, Q.device)
+    if out is None:
+        out = torch.empty_like(Q)
+    else:
+        _check_tensor(out, "out", Q.shape, torch.bfloat16, Q.device)
+    cm = meta.c_struct()
+    with _on(Q.device):
+        check(lib().mcs_sparse_step_compact(_ptr(Q), _ptr(K), _ptr(V), ctypes.byref(cm), _ptr(residual16),
+                                            _scale(meta.d, scale), _ptr(out), _stream(Q.device)),
+              "mcs_sparse_step_compact")
+    return out
+
+
 def dense(Q, K, V, scale: Optional[float] = None, out: Optional[torch.Tensor] = None) -> torch.Tensor:
     """Dense attention (a7): bf16 O [B, H, N, d]."""
     _check_qkv(Q, K, V)

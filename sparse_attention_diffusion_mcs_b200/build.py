@@ -13,7 +13,7 @@ MICRO_LIB_PATH = os.path.join(PKG_DIR, "libmcs_micro.so")
 SOURCES = ["mcs_api.cu"]
 MICRO_SOURCES = ["micro_gather.cu"]
 HEADERS = ["mcs_common.cuh", "ablation_kernels.cuh", "attn_kernel.cuh", "attn_dual_kernel.cuh", "pair_kernel.cuh", "colsum_kernel.cuh", "topk_kernel.cuh",
-           "group_kernels.cuh", "validate_kernels.cuh"]
+           "group_kernels.cuh", "validate_kernels.cuh", "residual_compact.cuh"]
 NVCC_FLAGS = [
     "-gencode", "arch=compute_100a,code=sm_100a",
     "-O3", "-lineinfo", "-std=c++17",

@@ -67,6 +67,7 @@ struct alignas(64) AttnArgs {
   const int32_t *pair_idx; // [BH, n_pairs, 2k]     pair kernel: union list of groups 2p, 2p+1
   const int32_t *pair_len; // [BH, n_pairs]         pair kernel: union sizes
   int n_pairs;             // ceil(n_groups / 2)
+  const bf16 *residual16;  // [BH, N, D] bf16       pair kernel, kModeStep: compact residual (replaces residual)
 };
 
 template <int D, int MODE>

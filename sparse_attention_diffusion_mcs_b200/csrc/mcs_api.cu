@@ -14,6 +14,7 @@
 #include "colsum_kernel.cuh"
 #include "group_kernels.cuh"
 #include "pair_kernel.cuh"
+#include "residual_compact.cuh"
 #include "topk_kernel.cuh"
 #include "validate_kernels.cuh"
 
@@ -595,6 +596,46 @@ mcs_status mcs_sparse_step(const void *Q, const void *K, const void *V, const mc
     return cuda_status(launch_pair_d<kModeStep>(meta->d, a, QKV{Q, K, V}, meta->B * meta->H, s));
   }
   return cuda_status(launch_attn_d<kModeStep>(meta->d, a, QKV{Q, K, V}, meta->n_groups, meta->B * meta->H, s));
+}
+
+mcs_status mcs_residual_compact(const float *residual, size_t n, void *residual_bf16, mcs_stream_t stream) {
+  if (n == 0) return MCS_OK;
+  if (!residual || !residual_bf16 || !aligned16(residual) || !aligned16(residual_bf16)) return MCS_ERR_INVALID_ARG;
+  int sms = 0;
+  cudaError_t e = sm_count(&sms);
+  if (e != cudaSuccess) return cuda_status(e);
+  const size_t want = (n / 8 + kCompactThreads - 1) / kCompactThreads;
+  const size_t cap = static_cast<size_t>(sms) * 8;
+  const unsigned grid = static_cast<unsigned>(want < 1 ? 1 : (want < cap ? want : cap));
+  residual_compact_kernel<<<grid, kCompactThreads, 0, reinterpret_cast<cudaStream_t>(stream)>>>(
+      residual, n, static_cast<bf16 *>(residual_bf16));
+  return cuda_status(cudaGetLastError());
+}
+
+mcs_status mcs_sparse_step_compact(const void *Q, const void *K, const void *V, const mcs_meta *meta,
+                                   const void *residual_bf16, float scale, void *O, mcs_stream_t stream) {
+  if (!meta) return MCS_ERR_INVALID_ARG;
+  mcs_status st = check_common(Q, K, V, meta->B, meta->H, meta->N, meta->d, scale);
+  if (st != MCS_OK) return st;
+  if (!O || !aligned16(O) || !meta->perm || !meta->kv_idx || !residual_bf16 || !aligned16(residual_bf16))
+    return MCS_ERR_INVALID_ARG;
+  if (!meta->pair_idx || !meta->pair_len) return MCS_ERR_INVALID_ARG;
+  if (!g_ok(meta->G)) return MCS_ERR_UNSUPPORTED;
+  if (meta->k < 1 || meta->k > meta->N || meta->n_groups != (meta->N + meta->G - 1) / meta->G)
+    return MCS_ERR_INVALID_ARG;
+  AttnArgs a = base_args(meta->N, scale);
+  a.G = meta->G;
+  a.k = meta->k;
+  a.n_groups = meta->n_groups;
+  a.perm = meta->perm;
+  a.kv_idx = meta->kv_idx;
+  a.residual16 = static_cast<const bf16 *>(residual_bf16);
+  a.O = static_cast<bf16 *>(O);
+  a.n_pairs = pairs_of(meta->n_groups);
+  a.pair_idx = meta->pair_idx;
+  a.pair_len = meta->pair_len;
+  return cuda_status(launch_pair_d<kModeStep>(meta->d, a, QKV{Q, K, V}, meta->B * meta->H,
+                                              reinterpret_cast<cudaStream_t>(stream)));
 }
 
 mcs_status mcs_dense(const void *Q, const void *K, const void *V, int B, int H, int N, int d, float scale,

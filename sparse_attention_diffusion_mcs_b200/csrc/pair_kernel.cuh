@@ -486,7 +486,26 @@ __global__ void __launch_bounds__(PairCfg<D>::THREADS, 1) pair_kernel(const __gr
     const float sl2 = a.scale_log2;
     // the epilogue's second input (residual, or the dense output), per row
     const float *ep_in = MODE == kModeStep ? a.residual : a.O32_in;
-    const bool has_res = ep_in != nullptr;   // a reused step may add no residual (a block-sparse comparison)
+    // or a compact (bf16) residual; a reused step may add none (a block-sparse comparison)
+    const bf16 *ep16 = MODE == kModeStep ? a.residual16 : nullptr;
+    const bool has_res = ep_in != nullptr || ep16 != nullptr;
+    constexpr int EC = 16;   // epilogue chunk (columns)
+    // chunk cc of this row's epilogue input: 4 float4 of fp32, or (compact)
+    // the 2 uint4 of its 16 bf16 values carried bit for bit in e[0], e[1]
+    auto load_in = [&](size_t row, int cc, float4 (&e)[EC / 4]) {
+      if (ep16 != nullptr) {
+        const uint4 *src = reinterpret_cast<const uint4 *>(ep16 + row + cc * EC);
+#pragma unroll
+        for (int u = 0; u < EC / 8; ++u) {
+          const uint4 t = __ldg(src + u);
+          e[u] = make_float4(__uint_as_float(t.x), __uint_as_float(t.y), __uint_as_float(t.z), __uint_as_float(t.w));
+        }
+      } else {
+        const float4 *src = reinterpret_cast<const float4 *>(ep_in + row + cc * EC);
+#pragma unroll
+        for (int u = 0; u < EC / 4; ++u) e[u] = __ldg(src + u);
+      }
+    };
     bool ok = true;
     int c = 0;       // this group's tiles so far (S buffer, barrier phases)
     for (int item = blockIdx.x; item < n_items && ok; item += gridDim.x) {
@@ -495,8 +514,13 @@ __global__ void __launch_bounds__(PairCfg<D>::THREADS, 1) pair_kernel(const __gr
       const int q = q_check(q_raw(w, X, r));
       const size_t row = (w.head + (q >= 0 ? q : 0)) * D;
       if (q >= 0 && has_res) {   // pull the epilogue row into L2 well before it is read
+        if (ep16 != nullptr) {
 #pragma unroll
-        for (int cc = 0; cc < D / 32; ++cc) asm volatile("prefetch.global.L2 [%0];" ::"l"(ep_in + row + cc * 32));
+          for (int cc = 0; cc < D / 64; ++cc) asm volatile("prefetch.global.L2 [%0];" ::"l"(ep16 + row + cc * 64));
+        } else {
+#pragma unroll
+          for (int cc = 0; cc < D / 32; ++cc) asm volatile("prefetch.global.L2 [%0];" ::"l"(ep_in + row + cc * 32));
+        }
       }
       const int j0 = X == 0 ? 0 : w.b0;
       const int j1 = X == 0 ? a_tiles : w.T;
@@ -576,13 +600,8 @@ __global__ void __launch_bounds__(PairCfg<D>::THREADS, 1) pair_kernel(const __gr
       }
       if (!ok) break;
       // the epilogue input of the first chunk is in flight while the last P.V runs
-      constexpr int EC = 16;   // epilogue chunk (columns)
       float4 ein[EC / 4];
-      if (q >= 0 && has_res) {
-        const float4 *src = reinterpret_cast<const float4 *>(ep_in + row);
-#pragma unroll
-        for (int u = 0; u < EC / 4; ++u) ein[u] = __ldg(src + u);
-      }
+      if (q >= 0 && has_res) load_in(row, 0, ein);
       // O is final once this item's last two P.V of the group have completed
       // (the earlier ones completed before the last S this group has seen)
       for (int t = (j1 - j0 >= 2 ? c - 2 : c - 1); t < c && ok; ++t)
@@ -594,11 +613,7 @@ __global__ void __launch_bounds__(PairCfg<D>::THREADS, 1) pair_kernel(const __gr
 #pragma unroll 1
       for (int cc = 0; cc < D / EC; ++cc) {
         float4 enx[EC / 4];   // next chunk's input in flight while this chunk is finished
-        if (q >= 0 && has_res && cc + 1 < D / EC) {
-          const float4 *src = reinterpret_cast<const float4 *>(ep_in + row + (cc + 1) * EC);
-#pragma unroll
-          for (int u = 0; u < EC / 4; ++u) enx[u] = __ldg(src + u);
-        }
+        if (q >= 0 && has_res && cc + 1 < D / EC) load_in(row, cc + 1, enx);
         float o[EC];
         tmem_ld16(tO + cc * EC, o);
         tmem_wait_ld();
@@ -606,12 +621,25 @@ __global__ void __launch_bounds__(PairCfg<D>::THREADS, 1) pair_kernel(const __gr
 #pragma unroll
           for (int i = 0; i < EC; ++i) o[i] *= inv_l;
           if (MODE == kModeStep) {
+            if (ep16 != nullptr) {
 #pragma unroll
-            for (int u = 0; u < EC / 4 && has_res; ++u) {
-              o[4 * u + 0] += ein[u].x;
-              o[4 * u + 1] += ein[u].y;
-              o[4 * u + 2] += ein[u].z;
-              o[4 * u + 3] += ein[u].w;
+              for (int u = 0; u < EC / 8; ++u) {
+                const uint32_t wv[4] = {__float_as_uint(ein[u].x), __float_as_uint(ein[u].y),
+                                        __float_as_uint(ein[u].z), __float_as_uint(ein[u].w)};
+#pragma unroll
+                for (int e = 0; e < 4; ++e) {   // element 2e in the low half, 2e + 1 in the high half
+                  o[8 * u + 2 * e] += __uint_as_float(wv[e] << 16);
+                  o[8 * u + 2 * e + 1] += __uint_as_float(wv[e] & 0xFFFF0000u);
+                }
+              }
+            } else if (has_res) {
+#pragma unroll
+              for (int u = 0; u < EC / 4; ++u) {
+                o[4 * u + 0] += ein[u].x;
+                o[4 * u + 1] += ein[u].y;
+                o[4 * u + 2] += ein[u].z;
+                o[4 * u + 3] += ein[u].w;
+              }
             }
             uint4 *op = reinterpret_cast<uint4 *>(a.O + row + cc * EC);
 #pragma unroll

@@ -191,3 +191,18 @@ def test_block_step_argument_errors(L):
     assert step(args(pidx=None)) == INVALID
     assert step(args(res=FAKE + 4)) == INVALID   # a residual must be 16-byte aligned
     assert step(args(scale=0.0)) == INVALID
+
+
+def test_compact_residual_argument_errors(L):
+    s = None
+    assert L.mcs_residual_compact(None, 0, None, s) == OK                  # nothing to convert
+    assert L.mcs_residual_compact(None, 8, FAKE, s) == INVALID
+    assert L.mcs_residual_compact(FAKE, 8, FAKE + 2, s) == INVALID         # misaligned output
+    m = _lib.McsMeta()
+    assert L.mcs_meta_init(ctypes.byref(m), 1, 2, 1024, 64, 64, 128) == OK
+    m.perm, m.kv_idx = FAKE, FAKE
+    assert L.mcs_sparse_step_compact(FAKE, FAKE, FAKE, ctypes.byref(m), FAKE, 0.125, FAKE, s) == INVALID  # no pairs
+    m.pair_idx, m.pair_len = FAKE, FAKE
+    assert L.mcs_sparse_step_compact(FAKE, FAKE, FAKE, ctypes.byref(m), None, 0.125, FAKE, s) == INVALID
+    assert L.mcs_sparse_step_compact(FAKE, FAKE, FAKE, ctypes.byref(m), FAKE + 8, 0.125, FAKE, s) == INVALID
+    assert L.mcs_sparse_step_compact(FAKE, FAKE, FAKE, None, FAKE, 0.125, FAKE, s) == INVALID

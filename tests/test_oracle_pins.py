@@ -394,3 +394,53 @@ def test_retained_mass_closed_forms():
     idx = orc.select_kv(c, 4)
     other = np.setdiff1d(np.arange(12), idx)
     assert abs(orc.retained_mass(c, idx, 5) + orc.retained_mass(c, other, 5) - 1.0) < 1e-14
+
+
+# --------------------------------------------------------------------------- compact residual storage
+
+def _all_finite_bf16():
+    u = np.arange(65536, dtype=np.uint32).astype(np.uint16)
+    with np.errstate(invalid="ignore"):
+        v = orc.widen_bf16(u)
+    keep = np.isfinite(v)
+    return u[keep], v[keep]
+
+
+def test_round_bf16_is_the_nearest_bf16_value_by_exhaustive_search():
+    """Every sample against all 65280 finite bf16 values: the result is at
+    minimal distance; among two at equal distance, the even-mantissa one."""
+    rng = np.random.default_rng(11)
+    bits = rng.integers(0, 2 ** 32, size=1500, dtype=np.uint64).astype(np.uint32)
+    ties = (bits[:500] & np.uint32(0xFFFF0000)) | np.uint32(0x8000)     # exactly half-way cases
+    x = np.concatenate([bits, ties]).view(np.float32)
+    x = x[np.isfinite(x)]
+    x = x[np.abs(x.astype(np.float64)) < 3.38e38]
+    got = orc.round_bf16(x)
+    u_all, v_all = _all_finite_bf16()
+    for chunk in np.array_split(np.arange(len(x)), 20):
+        xs = x[chunk].astype(np.float64)
+        dist = np.abs(xs[:, None] - v_all[None, :])
+        best = dist.min(axis=1)
+        g = orc.widen_bf16(got[chunk])
+        assert np.array_equal(np.abs(xs - g), best)
+        for i, row in zip(chunk, dist):
+            cands = u_all[row == row.min()]
+            cands = cands[~((cands == 0x8000) & (x[i] >= 0)) & ~((cands == 0) & (x[i] < 0))]  # signed zero of x
+            if len(cands) > 1:          # a tie: the even mantissa wins
+                even = cands[(cands & 1) == 0]
+                assert got[i] in even, (x[i], cands, got[i])
+
+
+def test_round_bf16_keeps_bf16_values_and_special_values():
+    u_all, v_all = _all_finite_bf16()
+    assert np.array_equal(orc.round_bf16(v_all.astype(np.float32)), u_all)      # every bf16 value is kept
+    assert orc.round_bf16(np.float32(np.inf))[()] == 0x7F80
+    assert orc.round_bf16(np.float32(-np.inf))[()] == 0xFF80
+    assert np.isnan(orc.widen_bf16(orc.round_bf16(np.float32(np.nan))))
+    top = orc.widen_bf16(np.uint16(0x7F7F))                 # largest finite bf16, odd mantissa
+    half_ulp = 2.0 ** (127 - 8)
+    assert orc.round_bf16(np.float32(top + half_ulp))[()] == 0x7F80               # the tie goes to even: infinity
+    assert orc.round_bf16(np.nextafter(np.float32(top + half_ulp), np.float32(0)))[()] == 0x7F7F
+    assert orc.round_bf16(np.float32(1.0 + 2.0 ** -8))[()] == 0x3F80               # tie between 1 and 1 + 2^-7
+    assert orc.round_bf16(np.float32(1.0 + 3 * 2.0 ** -8))[()] == 0x3F82           # tie: 1 + 2^-6 is even
+    assert orc.round_bf16(np.float32(-(1.0 + 2.0 ** -8)))[()] == 0xBF80
