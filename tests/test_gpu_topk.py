@@ -6,9 +6,12 @@ select_kv (ties to the lower key index, output ascending):
     threshold, equal keys spread over many warps' slices);
   * constant rows and all-zero rows (the candidate list overflows and the
     remaining digits are resolved over the whole row);
-  * lengths not a multiple of 4 (scalar loads), rows that fit in shared
-    memory and rows that do not (re-read from L2), a ragged last warp slice;
-  * k = 1, k = N - 1 and k >= N.
+  * lengths not a multiple of 4 (scalar loads), short and long rows, a
+    ragged last warp slice;
+  * k = 1, k = N - 1 and k >= N;
+  * many rows at once, repeatedly, whose candidates all need the second and
+    third digits (a clear of one digit's histogram racing the next digit's
+    counts would lose counts in some row, some time).
 """
 import numpy as np
 import pytest
@@ -38,11 +41,11 @@ def _rows(kind, rows, N, rng):
 
 
 CASES = [
-    ("lognormal", 6, 32760, 1638),      # the long-video row length, cached in shared memory
+    ("lognormal", 6, 32760, 1638),      # the long-video row length
     ("lognormal", 3, 65536, 1966),      # too long to cache
     ("lognormal", 4, 4099, 123),        # N % 4 != 0: scalar loads, ragged slices
-    ("lognormal", 4, 40960, 2048),      # the longest cached row
-    ("lognormal", 2, 40964, 2048),      # one vector past it
+    ("lognormal", 4, 40960, 2048),
+    ("lognormal", 2, 40964, 2048),
     ("few_values", 5, 15600, 1560),
     ("few_values", 3, 4097, 1000),
     ("constant", 3, 32760, 1638),
@@ -67,6 +70,18 @@ def test_select_topk_matches_oracle(kind, rows, N, k):
         assert np.array_equal(got[r], ref), f"{kind} row {r}: {np.sum(got[r] != ref)} indices differ"
 
 
+def test_select_topk_many_rows_repeatably():
+    rng = np.random.default_rng(77)
+    rows, N, k = 2000, 6000, 3000
+    s = _rows("near_constant", rows, N, rng)         # every key a candidate; passes 3 and 4 decide
+    ref = np.stack([orc.select_kv(s[r].astype(np.float64), k) for r in range(rows)])
+    dev = torch.from_numpy(s).cuda()
+    for rep in range(5):
+        got = mcs.select_topk(dev, k).cpu().numpy()
+        bad = np.nonzero((got != ref).any(axis=1))[0]
+        assert len(bad) == 0, f"repetition {rep}: {len(bad)} rows differ, first {bad[:5]}"
+
+
 def test_select_topk_batched_shape_and_empty():
     s = torch.rand(2, 3, 5, 777, device="cuda")
     out = mcs.select_topk(s, 50)
@@ -77,3 +92,47 @@ def test_select_topk_batched_shape_and_empty():
         assert np.array_equal(o[r], orc.select_kv(host[r].astype(np.float64), 50))
     empty = mcs.select_topk(torch.empty(0, 100, device="cuda"), 10)
     assert empty.shape == (0, 10)
+
+
+# ---------------------------------------------------------------------------
+# The plan's selection on the group scores it has just made: exactly what the
+# selection gives when called on those scores, including rows whose ties
+# overflow the candidate list.
+
+import synth  # noqa: E402
+from tests.gpu_util import dev_bf16  # noqa: E402
+
+
+def _plan_and_scores(Q, K, V, G, k):
+    B, H, N, d = Q.shape
+    q, kd, v = dev_bf16(Q), dev_bf16(K), dev_bf16(V)
+    ws = mcs.alloc_workspace(B, H, N, d, G, k, q.device)
+    meta = mcs.plan(q, kd, v, G, k, workspace=ws)
+    colsum = mcs.workspace_views(ws, B, H, N, d, G, k)["colsum"]
+    ref = mcs.select_topk(colsum, min(k, N))
+    torch.cuda.synchronize()
+    assert mcs.last_device_status() == 0
+    return meta.kv_idx.cpu().numpy(), ref.cpu().numpy(), colsum.cpu().numpy()
+
+
+@pytest.mark.parametrize("N,d,G,k", [(999, 64, 64, 100), (1024, 128, 128, 300), (2500, 128, 64, 1),
+                                     (777, 64, 128, 777), (1300, 128, 128, 5000)])
+def test_plan_selection_equals_select_topk_on_its_scores(N, d, G, k):
+    Q, K, V = synth.random_qkv(1, 2, N, d, seed=21, q_std=2.0)
+    got, ref, _ = _plan_and_scores(Q, K, V, G, k)
+    assert np.array_equal(got, ref)
+
+
+@pytest.mark.parametrize("N,d", [(1000, 128), (16384, 128), (13000, 64)])
+def test_plan_selection_on_constant_rows(N, d):
+    """K = 0 makes every score 0 and every group's probabilities uniform, so
+    each group-score row is constant: the selection is keys 0 .. k-1 (ties to
+    the lower index).  At N = 16384 and 13000 the whole row overflows the
+    candidate list and the remaining digits are resolved over the row."""
+    Q, _, V = synth.random_qkv(1, 1, N, d, seed=22)
+    K = np.zeros_like(Q)
+    k = 700
+    got, ref, cs = _plan_and_scores(Q, K, V, 128, k)
+    assert np.all(cs[0, 0] == cs[0, 0, :, :1])          # each group's row is constant
+    assert np.array_equal(got, ref)
+    assert np.array_equal(got[0, 0], np.broadcast_to(np.arange(k, dtype=np.int32), got[0, 0].shape))
