@@ -66,7 +66,7 @@ def parse_args():
     ap.add_argument("--ablate-rows", type=int, default=64, help="sampled queries per head for the ungrouped oracle")
     ap.add_argument("--blocks", action="store_true",
                     help="block-granular vs token selection: reused-step time and fidelity (not the contract line)")
-    ap.add_argument("--micro", choices=["gather"], default=None,
+    ap.add_argument("--micro", choices=["gather", "ex2", "mma", "all"], default=None,
                     help="run the gather microbenchmark alone: one JSON line per (mode, warps)")
     ap.add_argument("--sweep", action="store_true",
                     help="sparsity sweep on the 131K-token layer: one JSON line per (G, k) point "
@@ -540,20 +540,33 @@ def run_blocks(args):
 
 def run_micro(args):
     """--micro gather: the rate at which one CTA per SM brings index-listed
-    256-byte rows (bf16, d = 128) into shared memory, by TMA tile::gather4
-    from 1-8 warps and by cp.async from 1-8 warps, against TMA tile loads of
-    contiguous rows; one JSON line per point.  The source is 16.8 MB (one
-    head's K and V at d = 128), so it is L2-resident, as in the reused step."""
+    256-byte rows into shared memory, by TMA tile::gather4 from 1-8 warps and
+    by cp.async from 1-8 warps, against TMA tile loads of contiguous rows.
+    The source is 16.8 MB (one head's K and V at d = 128), so it is
+    L2-resident, as in the reused step.
+    --micro ex2: MUFU exponentials per SM cycle (8-32 warps per SM).
+    --micro mma: cycles per tcgen05 MMA for the reused step's two shapes (and
+    128x128 SS), issued back to back by one warp per SM, alone and while
+    eight other warps keep the MUFU or the FMA pipe busy.
+    One JSON line per point; not the contract line."""
     import torch
     from sparse_attention_diffusion_mcs_b200 import micro
     dev = torch.device("cuda", 0)
-    for mode, warps in (("gather4", (1, 2, 4, 7, 8)), ("cp.async", (1, 2, 4, 8)), ("tile", (1,))):
-        for nw in warps:
-            r = micro.gather_rate(mode, nw, device=dev)
-            r["micro"] = "index-listed 256-byte rows into shared memory, one CTA per SM"
-            print(json.dumps(r), flush=True)
+    if args.micro in ("gather", "all"):
+        for mode, warps in (("gather4", (1, 2, 4, 7, 8)), ("cp.async", (1, 2, 4, 8)), ("tile", (1,))):
+            for nw in warps:
+                r = micro.gather_rate(mode, nw, device=dev)
+                r["micro"] = "index-listed 256-byte rows into shared memory, one CTA per SM"
+                print(json.dumps(r), flush=True)
+    if args.micro in ("ex2", "all"):
+        for nw in (8, 16, 32):
+            print(json.dumps(micro.ex2_rate(nw, device=dev)), flush=True)
+    if args.micro in ("mma", "all"):
+        for shape in micro.MMA_SHAPES:
+            for chains in ((1, 2, 4) if shape.startswith("qk") else (1, 2)):
+                for load in micro.MMA_LOADS:
+                    print(json.dumps(micro.mma_rate(shape, load, chains=chains, device=dev)), flush=True)
     return 0
-
 
 def _drift_step_head(args):
     cfg, k, G, bh, seed_shift, step, q, kk, v = args

@@ -11,7 +11,7 @@ CSRC = os.path.join(PKG_DIR, "csrc")
 LIB_PATH = os.path.join(PKG_DIR, "libmcs.so")
 MICRO_LIB_PATH = os.path.join(PKG_DIR, "libmcs_micro.so")
 SOURCES = ["mcs_api.cu"]
-MICRO_SOURCES = ["micro_gather.cu"]
+MICRO_SOURCES = ["micro_gather.cu", "micro_pipes.cu"]
 HEADERS = ["mcs_common.cuh", "ablation_kernels.cuh", "attn_kernel.cuh", "attn_dual_kernel.cuh", "pair_kernel.cuh", "colsum_kernel.cuh", "topk_kernel.cuh",
            "group_kernels.cuh", "validate_kernels.cuh", "residual_compact.cuh"]
 NVCC_FLAGS = [
@@ -59,8 +59,9 @@ def _compile(lib, sources, verbose):
 
 
 def build(force: bool = False, verbose: bool = False) -> str:
-    """Compile libmcs.so (the hot path) and libmcs_micro.so (the gather
-    microbenchmark) in-tree for sm_100a; returns libmcs.so's path."""
+    """Compile libmcs.so (the hot path) and libmcs_micro.so (the gather, MMA
+    and exponential microbenchmarks) in-tree for sm_100a; returns libmcs.so's
+    path."""
     if force or not _up_to_date(LIB_PATH, SOURCES, "mcs.h"):
         _compile(LIB_PATH, SOURCES, verbose)
     if force or not _up_to_date(MICRO_LIB_PATH, MICRO_SOURCES, "mcs_micro.h"):

@@ -54,6 +54,13 @@ def test_micro_library_exports_its_header():
     assert M.mcs_micro_gather(FAKE, 1024, FAKE, 1, 1, 0, 9, None) == INVALID      # more than 8 warps
     assert M.mcs_micro_gather(FAKE, 1024, FAKE, 1, 1, 3, 1, None) == INVALID      # no such mode
     assert M.mcs_micro_gather(FAKE + 8, 1024, FAKE, 1, 1, 0, 1, None) == INVALID  # misaligned source
+    assert M.mcs_micro_ex2(1, 8, 16, None, None) == INVALID
+    assert M.mcs_micro_ex2(1, 33, 16, FAKE, None) == INVALID                      # more than 32 warps
+    assert M.mcs_micro_mma(1, 3, 16, 0, 1, FAKE, None) == INVALID                  # no such shape
+    assert M.mcs_micro_mma(1, 0, 16, 3, 1, FAKE, None) == INVALID                  # no such load
+    assert M.mcs_micro_mma(1, 0, 0, 0, 1, FAKE, None) == INVALID
+    assert M.mcs_micro_mma(1, 1, 16, 0, 3, FAKE, None) == INVALID                  # N = 128: two accumulators at most
+    assert M.mcs_micro_mma(1, 0, 16, 0, 5, FAKE, None) == INVALID
 
 
 def test_version_and_status_strings(L):
