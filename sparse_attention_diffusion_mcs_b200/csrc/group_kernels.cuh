@@ -60,12 +60,14 @@ __global__ void mean_finalize_kernel(const double *__restrict__ part, int N, int
 
 // ---------------------------------------------------------------- covariance
 // 256 threads as a 16 x 16 grid; thread (ti, tj) accumulates C[ti + 16a][tj + 16b]
-// for a, b < R = D/16 in fp64 registers (columns interleaved so the shared
-// memory reads of one warp hit distinct banks).  Rows are centred and staged
-// through a double-buffered shared tile, the next tile's 16-byte loads in
-// flight while the current one is consumed.  The mirror entry C[j][i] is the
-// same sequence of fma(x_i, x_j, .) in the same row order, so the partial
-// matrices are exactly symmetric.
+// in fp64 registers (columns interleaved so the shared memory reads of one
+// warp hit distinct banks) for the block pairs a <= b < R = D/16 only, and
+// writes each a < b entry twice, at (i, j) and at its mirror (j, i): the
+// mirror would be the same sequence of fma(x_i, x_j, .) in the same row order
+// (the product commutes), so the partial matrices are exactly symmetric and
+// the lower block triangle (R(R-1)/2 of the R^2 block pairs) is not computed.
+// Rows are centred and staged through a double-buffered shared tile, the next
+// tile's 16-byte loads in flight while the current one is consumed.
 template <int D>
 __global__ void __launch_bounds__(256) cov_kernel(const bf16 *__restrict__ Q, const double *__restrict__ mean,
                                                   int N, int n_chunks, double *__restrict__ part) {
@@ -98,11 +100,11 @@ __global__ void __launch_bounds__(256) cov_kernel(const bf16 *__restrict__ Q, co
     for (int e = 0; e < 8; ++e)
       xs[buf][srow][scol + e] = live ? static_cast<double>(__bfloat162float(h[e])) - mus[e] : 0.0;
   };
-  double acc[R][R];
+  double acc[R][R];   // only a <= b is used
 #pragma unroll
   for (int a = 0; a < R; ++a)
 #pragma unroll
-    for (int b = 0; b < R; ++b) acc[a][b] = 0.0;
+    for (int b = a; b < R; ++b) acc[a][b] = 0.0;
   int buf = 0;
   stage(0, r0, fetch(r0));
   __syncthreads();
@@ -120,7 +122,7 @@ __global__ void __launch_bounds__(256) cov_kernel(const bf16 *__restrict__ Q, co
 #pragma unroll
       for (int a = 0; a < R; ++a)
 #pragma unroll
-        for (int b = 0; b < R; ++b) acc[a][b] = fma(xi[a], xj[b], acc[a][b]);
+        for (int b = a; b < R; ++b) acc[a][b] = fma(xi[a], xj[b], acc[a][b]);
     }
     if (more) stage(buf ^ 1, rb + ROWS, nxt);
     __syncthreads();
@@ -130,7 +132,10 @@ __global__ void __launch_bounds__(256) cov_kernel(const bf16 *__restrict__ Q, co
 #pragma unroll
   for (int a = 0; a < R; ++a)
 #pragma unroll
-    for (int b = 0; b < R; ++b) out[(ti + 16 * a) * D + tj + 16 * b] = acc[a][b];
+    for (int b = a; b < R; ++b) {
+      out[(ti + 16 * a) * D + tj + 16 * b] = acc[a][b];
+      if (b > a) out[(tj + 16 * b) * D + ti + 16 * a] = acc[a][b];
+    }
 }
 
 // C = (sum of the chunk partials, in chunk order) / N; one thread per entry.
@@ -153,7 +158,8 @@ __global__ void __launch_bounds__(256) cov_reduce_kernel(const double *__restric
 // and then with C itself (copied into the same shared buffer) give v.
 // M stays exactly symmetric (T[i][j] and T[j][i] are the same fma sequence),
 // so T = M.M is formed as sum_t M[t][i] M[t][j]: both operands are read from
-// row t, and thread (ti, tj) keeps its R x R block of T in registers.
+// row t, and thread (ti, tj) keeps its blocks a <= b of T in registers and
+// writes each a < b entry also at its mirror (as the covariance does).
 template <int D>
 __global__ void __launch_bounds__(256) eig_kernel(const double *__restrict__ cov, double *__restrict__ vdir,
                                                   float *__restrict__ lambda) {
@@ -187,11 +193,11 @@ __global__ void __launch_bounds__(256) eig_kernel(const double *__restrict__ cov
   for (int e = tid; e < D * D; e += 256) M[e] = Cm[e] / tr;
   __syncthreads();
   for (int sq = 0; sq < 10; ++sq) {        // M <- M^2 / trace(M^2)  ->  C^(2^10), normalised
-    double acc[R][R];
+    double acc[R][R];   // only a <= b is used
 #pragma unroll
     for (int a = 0; a < R; ++a)
 #pragma unroll
-      for (int b = 0; b < R; ++b) acc[a][b] = 0.0;
+      for (int b = a; b < R; ++b) acc[a][b] = 0.0;
 #pragma unroll 2
     for (int t = 0; t < D; ++t) {
       double xi[R], xj[R];
@@ -203,7 +209,7 @@ __global__ void __launch_bounds__(256) eig_kernel(const double *__restrict__ cov
 #pragma unroll
       for (int a = 0; a < R; ++a)
 #pragma unroll
-        for (int b = 0; b < R; ++b) acc[a][b] = fma(xi[a], xj[b], acc[a][b]);
+        for (int b = a; b < R; ++b) acc[a][b] = fma(xi[a], xj[b], acc[a][b]);
     }
     double dsum = 0.0;
     if (ti == tj)
@@ -213,7 +219,11 @@ __global__ void __launch_bounds__(256) eig_kernel(const double *__restrict__ cov
 #pragma unroll
     for (int a = 0; a < R; ++a)
 #pragma unroll
-      for (int b = 0; b < R; ++b) M[(ti + 16 * a) * D + tj + 16 * b] = acc[a][b] / t2;
+      for (int b = a; b < R; ++b) {
+        const double x = acc[a][b] / t2;
+        M[(ti + 16 * a) * D + tj + 16 * b] = x;
+        if (b > a) M[(tj + 16 * b) * D + ti + 16 * a] = x;
+      }
     __syncthreads();
   }
   // start from the column of M with the largest diagonal entry
