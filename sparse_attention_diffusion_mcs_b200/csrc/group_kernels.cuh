@@ -15,7 +15,9 @@
 //                     squaring + power iteration, sign fixed so the
 //                     largest-magnitude component is positive
 //   project_kernel    p_n = (q_n - mu) . v  -> order-preserving uint64 key
-//   sort_kernel       per head: stable LSD radix sort of (key, n) -> perm
+//   sort_hist_kernel, sort_scatter_kernel
+//                     per head, over several CTAs: stable LSD radix sort of
+//                     (key, n) -> perm
 #pragma once
 
 #include "mcs_common.cuh"
@@ -314,92 +316,126 @@ __global__ void __launch_bounds__(256) project_kernel(const bf16 *__restrict__ Q
 }
 
 // ---------------------------------------------------------------- stable LSD radix sort
-// One CTA per head, 8 passes of 8 bits over 64-bit keys.  Each pass:
-// histogram, exclusive scan, then a scatter over tiles of 1024 keys in index
-// order, ranking equal digits by (warp, lane) so the pass is stable.
-__global__ void __launch_bounds__(kSortThreads) sort_kernel(unsigned long long *keys_a, int32_t *vals_a,
-                                                            unsigned long long *keys_b, int32_t *vals_b,
-                                                            int N, int32_t *__restrict__ perm) {
+// 8 passes of 8 bits over 64-bit keys.  A head's array is cut into `parts`
+// contiguous chunks of whole 1024-key tiles, one CTA each, so a head's sort
+// runs on several SMs.  Per pass, sort_hist_kernel counts each chunk's digits
+// and sort_scatter_kernel places each chunk's keys from base[digit] = (the
+// head's keys of smaller digits) + (keys of this digit in earlier chunks),
+// scattering its tiles in index order and ranking equal digits inside a tile
+// by (warp, lane): stable, exactly the order one CTA per head would give.
+__global__ void __launch_bounds__(kSortThreads) sort_hist_kernel(const unsigned long long *__restrict__ keys, int N,
+                                                                 int chunk, int shift, unsigned *__restrict__ ghist) {
   __shared__ unsigned bins[256];
+  const int part = blockIdx.x, bh = blockIdx.y, parts = gridDim.x;
+  for (int i = threadIdx.x; i < 256; i += kSortThreads) bins[i] = 0;
+  __syncthreads();
+  const unsigned long long *k = keys + static_cast<size_t>(bh) * N;
+  const int j0 = part * chunk, j1 = min(N, j0 + chunk);
+  for (int j = j0 + static_cast<int>(threadIdx.x); j < j1; j += kSortThreads)
+    atomicAdd(&bins[static_cast<unsigned>(k[j] >> shift) & 255u], 1u);
+  __syncthreads();
+  for (int i = threadIdx.x; i < 256; i += kSortThreads) ghist[(static_cast<size_t>(bh) * parts + part) * 256 + i] = bins[i];
+}
+
+// vout_head: the pass's value output for this head (the next pass's input, or
+// the final perm row)
+__global__ void __launch_bounds__(kSortThreads) sort_scatter_kernel(const unsigned long long *__restrict__ kin,
+                                                                    const int32_t *__restrict__ vin,
+                                                                    unsigned long long *__restrict__ kout,
+                                                                    int32_t *__restrict__ vout, int N, int chunk,
+                                                                    int shift, const unsigned *__restrict__ ghist) {
   __shared__ unsigned base[256];
   __shared__ unsigned tile_tot[256];
   __shared__ unsigned short wcnt[32][256];   // per-warp digit counts, then exclusive prefixes
-  const int bh = blockIdx.x;
+  const int part = blockIdx.x, bh = blockIdx.y, parts = gridDim.x;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const unsigned lt_mask = (1u << lane) - 1u;
-  unsigned long long *kin = keys_a + static_cast<size_t>(bh) * N;
-  int32_t *vin = vals_a + static_cast<size_t>(bh) * N;
-  unsigned long long *kout = keys_b + static_cast<size_t>(bh) * N;
-  int32_t *vout = vals_b + static_cast<size_t>(bh) * N;
-
-  for (int pass = 0; pass < 8; ++pass) {
-    const int shift = pass * 8;
-    for (int i = tid; i < 256; i += kSortThreads) bins[i] = 0;
+  if (warp == 0) {   // lane l owns digits 8l .. 8l+7
+    unsigned tot[8], before[8], sum = 0;
+#pragma unroll
+    for (int b = 0; b < 8; ++b) {
+      const int d = lane * 8 + b;
+      unsigned t = 0, e = 0;
+      for (int pp = 0; pp < parts; ++pp) {
+        const unsigned x = ghist[(static_cast<size_t>(bh) * parts + pp) * 256 + d];
+        t += x;
+        e += pp < part ? x : 0u;
+      }
+      tot[b] = t;
+      before[b] = e;
+      sum += t;
+    }
+    unsigned inc = sum;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const unsigned y = __shfl_up_sync(0xffffffffu, inc, o);
+      if (lane >= o) inc += y;
+    }
+    unsigned run = inc - sum;
+#pragma unroll
+    for (int b = 0; b < 8; ++b) {
+      base[lane * 8 + b] = run + before[b];
+      run += tot[b];
+    }
+  }
+  __syncthreads();
+  const unsigned long long *ki = kin + static_cast<size_t>(bh) * N;
+  const int32_t *vi = vin + static_cast<size_t>(bh) * N;
+  unsigned long long *ko = kout + static_cast<size_t>(bh) * N;
+  int32_t *vo = vout + static_cast<size_t>(bh) * N;
+  const int j0 = part * chunk, j1 = min(N, j0 + chunk);
+  for (int t0 = j0; t0 < j1; t0 += kSortThreads) {
+    const int j = t0 + tid;
+    const bool valid = j < j1;
+    unsigned long long key = 0;
+    int32_t val = 0;
+    if (valid) {
+      key = ki[j];
+      val = vi[j];
+    }
+    const unsigned digit = valid ? (static_cast<unsigned>(key >> shift) & 255u) : 256u;
+    for (int b = lane; b < 256; b += 32) wcnt[warp][b] = 0;
+    __syncwarp();
+    const unsigned peers = __match_any_sync(0xffffffffu, digit);
+    const unsigned rank_in_warp = __popc(peers & lt_mask);
+    if (valid && rank_in_warp == 0) wcnt[warp][digit] = static_cast<unsigned short>(__popc(peers));
     __syncthreads();
-    for (int j = tid; j < N; j += kSortThreads) atomicAdd(&bins[static_cast<unsigned>(kin[j] >> shift) & 255u], 1u);
-    __syncthreads();
-    if (warp == 0) {
-      unsigned c[8], sum = 0;
-#pragma unroll
-      for (int b = 0; b < 8; ++b) {
-        c[b] = bins[lane * 8 + b];
-        sum += c[b];
+    if (tid < 256) {
+      unsigned run = 0;
+      for (int w = 0; w < 32; ++w) {
+        const unsigned cnt = wcnt[w][tid];
+        wcnt[w][tid] = static_cast<unsigned short>(run);
+        run += cnt;
       }
-      unsigned inc = sum;
-#pragma unroll
-      for (int o = 1; o < 32; o <<= 1) {
-        const unsigned y = __shfl_up_sync(0xffffffffu, inc, o);
-        if (lane >= o) inc += y;
-      }
-      unsigned run = inc - sum;
-#pragma unroll
-      for (int b = 0; b < 8; ++b) {
-        base[lane * 8 + b] = run;
-        run += c[b];
-      }
+      tile_tot[tid] = run;
     }
     __syncthreads();
-    for (int t0 = 0; t0 < N; t0 += kSortThreads) {
-      const int j = t0 + tid;
-      const bool valid = j < N;
-      unsigned long long key = 0;
-      int32_t val = 0;
-      if (valid) {
-        key = kin[j];
-        val = vin[j];
-      }
-      const unsigned digit = valid ? (static_cast<unsigned>(key >> shift) & 255u) : 256u;
-      for (int b = lane; b < 256; b += 32) wcnt[warp][b] = 0;
-      __syncwarp();
-      const unsigned peers = __match_any_sync(0xffffffffu, digit);
-      const unsigned rank_in_warp = __popc(peers & lt_mask);
-      if (valid && rank_in_warp == 0) wcnt[warp][digit] = static_cast<unsigned short>(__popc(peers));
-      __syncthreads();
-      if (tid < 256) {
-        unsigned run = 0;
-        for (int w = 0; w < 32; ++w) {
-          const unsigned cnt = wcnt[w][tid];
-          wcnt[w][tid] = static_cast<unsigned short>(run);
-          run += cnt;
-        }
-        tile_tot[tid] = run;
-      }
-      __syncthreads();
-      if (valid) {
-        const unsigned pos = base[digit] + wcnt[warp][digit] + rank_in_warp;
-        kout[pos] = key;
-        vout[pos] = val;
-      }
-      __syncthreads();
-      if (tid < 256) base[tid] += tile_tot[tid];
-      __syncthreads();
+    if (valid) {
+      const unsigned pos = base[digit] + wcnt[warp][digit] + rank_in_warp;
+      ko[pos] = key;
+      vo[pos] = val;
     }
-    unsigned long long *kt = kin; kin = kout; kout = kt;
-    int32_t *vt = vin; vin = vout; vout = vt;
+    __syncthreads();
+    if (tid < 256) base[tid] += tile_tot[tid];
     __syncthreads();
   }
-  // after an even number of passes the sorted data is back in keys_a / vals_a
-  for (int j = tid; j < N; j += kSortThreads) perm[static_cast<size_t>(bh) * N + j] = vin[j];
+}
+
+// chunks per head: about two CTAs per SM of a 148-SM B200 in all (a fixed
+// figure, so the workspace size does not depend on the device), whole tiles,
+// at most 64
+constexpr int kSortSms = 148;
+inline int sort_parts(int BH, int N, int sms = kSortSms) {
+  const int tiles = (N + kSortThreads - 1) / kSortThreads;
+  int parts = BH > 0 ? (2 * sms) / BH : 1;
+  parts = parts < 1 ? 1 : (parts > 64 ? 64 : parts);
+  if (parts > tiles) parts = tiles > 0 ? tiles : 1;
+  const int chunk = ((tiles + parts - 1) / parts) * kSortThreads;
+  return N > 0 ? (N + chunk - 1) / chunk : 1;
+}
+inline int sort_chunk(int N, int parts) {
+  const int tiles = (N + kSortThreads - 1) / kSortThreads;
+  return ((tiles + parts - 1) / parts) * kSortThreads;
 }
 
 }  // namespace mcs

@@ -6,6 +6,7 @@
 #include <cstdint>
 #include <cstring>
 #include <mutex>
+#include <utility>
 
 #include "../../include/mcs.h"
 #include "ablation_kernels.cuh"
@@ -209,7 +210,7 @@ AttnArgs base_args(int N, float scale) {
 
 // ---------------------------------------------------------------- plan workspace
 struct PlanWs {
-  size_t mean_part, mean, cov_part, cov64, vdir, lambda, keys0, vals0, keys1, vals1;
+  size_t mean_part, mean, cov_part, cov64, vdir, lambda, keys0, vals0, keys1, vals1, ghist;
   size_t row_m, row_l, O32, colsum, pair_idx, pair_len, total;
 };
 
@@ -234,6 +235,7 @@ PlanWs plan_ws(int B, int H, int N, int d, int G, int k) {
   w.vals0 = take(BH * N * 4);
   w.keys1 = take(BH * N * 8);
   w.vals1 = take(BH * N * 4);
+  w.ghist = take(BH * static_cast<size_t>(sort_parts(static_cast<int>(BH), N)) * 256 * 4);
   w.row_m = take(BH * N * 4);
   w.row_l = take(BH * N * 4);
   w.O32 = take(BH * N * static_cast<size_t>(d) * 4);
@@ -271,9 +273,20 @@ cudaError_t run_group(const void *Q, int BH, int N, int32_t *perm, void *ws, con
   project_kernel<D><<<dim3((N + 7) / 8, BH), 256, 0, s>>>(q, at<double>(ws, w.mean), at<double>(ws, w.vdir), N,
                                                            at<unsigned long long>(ws, w.keys0),
                                                            at<int32_t>(ws, w.vals0));
-  sort_kernel<<<BH, kSortThreads, 0, s>>>(at<unsigned long long>(ws, w.keys0), at<int32_t>(ws, w.vals0),
-                                          at<unsigned long long>(ws, w.keys1), at<int32_t>(ws, w.vals1), N,
-                                          perm);
+  if ((e = cudaGetLastError()) != cudaSuccess) return e;
+  // stable LSD radix sort of (key, token) over several CTAs per head; the last
+  // pass writes its tokens straight into perm
+  const int parts = sort_parts(BH, N), chunk = sort_chunk(N, parts);
+  unsigned *gh = at<unsigned>(ws, w.ghist);
+  unsigned long long *ka = at<unsigned long long>(ws, w.keys0), *kb = at<unsigned long long>(ws, w.keys1);
+  int32_t *va = at<int32_t>(ws, w.vals0), *vb = at<int32_t>(ws, w.vals1);
+  const dim3 grid(parts, BH);
+  for (int pass = 0; pass < 8; ++pass) {
+    sort_hist_kernel<<<grid, kSortThreads, 0, s>>>(ka, N, chunk, 8 * pass, gh);
+    sort_scatter_kernel<<<grid, kSortThreads, 0, s>>>(ka, va, kb, pass == 7 ? perm : vb, N, chunk, 8 * pass, gh);
+    std::swap(ka, kb);
+    std::swap(va, vb);
+  }
   return cudaGetLastError();
 }
 
