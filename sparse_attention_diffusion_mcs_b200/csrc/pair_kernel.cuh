@@ -21,9 +21,7 @@
 //  kModeStep      O_i = softmax over the group's kept keys of (scale Q_i.K_j)
 //                 applied to V, plus the cached residual R_i; bf16 out
 //                 (aiqbench.com abstract: groups, KV indices and residuals
-//                 "reused across subsequent denoising steps").  The residual
-//                 is read as fp32, or from its bf16 copy (residual16), or
-//                 not at all (the block-sparse comparison may run without one).
+//                 "reused across subsequent denoising steps").
 //  kModePlanResid R_i = O_dense_i - O_sparse_i with O_dense from the plan's
 //                 statistics pass ("residuals between dense and sparse
 //                 attention outputs").
