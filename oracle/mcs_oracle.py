@@ -125,8 +125,11 @@ def principal_direction(Q):
 
 
 def projections(Q, mu, v) -> np.ndarray:
-    """p_n = (Q_n - mu) . v"""
-    return (_as_f64(Q) - mu) @ v
+    """p_n = (Q_n - mu) . v, each row's dot product summed on its own, so that
+    equal query rows get equal projections and the stable sort keeps them in
+    token order (a matrix-vector product may round equal rows differently,
+    depending on where they fall in its row blocks and threads)."""
+    return ((_as_f64(Q) - mu) * v).sum(axis=1)
 
 
 def group_queries(Q) -> np.ndarray:

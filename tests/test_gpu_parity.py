@@ -152,6 +152,24 @@ def test_plan_group_matches_oracle_order(cfg_or_shape):
             assert np.array_equal(perm[b, h], ref), f"b{b} h{h}: {np.sum(perm[b, h] != ref)} positions differ"
 
 
+@pytest.mark.parametrize("N,d,BH", [(5000, 64, 1), (9000, 128, 2), (3100, 64, 3)])
+def test_plan_group_stable_on_ties_across_sort_chunks(N, d, BH):
+    """Runs of identical query rows give identical projections, so their
+    order is decided by the sort's stability alone (ascending token index).
+    At these sizes a head's sort is split over several CTAs (chunks of 1024
+    keys, the last one ragged), so equal keys meet across chunk borders."""
+    rng = np.random.default_rng(N + d)
+    Q, _, _ = synth.random_qkv(1, BH, N, d, seed=9)
+    for h in range(BH):
+        src = rng.integers(0, N, size=N // 3)          # a third of the rows copy another row
+        dst = rng.integers(0, N, size=N // 3)
+        Q[0, h, dst] = Q[0, h, src]
+    perm = mcs.plan_group(dev_bf16(Q)).cpu().numpy()
+    for h in range(BH):
+        ref = orc.group_queries(Q[0, h])
+        assert np.array_equal(perm[0, h], ref), f"h{h}: {np.sum(perm[0, h] != ref)} positions differ"
+
+
 # ----------------------------------------------------------------------------- selection (a2-a4)
 
 @pytest.mark.parametrize("cfg,G,k", [(1, 64, 128), (1, 128, 300), (1, 64, 1), (1, 128, 1024)])

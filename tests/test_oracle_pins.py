@@ -121,6 +121,29 @@ def test_group_queries_ties_keep_index_order():
     assert list(perm) == [0, 3, 6, 1, 4, 7, 2, 5, 8]
 
 
+@pytest.mark.parametrize("N,d", [(9000, 128), (5000, 64)])
+def test_group_queries_equal_rows_keep_index_order_at_size(N, d):
+    """Equal query rows have equal projections, so the stable sort keeps each
+    set of equal rows in token order, wherever the rows lie in the array (a
+    blocked or threaded matrix-vector product can round equal rows apart)."""
+    rng = np.random.default_rng(N + d)
+    Q = rng.standard_normal((N, d))
+    src = rng.integers(0, N, size=N // 3)
+    dst = rng.integers(0, N, size=N // 3)
+    Q[dst] = Q[src]
+    perm = orc.group_queries(Q)
+    where = np.empty(N, np.int64)
+    where[perm] = np.arange(N)
+    _, inv = np.unique(Q, axis=0, return_inverse=True)
+    inv = inv.ravel()
+    order = np.lexsort((np.arange(N), inv))           # tokens by set, ascending inside each set
+    same_set = inv[order][1:] == inv[order][:-1]
+    assert same_set.sum() > N // 5                    # many sets of equal rows
+    a, b = order[:-1][same_set], order[1:][same_set]
+    assert np.all(where[a] < where[b])                # lower token first ...
+    assert np.all(where[b] - where[a] == 1)           # ... and adjacent: nothing sorts between equal rows
+
+
 def test_groups_partition_with_partial_tail():
     perm = np.arange(10)[::-1]
     groups = [orc.group_rows(perm, 4, g) for g in range(3)]
