@@ -330,22 +330,26 @@ cudaError_t run_scores(const void *Q, const void *K, const int32_t *perm, int BH
   return cudaGetLastError();
 }
 
-// top-k of `rows` rows of N scores each, k <= N
-cudaError_t launch_topk(const float *scores, int rows, int N, int k, int32_t *kv_idx, cudaStream_t s) {
-  if (rows == 0) return cudaSuccess;
-  const bool cache = static_cast<size_t>(N) * 4 <= static_cast<size_t>(kTopkRowCacheBytes);
-  const int smem = kTopkFixedSmem + (cache ? N * 4 : 0);
-  cudaError_t e;
-  if (N % 4 == 0 && aligned16(scores)) {
-    e = set_smem(topk_kernel<4>, smem);
-    if (e != cudaSuccess) return e;
-    topk_kernel<4><<<rows, kTopkThreads, smem, s>>>(scores, N, k, cache ? 1 : 0, kv_idx);
-  } else {
-    e = set_smem(topk_kernel<1>, smem);
-    if (e != cudaSuccess) return e;
-    topk_kernel<1><<<rows, kTopkThreads, smem, s>>>(scores, N, k, cache ? 1 : 0, kv_idx);
-  }
+// top-k of `rows` rows of N scores each: as many CTAs as fit on the device at
+// once (or one per row), each over a contiguous run of rows
+template <int VEC>
+cudaError_t launch_topk_vec(const float *scores, long long rows, int N, int k, int32_t *kv_idx, cudaStream_t s) {
+  cudaError_t e = set_smem(topk_kernel<VEC>, kTopkSmem);
+  if (e != cudaSuccess) return e;
+  int sms = 0, per_sm = 0;
+  if ((e = sm_count(&sms)) != cudaSuccess) return e;
+  e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, topk_kernel<VEC>, kTopkThreads, kTopkSmem);
+  if (e != cudaSuccess) return e;
+  const long long fit = static_cast<long long>(sms) * (per_sm > 0 ? per_sm : 1);
+  const int grid = static_cast<int>(rows < fit ? rows : fit);
+  topk_kernel<VEC><<<grid, kTopkThreads, kTopkSmem, s>>>(scores, rows, N, k, kv_idx);
   return cudaGetLastError();
+}
+
+cudaError_t launch_topk(const float *scores, long long rows, int N, int k, int32_t *kv_idx, cudaStream_t s) {
+  if (rows == 0) return cudaSuccess;
+  if (N % 4 == 0 && aligned16(scores)) return launch_topk_vec<4>(scores, rows, N, k, kv_idx, s);
+  return launch_topk_vec<1>(scores, rows, N, k, kv_idx, s);
 }
 
 cudaError_t run_topk(int BH, int N, int G, int k, int32_t *kv_idx, void *ws, const PlanWs &w,

@@ -8,23 +8,34 @@
 // Non-negative IEEE floats order like their bit patterns as uint32, so the
 // k-th largest value T is found by a most-significant-digit radix select over
 // the 31 magnitude bits in three digits (D1 bits, then the rest in two).  The
-// first digit is counted over the whole row; the keys whose first digit
-// equals the threshold's are then copied into a shared memory candidate list,
-// and the two remaining digits are resolved on that list alone.  Every key
-// with bits > T and the first (k - #greater) keys with bits == T are kept.
-// Each warp owns a contiguous slice of the row, so the per-warp counts give
-// every warp its output offset and the warps write their selections in index
-// order: the output comes out ascending without a sort.
+// first digit is counted over the whole row in one walk that reads the row
+// from HBM; the keys whose first digit is at least b1 (the threshold's) go to
+// a shared memory candidate list, and the two remaining digits are resolved
+// on that list alone.  Every key with bits > T and the first (k - #greater)
+// keys with bits == T are kept, written ascending.
+//
+// b1 is known only once the walk is over, so the walk lists the keys whose
+// first digit is at least a guess: the previous row's b1 less one bin.  A CTA
+// takes a contiguous run of rows, i.e. adjacent query groups of one head,
+// whose score rows are alike (on the 32K-token video layer b1 moves by at
+// most one of 4096 bins between adjacent groups).  After the walk the
+// histogram says exactly whether the guess held (b1 >= guess, no overflow);
+// if not, a second walk (from L2) lists the keys with first digit >= b1, and
+// if even those overflow the list (a near-constant row, a large k) the
+// remaining digits are resolved by walks over the whole row.
+//
+// Output: when no key equal to T has to be dropped, the selected keys are
+// marked in a bitmap of the row (in the histogram's memory, N <= 131072), and
+// a block scan over the bitmap's word counts gives every thread the output
+// offset of its words: ascending without a sort and without walking the row.
+// Otherwise each warp owns a contiguous slice of the row, per-warp counts
+// above and equal to T give every warp its output offset and its share of the
+// ties (the first ones in index order), and the warps walk their slices and
+// write their selections in index order.
 //
 // topk_row is that selection for one row by one CTA of NT threads;
-// topk_kernel runs it with one CTA of 512 threads per row of a score matrix:
-// pass 1 reads the row from HBM with 16-byte loads four deep per lane, and
-// the candidate and output passes read it again, from L2; with 64 KB of
-// shared memory per CTA, several rows are in flight per SM (a 1024-thread
-// CTA caching the row in 160 KB of shared memory, one per SM, took 40 % more
-// time on the 32K-token layer's 6144 rows).  If the candidate list overflows
-// (a near-constant row), the remaining digits are resolved by passes over the
-// whole row instead.
+// topk_kernel runs it with 512-thread CTAs, three per SM (64 KB of shared
+// memory each), each over a contiguous run of rows.
 #pragma once
 
 #include "mcs_common.cuh"
@@ -32,9 +43,11 @@
 namespace mcs {
 
 constexpr int kTopkThreads = 512;
+constexpr int kTopkCtasPerSm = 3;
 constexpr int kTopkCandCap = 6144;                 // candidate list entries (bits + index)
-constexpr int kTopkRowCacheBytes = 0;             // rows are not kept in shared memory (see above)
-constexpr int kTopkFixedSmem = (4096 + 2 * kTopkCandCap) * 4;   // histogram + candidate list
+constexpr int kTopkHistWords = 4096;               // first-digit histogram, later the output bitmap
+constexpr int kTopkSmem = (kTopkHistWords + 2 * kTopkCandCap) * 4;   // histogram + candidate list
+constexpr unsigned kTopkGuessMargin = 1;           // bins below the previous row's b1 listed in pass 1
 constexpr unsigned kTopkMagnitude = 0x7fffffffu;   // scores are >= 0; the sign bit is ignored
 
 // The statically sized scratch of one row selection.
@@ -42,7 +55,7 @@ struct TopkShared {
   int wsum[33];
   int gt_cnt[32], eq_cnt[32], w_take[32], w_base[32];
   unsigned s_bin;
-  int s_rank, s_ncand;
+  int s_rank, s_ncand, s_eq;
 };
 
 // exclusive scan of one int per thread over an NT-thread block; *total gets the sum
@@ -110,7 +123,7 @@ __device__ __forceinline__ unsigned topk_select_bin(const unsigned *hist, int nb
 // per step and four steps of loads in flight; f(j0, keys, valid) is called by
 // every lane of the warp for every step (it may use warp votes).
 template <int VEC, class F>
-__device__ __forceinline__ void topk_walk(const unsigned *src, bool from_smem, int lo, int hi, F &&f) {
+__device__ __forceinline__ void topk_walk(const unsigned *src, int lo, int hi, F &&f) {
   constexpr int STEP = 32 * VEC;
   const int lane = threadIdx.x & 31;
   for (int b = lo; b < hi; b += 4 * STEP) {
@@ -120,14 +133,13 @@ __device__ __forceinline__ void topk_walk(const unsigned *src, bool from_smem, i
       const int j0 = b + u * STEP + VEC * lane;
       if (j0 < hi) {
         if constexpr (VEC == 4) {
-          const uint4 *p = reinterpret_cast<const uint4 *>(src + j0);
-          const uint4 v = from_smem ? *p : __ldg(p);
+          const uint4 v = __ldg(reinterpret_cast<const uint4 *>(src + j0));
           x[u][0] = v.x;
           x[u][1] = v.y;
           x[u][2] = v.z;
           x[u][3] = v.w;
         } else {
-          x[u][0] = from_smem ? src[j0] : __ldg(src + j0);
+          x[u][0] = __ldg(src + j0);
         }
       } else {
 #pragma unroll
@@ -146,80 +158,108 @@ __device__ __forceinline__ void topk_walk(const unsigned *src, bool from_smem, i
   }
 }
 
+// Append the keys with c[e] set (key[e] at index j0 + e) to the candidate
+// list, one shared-memory atomic per warp and step; entries past cap are
+// counted but not stored.  Called by every lane of the warp.
+template <int VEC>
+__device__ __forceinline__ void topk_append(int j0, const unsigned *key, const bool *c, unsigned *cand_bits,
+                                            int *cand_idx, int cap, int *ncand) {
+  const int lane = threadIdx.x & 31;
+  const unsigned lt = (1u << lane) - 1u;
+  unsigned bal[VEC];
+  int n = 0;
+#pragma unroll
+  for (int e = 0; e < VEC; ++e) {
+    bal[e] = __ballot_sync(0xffffffffu, c[e]);
+    n += __popc(bal[e]);
+  }
+  if (n == 0) return;   // warp-uniform
+  int base = 0;
+  if (lane == 0) base = atomicAdd(ncand, n);
+  base = __shfl_sync(0xffffffffu, base, 0);
+#pragma unroll
+  for (int e = 0; e < VEC; ++e) {
+    const int pos = base + __popc(bal[e] & lt);
+    if (c[e] && pos < cap) {
+      cand_bits[pos] = key[e];
+      cand_idx[pos] = j0 + e;
+    }
+    base += __popc(bal[e]);
+  }
+}
+
 // The k largest of the row's N scores (row_g: their bit patterns), ties to the
 // lower index, written ascending to out[0, k), by the NT threads of the CTA
-// (all of them call it).  row_g is read-only for the whole kernel.  hist:
-// 2^D1 zeroed bins (D1: the first digit's width).  cand_bits / cand_idx:
-// cand_cap entries each.  row_sm: a shared copy of the row (N entries) to
-// fill in pass 1 and read later, or nullptr.  Every thread of the CTA must
-// reach this call (it synchronises the block).
+// (all of them call it; it synchronises the block).  row_g is read-only for
+// the whole kernel.  hist: kTopkHistWords zeroed words (left zeroed on
+// return).  cand_bits / cand_idx: cand_cap entries each.  guess: pass 1 lists
+// the keys whose first digit is >= guess (1 << D1 lists none).  Returns the
+// first digit of the row's threshold (the next row's guess is derived from
+// it), or 1 << D1 when every key is kept.
 template <int VEC, int NT, int D1>
-__device__ void topk_row(const unsigned *row_g, int N, int k, unsigned *hist, unsigned *cand_bits, int *cand_idx,
-                         int cand_cap, unsigned *row_sm, TopkShared &sh, int32_t *out) {
+__device__ unsigned topk_row(const unsigned *row_g, int N, int k, unsigned *hist, unsigned *cand_bits, int *cand_idx,
+                             int cand_cap, unsigned guess, TopkShared &sh, int32_t *out) {
   static_assert(NT % 32 == 0 && NT / 32 <= 32, "whole warps, at most 32");
   constexpr int NW = NT / 32;
   constexpr int D2 = (32 - D1) / 2, D3 = 31 - D1 - D2;   // the two remaining digits
   constexpr int S1 = 31 - D1;                           // shift of the first digit
   constexpr int NB1 = 1 << D1;
+  static_assert(NB1 <= kTopkHistWords && (1 << D2) <= kTopkHistWords, "digits fit the histogram");
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  const unsigned lt = (1u << lane) - 1u;
 
   if (k >= N) {
     for (int j = tid; j < N; j += NT) out[j] = j;
-    return;
+    return static_cast<unsigned>(NB1);
   }
   constexpr int STEP = 32 * VEC;
   const int span = ((N + NW - 1) / NW + STEP - 1) / STEP * STEP;
   const int lo = min(N, warp * span), hi = min(N, lo + span);
-  const bool cached = row_sm != nullptr;
-  const unsigned *src = cached ? row_sm : row_g;
 
   if (tid < 32) sh.gt_cnt[tid] = sh.eq_cnt[tid] = 0;
-  if (tid == 0) sh.s_ncand = 0;
+  if (tid == 0) {
+    sh.s_ncand = 0;
+    sh.s_eq = 0;
+  }
   __syncthreads();
 
-  // ---- pass 1 (global): cache the row, count the first digit
-  topk_walk<VEC>(row_g, false, lo, hi, [&](int j0, const unsigned *key, bool valid) {
-    if (!valid) return;
+  // ---- pass 1 (HBM): count the first digit; list the keys whose first digit is >= guess
+  topk_walk<VEC>(row_g, lo, hi, [&](int j0, const unsigned *key, bool valid) {
+    bool c[VEC];
 #pragma unroll
     for (int e = 0; e < VEC; ++e) {
-      if (cached) row_sm[j0 + e] = key[e];
-      atomicAdd(&hist[key[e] >> S1], 1u);
+      const unsigned d = key[e] >> S1;
+      if (valid) atomicAdd(&hist[d], 1u);
+      c[e] = valid && d >= guess;
     }
+    topk_append<VEC>(j0, key, c, cand_bits, cand_idx, cand_cap, &sh.s_ncand);
   });
   __syncthreads();
   int kk = k;
   const unsigned b1 = topk_select_bin<NT>(hist, NB1, kk, sh);
+  const int in_bin = static_cast<int>(hist[b1]);
+  const int n_above = k - kk;               // keys whose first digit is above b1
+  const int n_first = sh.s_ncand;
+  __syncthreads();                          // every thread has read them
   for (int i = tid; i < NB1; i += NT) hist[i] = 0;
+  bool listed = b1 >= guess && n_first <= cand_cap;
+  const bool relist = !listed && n_above + in_bin <= cand_cap;
+  if (relist && tid == 0) sh.s_ncand = 0;
+  __syncthreads();                          // histogram clear and list reset seen by all
 
-  // ---- pass 2: per-warp count above the threshold's bin; candidates into the list
-  int above = 0;
-  topk_walk<VEC>(src, cached, lo, hi, [&](int j0, const unsigned *key, bool valid) {
+  // ---- pass 2 (L2), only when the guess missed: list the keys whose first digit is >= b1
+  if (relist) {
+    topk_walk<VEC>(row_g, lo, hi, [&](int j0, const unsigned *key, bool valid) {
+      bool c[VEC];
 #pragma unroll
-    for (int e = 0; e < VEC; ++e) {
-      const unsigned d = key[e] >> S1;
-      above += (valid && d > b1) ? 1 : 0;
-      const bool c = valid && d == b1;
-      const unsigned bal = __ballot_sync(0xffffffffu, c);
-      if (bal == 0u) continue;
-      int base = 0;
-      if (lane == 0) base = atomicAdd(&sh.s_ncand, __popc(bal));
-      base = __shfl_sync(0xffffffffu, base, 0);
-      const int pos = base + __popc(bal & lt);
-      if (c && pos < cand_cap) {
-        cand_bits[pos] = key[e];
-        cand_idx[pos] = j0 + e;
-      }
-    }
-  });
-#pragma unroll
-  for (int o = 16; o > 0; o >>= 1) above += __shfl_xor_sync(0xffffffffu, above, o);
-  if (lane == 0) sh.gt_cnt[warp] = above;
-  __syncthreads();
-  const int ncand = sh.s_ncand;
-  const bool listed = ncand <= cand_cap;
+      for (int e = 0; e < VEC; ++e) c[e] = valid && (key[e] >> S1) >= b1;
+      topk_append<VEC>(j0, key, c, cand_bits, cand_idx, cand_cap, &sh.s_ncand);
+    });
+    __syncthreads();
+    listed = true;
+  }
+  const int ncand = listed ? sh.s_ncand : 0;
 
-  // ---- passes 3, 4: the second and third digits, over the candidates
+  // ---- passes 3, 4: the second and third digits, over the candidates (or the row)
   unsigned prefix = b1 << S1, mask = static_cast<unsigned>(NB1 - 1) << S1;
   for (int pass = 0; pass < 2; ++pass) {
     const int shift = pass == 0 ? D3 : 0;
@@ -231,7 +271,7 @@ __device__ void topk_row(const unsigned *row_g, int N, int k, unsigned *hist, un
         if ((x & mask) == prefix) atomicAdd(&hist[(x >> shift) & dm], 1u);
       }
     } else {
-      topk_walk<VEC>(src, cached, lo, hi, [&](int, const unsigned *key, bool valid) {
+      topk_walk<VEC>(row_g, lo, hi, [&](int, const unsigned *key, bool valid) {
         if (!valid) return;
 #pragma unroll
         for (int e = 0; e < VEC; ++e)
@@ -248,7 +288,41 @@ __device__ void topk_row(const unsigned *row_g, int N, int k, unsigned *hist, un
   const unsigned T = prefix;
   const int need_eq = kk;   // keys equal to T to keep: the first need_eq of them in index order
 
-  // ---- per-warp counts of keys above T and equal to T
+  // ---- keys equal to T: if all of them are kept, mark the selection in a bitmap
+  const int W = (N + 31) / 32;
+  if (listed) {
+    int q = 0;
+    for (int i = tid; i < ncand; i += NT) q += cand_bits[i] == T ? 1 : 0;
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) q += __shfl_xor_sync(0xffffffffu, q, o);
+    if (lane == 0 && q > 0) atomicAdd(&sh.s_eq, q);
+    __syncthreads();
+  }
+  if (listed && sh.s_eq == need_eq && W <= kTopkHistWords) {
+    for (int i = tid; i < ncand; i += NT)
+      if (cand_bits[i] >= T) atomicOr(&hist[cand_idx[i] >> 5], 1u << (cand_idx[i] & 31));
+    __syncthreads();
+    const int per = (W + NT - 1) / NT;
+    const int w0 = min(W, tid * per), w1 = min(W, w0 + per);
+    int cnt = 0;
+    for (int w = w0; w < w1; ++w) cnt += __popc(hist[w]);
+    int total;
+    int pos = topk_block_scan<NT>(cnt, sh.wsum, &total);
+    for (int w = w0; w < w1; ++w) {
+      unsigned bits = hist[w];
+      while (bits != 0u) {
+        const int b = __ffs(bits) - 1;
+        if (pos < k) out[pos] = w * 32 + b;
+        ++pos;
+        bits &= bits - 1u;
+      }
+    }
+    __syncthreads();   // every word read before the bitmap is cleared
+    for (int i = tid; i < W; i += NT) hist[i] = 0;
+    return b1;
+  }
+
+  // ---- otherwise per-warp counts of keys above T and equal to T
   if (listed) {
     for (int i = tid; i < ncand; i += NT) {
       const unsigned x = cand_bits[i];
@@ -258,11 +332,10 @@ __device__ void topk_row(const unsigned *row_g, int N, int k, unsigned *hist, un
     }
   } else {
     int g = 0, q = 0;
-    topk_walk<VEC>(src, cached, lo, hi, [&](int, const unsigned *key, bool valid) {
+    topk_walk<VEC>(row_g, lo, hi, [&](int, const unsigned *key, bool valid) {
       if (!valid) return;
 #pragma unroll
       for (int e = 0; e < VEC; ++e) {
-        if ((key[e] >> S1) != b1) continue;
         g += key[e] > T ? 1 : 0;
         q += key[e] == T ? 1 : 0;
       }
@@ -273,7 +346,7 @@ __device__ void topk_row(const unsigned *row_g, int N, int k, unsigned *hist, un
       q += __shfl_xor_sync(0xffffffffu, q, o);
     }
     if (lane == 0) {
-      sh.gt_cnt[warp] += g;
+      sh.gt_cnt[warp] = g;
       sh.eq_cnt[warp] = q;
     }
   }
@@ -299,10 +372,11 @@ __device__ void topk_row(const unsigned *row_g, int N, int k, unsigned *hist, un
   }
   __syncthreads();
 
-  // ---- pass 5: each warp writes its selected keys in index order
+  // ---- each warp writes its selected keys in index order
+  const unsigned lt = (1u << lane) - 1u;
   const int eq_take = sh.w_take[warp];
   int written = sh.w_base[warp], eq_seen = 0;
-  topk_walk<VEC>(src, cached, lo, hi, [&](int j0, const unsigned *key, bool valid) {
+  topk_walk<VEC>(row_g, lo, hi, [&](int j0, const unsigned *key, bool valid) {
     unsigned beq[VEC];
     int own_eq = 0;
 #pragma unroll
@@ -337,25 +411,30 @@ __device__ void topk_row(const unsigned *row_g, int N, int k, unsigned *hist, un
     }
     written += step_sel;
   });
+  return b1;
 }
 
-// One CTA per row of a read-only score matrix.  VEC = 4 needs N % 4 == 0 and
-// a 16-byte aligned score array.
+// Rows [r0, r1) of a read-only score matrix per CTA, a contiguous run so
+// that each row's guess comes from its neighbour.  VEC = 4 needs N % 4 == 0
+// and a 16-byte aligned score array.
 template <int VEC>
-__global__ void __launch_bounds__(kTopkThreads) topk_kernel(const float *__restrict__ colsum, int N, int k,
-                                                            int cache_row, int32_t *__restrict__ kv_idx) {
-  // dynamic shared memory: histogram, candidate list, then the row when cache_row
+__global__ void __launch_bounds__(kTopkThreads, kTopkCtasPerSm)
+    topk_kernel(const float *__restrict__ colsum, long long rows, int N, int k, int32_t *__restrict__ kv_idx) {
+  // dynamic shared memory: histogram (later the output bitmap), candidate list
   extern __shared__ __align__(16) unsigned topk_sm[];
   unsigned *hist = topk_sm;
-  unsigned *cand_bits = hist + 4096;
+  unsigned *cand_bits = hist + kTopkHistWords;
   int *cand_idx = reinterpret_cast<int *>(cand_bits + kTopkCandCap);
-  unsigned *row_sm = reinterpret_cast<unsigned *>(cand_idx + kTopkCandCap);
   __shared__ TopkShared sh;
-  const size_t row = blockIdx.x;
-  for (int i = threadIdx.x; i < 4096; i += kTopkThreads) hist[i] = 0;
-  topk_row<VEC, kTopkThreads, 12>(reinterpret_cast<const unsigned *>(colsum + row * N), N, k, hist,
-                                        cand_bits, cand_idx, kTopkCandCap, cache_row ? row_sm : nullptr, sh,
-                                        kv_idx + row * k);
+  for (int i = threadIdx.x; i < kTopkHistWords; i += kTopkThreads) hist[i] = 0;
+  const long long r0 = rows * blockIdx.x / gridDim.x, r1 = rows * (blockIdx.x + 1) / gridDim.x;
+  unsigned guess = 1u << 12;   // the first row lists nothing in pass 1
+  for (long long r = r0; r < r1; ++r) {
+    const unsigned b1 = topk_row<VEC, kTopkThreads, 12>(reinterpret_cast<const unsigned *>(colsum + r * N), N, k,
+                                                        hist, cand_bits, cand_idx, kTopkCandCap, guess, sh,
+                                                        kv_idx + r * k);
+    guess = b1 > kTopkGuessMargin ? b1 - kTopkGuessMargin : 0u;
+  }
 }
 
 }  // namespace mcs

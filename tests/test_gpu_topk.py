@@ -11,7 +11,13 @@ select_kv (ties to the lower key index, output ascending):
   * k = 1, k = N - 1 and k >= N;
   * many rows at once, repeatedly, whose candidates all need the second and
     third digits (a clear of one digit's histogram racing the next digit's
-    counts would lose counts in some row, some time).
+    counts would lose counts in some row, some time);
+  * long runs of rows per CTA, mixing rows alike their predecessor (the
+    first walk's guess of the threshold's first digit holds), rows whose
+    scale jumps by 2^10 either way (the guess misses: the keys are listed
+    again, or the first list overflows), rows with ties at the threshold and
+    constant rows;
+  * rows longer than the output bitmap (N > 131072).
 """
 import numpy as np
 import pytest
@@ -56,6 +62,8 @@ CASES = [
     ("few_values", 3, 1000, 999),
     ("lognormal", 2, 37, 64),           # k >= N: every key
     ("lognormal", 2, 1, 1),
+    ("lognormal", 3, 131076, 500),      # longer than the output bitmap
+    ("lognormal", 2, 262144, 20000),
 ]
 
 
@@ -80,6 +88,33 @@ def test_select_topk_many_rows_repeatably():
         got = mcs.select_topk(dev, k).cpu().numpy()
         bad = np.nonzero((got != ref).any(axis=1))[0]
         assert len(bad) == 0, f"repetition {rep}: {len(bad)} rows differ, first {bad[:5]}"
+
+
+def _mixed_rows(rng, rows, N):
+    s = rng.lognormal(-9.0, 2.0, size=(rows, N)).astype(np.float32)
+    kind = rng.integers(0, 12, size=rows)
+    for r in range(rows):
+        if kind[r] == 0:
+            s[r] *= np.float32(2.0 ** 10)
+        elif kind[r] == 1:
+            s[r] *= np.float32(2.0 ** -10)
+        elif kind[r] == 2:
+            s[r] = rng.choice(np.array([0.0, 1e-6, 2.5e-3, 0.125], np.float32), size=N, p=[0.4, 0.3, 0.25, 0.05])
+        elif kind[r] == 3:
+            s[r] = np.float32(3.0e-4)
+    return s, kind
+
+
+@pytest.mark.parametrize("rows,N,k", [(3000, 4096, 200), (1500, 32760, 1638), (700, 4099, 300)])
+def test_select_topk_runs_of_mixed_rows(rows, N, k):
+    """More rows than CTAs, so each CTA walks a run of rows and guesses each
+    row's threshold digit from the row before; every row index-exact."""
+    rng = np.random.default_rng(rows + N + k)
+    s, kind = _mixed_rows(rng, rows, N)
+    assert rows > 3 * 148 and len(set(kind.tolist())) == 12
+    got = mcs.select_topk(torch.from_numpy(s).cuda(), k).cpu().numpy()
+    bad = [r for r in range(rows) if not np.array_equal(got[r], orc.select_kv(s[r].astype(np.float64), k))]
+    assert not bad, f"{len(bad)} rows differ, first {bad[:5]} (kinds {[int(kind[r]) for r in bad[:5]]})"
 
 
 def test_select_topk_batched_shape_and_empty():
