@@ -8,21 +8,22 @@
 // Non-negative IEEE floats order like their bit patterns as uint32, so the
 // k-th largest value T is found by a most-significant-digit radix select over
 // the 31 magnitude bits in three digits (D1 bits, then the rest in two).  The
-// first digit is counted over the whole row in one walk that reads the row
-// from HBM; the keys whose first digit is at least b1 (the threshold's) go to
-// a shared memory candidate list, and the two remaining digits are resolved
-// on that list alone.  Every key with bits > T and the first (k - #greater)
-// keys with bits == T are kept, written ascending.
+// keys whose first digit is at least b1 (the threshold's) go to a shared
+// memory candidate list, and the digits are resolved on that list alone.
+// Every key with bits > T and the first (k - #greater) keys with bits == T
+// are kept, written ascending.
 //
-// b1 is known only once the walk is over, so the walk lists the keys whose
-// first digit is at least a guess: the previous row's b1 less one bin.  A CTA
-// takes a contiguous run of rows, i.e. adjacent query groups of one head,
-// whose score rows are alike (on the 32K-token video layer b1 moves by at
-// most one of 4096 bins between adjacent groups).  After the walk the
-// histogram says exactly whether the guess held (b1 >= guess, no overflow);
-// if not, a second walk (from L2) lists the keys with first digit >= b1, and
-// if even those overflow the list (a near-constant row, a large k) the
-// remaining digits are resolved by walks over the whole row.
+// A CTA takes a contiguous run of rows, i.e. adjacent query groups of one
+// head, whose score rows are alike (on the 32K-token video layer b1 moves by
+// at most one of 4096 bins between adjacent groups).  So the walk that reads
+// a row from HBM only lists the keys whose first digit is at least a guess,
+// the previous row's b1 less one bin, with no per-key histogram.  If at least
+// k keys were listed (and the list did not overflow), the k-th largest key
+// and every key above it are on the list, and all three digits are resolved
+// there.  Otherwise (the run's first row, or a miss) the first digit is
+// counted over the whole row, a further walk lists the keys with first digit
+// >= b1, and if even those overflow the list (a near-constant row, a large k)
+// the remaining digits are resolved by walks over the whole row.
 //
 // Output: when no key equal to T has to be dropped, the selected keys are
 // marked in a bitmap of the row (in the histogram's memory, N <= 131072), and
@@ -35,7 +36,11 @@
 //
 // topk_row is that selection for one row by one CTA of NT threads;
 // topk_kernel runs it with 512-thread CTAs, three per SM (64 KB of shared
-// memory each), each over a contiguous run of rows.
+// memory each), each over a contiguous run of rows.  On the 32K-token video
+// layer (6144 rows of 32,760 scores) DRAM runs at about a quarter of its peak
+// while the SMs issue about 2.8 instructions per cycle of 4: the pace is set
+// by each row's chain of walk and barrier-separated candidate phases, of
+// which three CTAs per SM overlap only three.
 #pragma once
 
 #include "mcs_common.cuh"
@@ -158,33 +163,73 @@ __device__ __forceinline__ void topk_walk(const unsigned *src, int lo, int hi, F
   }
 }
 
-// Append the keys with c[e] set (key[e] at index j0 + e) to the candidate
-// list, one shared-memory atomic per warp and step; entries past cap are
-// counted but not stored.  Called by every lane of the warp.
+// List the keys of this warp's slice [lo, hi) whose magnitude bits are >= thr
+// (bits and index) on the candidate list; entries past cap are counted but
+// not stored.  Per lane, 4 steps of VEC keys are loaded at once; the lane
+// counts its candidates among them, and one warp scan of those counts plus
+// one shared-memory atomic per warp give every lane its list positions (the
+// list's order is free: the selection is sorted by the output bitmap or by
+// the per-warp walk).
 template <int VEC>
-__device__ __forceinline__ void topk_append(int j0, const unsigned *key, const bool *c, unsigned *cand_bits,
-                                            int *cand_idx, int cap, int *ncand) {
+__device__ __forceinline__ void topk_list_walk(const unsigned *src, int lo, int hi, unsigned thr, unsigned *cand_bits,
+                                               int *cand_idx, int cap, int *ncand) {
+  constexpr int STEP = 32 * VEC;
   const int lane = threadIdx.x & 31;
-  const unsigned lt = (1u << lane) - 1u;
-  unsigned bal[VEC];
-  int n = 0;
+  for (int b = lo; b < hi; b += 4 * STEP) {
+    unsigned x[4][VEC];
 #pragma unroll
-  for (int e = 0; e < VEC; ++e) {
-    bal[e] = __ballot_sync(0xffffffffu, c[e]);
-    n += __popc(bal[e]);
-  }
-  if (n == 0) return;   // warp-uniform
-  int base = 0;
-  if (lane == 0) base = atomicAdd(ncand, n);
-  base = __shfl_sync(0xffffffffu, base, 0);
+    for (int u = 0; u < 4; ++u) {
+      const int j0 = b + u * STEP + VEC * lane;
+      if (j0 < hi) {
+        if constexpr (VEC == 4) {
+          const uint4 v = __ldg(reinterpret_cast<const uint4 *>(src + j0));
+          x[u][0] = v.x;
+          x[u][1] = v.y;
+          x[u][2] = v.z;
+          x[u][3] = v.w;
+        } else {
+          x[u][0] = __ldg(src + j0);
+        }
+      } else {
 #pragma unroll
-  for (int e = 0; e < VEC; ++e) {
-    const int pos = base + __popc(bal[e] & lt);
-    if (c[e] && pos < cap) {
-      cand_bits[pos] = key[e];
-      cand_idx[pos] = j0 + e;
+        for (int e = 0; e < VEC; ++e) x[u][e] = 0u;
+      }
     }
-    base += __popc(bal[e]);
+    // sel bit (u * VEC + e): key x[u][e] is in the slice and listed
+    unsigned sel = 0u;
+#pragma unroll
+    for (int u = 0; u < 4; ++u)
+#pragma unroll
+      for (int e = 0; e < VEC; ++e) {
+        x[u][e] &= kTopkMagnitude;
+        const bool in = b + u * STEP + VEC * lane + e < hi;
+        sel |= (in && x[u][e] >= thr) ? 1u << (u * VEC + e) : 0u;
+      }
+    const int m = __popc(sel);
+    int incl = m;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int y = __shfl_up_sync(0xffffffffu, incl, o);
+      if (lane >= o) incl += y;
+    }
+    const int total = __shfl_sync(0xffffffffu, incl, 31);
+    if (total > 0) {   // warp-uniform
+      int base = 0;
+      if (lane == 31) base = atomicAdd(ncand, total);
+      int pos = __shfl_sync(0xffffffffu, base, 31) + incl - m;
+#pragma unroll
+      for (int u = 0; u < 4; ++u)
+#pragma unroll
+        for (int e = 0; e < VEC; ++e) {
+          if ((sel >> (u * VEC + e)) & 1u) {
+            if (pos < cap) {
+              cand_bits[pos] = x[u][e];
+              cand_idx[pos] = b + u * STEP + VEC * lane + e;
+            }
+            ++pos;
+          }
+        }
+    }
   }
 }
 
@@ -193,9 +238,10 @@ __device__ __forceinline__ void topk_append(int j0, const unsigned *key, const b
 // (all of them call it; it synchronises the block).  row_g is read-only for
 // the whole kernel.  hist: kTopkHistWords zeroed words (left zeroed on
 // return).  cand_bits / cand_idx: cand_cap entries each.  guess: pass 1 lists
-// the keys whose first digit is >= guess (1 << D1 lists none).  Returns the
-// first digit of the row's threshold (the next row's guess is derived from
-// it), or 1 << D1 when every key is kept.
+// the keys whose first digit is >= guess (1 << D1 or more: no guess, the
+// first digit is counted over the row).  Returns the first digit of the
+// row's threshold (the next row's guess is derived from it), or 1 << D1 when
+// every key is kept.
 template <int VEC, int NT, int D1>
 __device__ unsigned topk_row(const unsigned *row_g, int N, int k, unsigned *hist, unsigned *cand_bits, int *cand_idx,
                              int cand_cap, unsigned guess, TopkShared &sh, int32_t *out) {
@@ -222,40 +268,47 @@ __device__ unsigned topk_row(const unsigned *row_g, int N, int k, unsigned *hist
   }
   __syncthreads();
 
-  // ---- pass 1 (HBM): count the first digit; list the keys whose first digit is >= guess
-  topk_walk<VEC>(row_g, lo, hi, [&](int j0, const unsigned *key, bool valid) {
-    bool c[VEC];
-#pragma unroll
-    for (int e = 0; e < VEC; ++e) {
-      const unsigned d = key[e] >> S1;
-      if (valid) atomicAdd(&hist[d], 1u);
-      c[e] = valid && d >= guess;
-    }
-    topk_append<VEC>(j0, key, c, cand_bits, cand_idx, cand_cap, &sh.s_ncand);
-  });
-  __syncthreads();
   int kk = k;
-  const unsigned b1 = topk_select_bin<NT>(hist, NB1, kk, sh);
-  const int in_bin = static_cast<int>(hist[b1]);
-  const int n_above = k - kk;               // keys whose first digit is above b1
-  const int n_first = sh.s_ncand;
-  __syncthreads();                          // every thread has read them
-  for (int i = tid; i < NB1; i += NT) hist[i] = 0;
-  bool listed = b1 >= guess && n_first <= cand_cap;
-  const bool relist = !listed && n_above + in_bin <= cand_cap;
-  if (relist && tid == 0) sh.s_ncand = 0;
-  __syncthreads();                          // histogram clear and list reset seen by all
-
-  // ---- pass 2 (L2), only when the guess missed: list the keys whose first digit is >= b1
-  if (relist) {
-    topk_walk<VEC>(row_g, lo, hi, [&](int j0, const unsigned *key, bool valid) {
-      bool c[VEC];
+  unsigned b1 = 0;
+  bool listed = false;
+  if (guess < static_cast<unsigned>(NB1)) {
+    // ---- pass 1 (HBM): list the keys whose first digit is >= guess
+    topk_list_walk<VEC>(row_g, lo, hi, guess << S1, cand_bits, cand_idx, cand_cap, &sh.s_ncand);
+    __syncthreads();
+    const int n1 = sh.s_ncand;
+    // at least k keys listed: the k-th largest is among them, and so is every
+    // key at or above it; the first digit is then counted over the list alone
+    listed = n1 >= k && n1 <= cand_cap;
+    if (listed) {
+      for (int i = tid; i < n1; i += NT) atomicAdd(&hist[cand_bits[i] >> S1], 1u);
+      __syncthreads();
+      b1 = topk_select_bin<NT>(hist, NB1, kk, sh);
+      for (int i = static_cast<int>(guess) + tid; i < NB1; i += NT) hist[i] = 0;
+      __syncthreads();
+    }
+  }
+  if (!listed) {
+    // ---- no guess, or it missed: count the first digit over the row (from
+    // HBM, or from L2 after a pass 1), then list the keys with first digit >= b1
+    topk_walk<VEC>(row_g, lo, hi, [&](int, const unsigned *key, bool valid) {
+      if (!valid) return;
 #pragma unroll
-      for (int e = 0; e < VEC; ++e) c[e] = valid && (key[e] >> S1) >= b1;
-      topk_append<VEC>(j0, key, c, cand_bits, cand_idx, cand_cap, &sh.s_ncand);
+      for (int e = 0; e < VEC; ++e) atomicAdd(&hist[key[e] >> S1], 1u);
     });
     __syncthreads();
-    listed = true;
+    b1 = topk_select_bin<NT>(hist, NB1, kk, sh);
+    const int in_bin = static_cast<int>(hist[b1]);
+    const int n_above = k - kk;             // keys whose first digit is above b1
+    __syncthreads();                        // every thread has read hist[b1]
+    for (int i = tid; i < NB1; i += NT) hist[i] = 0;
+    const bool relist = n_above + in_bin <= cand_cap;
+    if (relist && tid == 0) sh.s_ncand = 0;
+    __syncthreads();                        // histogram clear and list reset seen by all
+    if (relist) {
+      topk_list_walk<VEC>(row_g, lo, hi, b1 << S1, cand_bits, cand_idx, cand_cap, &sh.s_ncand);
+      __syncthreads();
+      listed = true;
+    }
   }
   const int ncand = listed ? sh.s_ncand : 0;
 
