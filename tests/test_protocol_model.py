@@ -29,7 +29,11 @@ phases across items; the Q buffer is refilled for the next item once the
 current item's last Q.K^T has executed (a "Q empty" barrier), and the next
 item's first P.V, which overwrites O, must not run before the epilogue has
 read it.  The third is the group-score kernel (colsum_kernel.cuh), whose
-reducing warps hand each S buffer back to the MMA thread explicitly.
+reducing warps hand each S buffer back to the MMA thread explicitly.  The
+fourth is one K/V ring fed by several producer warps, as in the sparse
+kernels: it holds while each warp's copies carry part of every phase's
+transaction bytes, and a variant in which one warp's plain arrival completes
+each phase leaves the other warps waiting on phases that never come.
 """
 import random
 
@@ -592,3 +596,114 @@ def test_colsum_model_catches_planted_defects(defect):
             failures += 1
     assert failures > 0
 
+
+
+# ---------------------------------------------------------------------------
+# one K/V ring fed by several producer warps (pair_kernel.cuh, attn_kernel.cuh)
+# ---------------------------------------------------------------------------
+#
+# Every producer warp waits on a slot's empty barrier before issuing its share
+# of the tile's gather4 copies; warp 0 alone makes the phase's one arrival,
+# with the tile's transaction bytes.  Because each warp's copies carry part of
+# those bytes, a slot's full phase, and so its next empty phase, cannot
+# complete before every warp has passed its own wait: no warp falls two
+# phases behind, where a parity wait would mistake a later phase for the one
+# it waits on.  A producer scheme in which warp 0 completes each phase on its
+# own (a plain arrival, the other warps issuing nothing) loses that coupling.
+
+class Ring:
+    def __init__(self, T, NS, W, coupled):
+        self.T, self.NS, self.W, self.coupled = T, NS, W, coupled
+        self.full = [Barrier(1) for _ in range(NS)]
+        self.empty = [Barrier(1) for _ in range(NS)]
+        self.landed = {}                   # tile -> copies landed
+        self.arrived = set()               # tiles whose phase arrival warp 0 made
+        self.consumed = set()
+        self.copies = []                   # (slot, tile) in flight
+
+    def step_copy(self, i):
+        s, j = self.copies.pop(i)
+        self.landed[j] = self.landed.get(j, 0) + 1
+        self.full[s].complete_tx(1)
+
+
+def ring_producer(R, w):
+    yield from ()
+    for j in range(R.T):
+        s = j % R.NS
+        t = j - R.NS
+        yield wait(R.empty[s], ((j // R.NS) & 1) ^ 1, lambda t=t: t < 0 or t in R.consumed,
+                   f"warp {w}: slot of tile {t} free")
+        if w == 0:
+            R.arrived.add(j)
+            if R.coupled:
+                R.full[s].arrive_expect_tx(R.W)
+            else:
+                R.full[s].arrive()
+        if R.coupled:
+            R.copies.append((s, j))
+
+
+def ring_consumer(R):
+    for j in range(R.T):
+        s = j % R.NS
+        ready = (lambda j=j: j in R.arrived and R.landed.get(j, 0) == R.W) if R.coupled else (lambda j=j: j in R.arrived)
+        yield wait(R.full[s], (j // R.NS) & 1, ready, f"tile {j} in its slot")
+        R.consumed.add(j)
+        R.empty[s].arrive()
+
+
+def run_ring(T, NS, W, coupled, seed, max_steps=200000):
+    rng = random.Random(seed)
+    R = Ring(T, NS, W, coupled)
+    actors = {f"w{w}": ring_producer(R, w) for w in range(W)}
+    actors["mma"] = ring_consumer(R)
+    blocked = {name: None for name in actors}
+    finished = set()
+
+    def advance(name):
+        try:
+            blocked[name] = next(actors[name])
+        except StopIteration:
+            finished.add(name)
+            blocked[name] = None
+
+    for name in list(actors):
+        advance(name)
+    for _ in range(max_steps):
+        if len(finished) == len(actors):
+            return R
+        moves = [("actor", n) for n, w in blocked.items()
+                 if n not in finished and w is not None and w[0].parity_done(w[1])]
+        moves += [("copy", i) for i in range(len(R.copies))]
+        if not moves:
+            raise ProtocolError(f"deadlock: waiting {[(n, w[3]) for n, w in blocked.items() if n not in finished]}")
+        kind, arg = rng.choice(moves)
+        if kind == "copy":
+            R.step_copy(arg)
+        else:
+            w = blocked[arg]
+            check(w[2](), f"{arg}: wait for '{w[3]}' returned before it happened")
+            advance(arg)
+    raise ProtocolError("schedule did not finish")
+
+
+@pytest.mark.parametrize("NS", [2, 5])
+@pytest.mark.parametrize("W", [3, 4])
+def test_ring_producer_warps_coupled_by_transaction_bytes(NS, W):
+    for seed in range(150):
+        R = run_ring(12, NS, W, True, seed)
+        assert R.consumed == set(range(12))
+
+
+def test_ring_producer_warps_without_bytes_can_wait_forever():
+    """warp 0's plain arrival alone completes each phase: some schedule
+    leaves another producer warp waiting on a phase that never comes."""
+    failures = 0
+    for seed in range(300):
+        try:
+            run_ring(12, 2, 4, False, seed)
+        except ProtocolError as e:
+            assert "deadlock" in str(e)
+            failures += 1
+    assert failures > 0
