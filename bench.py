@@ -922,6 +922,20 @@ def main():
         "bytes_per_launch": gathered, "gbs": gathered / t_step / 1e9,
         "ceiling_gbs": gather_ceiling, "ceiling": "TMA tile::gather4 from 7 warps per SM (measured)",
         "frac_of_ceiling": gathered / t_step / 1e9 / gather_ceiling if gather_ceiling else None}
+    # its exponential side: one ex2 per kept (query, key) pair, against the MUFU
+    # rate (16 per SM per cycle, measured by the committed microbenchmark) at
+    # the median SM clock sampled over the timed steps
+    try:
+        mhz = clk.get("sm_mhz") if isinstance(clk, dict) else None
+        if mhz:
+            n_exp = float(BH) * N * kk
+            ex2_rate = 16.0 * torch.cuda.get_device_properties(dev).multi_processor_count * mhz * 1e6
+            kernels["step"]["exp"] = {
+                "count_per_launch": n_exp, "per_s": n_exp / t_step, "ceiling_per_s": ex2_rate,
+                "ceiling": "MUFU ex2, 16 per SM per cycle (measured) at the median SM clock",
+                "frac_of_ceiling": n_exp / t_step / ex2_rate}
+    except Exception:   # a missing clock sample or device property leaves the term out
+        pass
 
     def roof(s):
         r = kernels[s]
